@@ -1,0 +1,500 @@
+"""Benchmark: one layer's paged-KV attention step on synthetic, seeded inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is the whole hot path for one batch: slot mapping of the new tokens,
+the cache write (reshape_and_cache) and the attention call (pa_decode for
+decode batches, pa_mixed_step for a chunked-prefill step).  Inputs are
+resident in HBM when timing starts; L2 is flushed (a 512 MiB write) before
+every step and only the step itself sits between its CUDA events.  With
+torchrun (N > 1) every rank runs its own batch on its own GPU (sequences are
+independent: weak scaling, no collective on the data path); the time is the
+max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (float64 NumPy, the test reference) on
+a bounded sample of the same workload, on this host's cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    "tiny": ("tiny_decode", 1),
+    "llama8b_decode": ("llama8b_decode", 2),
+    "long_context": ("long_context_decode", 3),
+    "mixed": ("mixed_step", 4),
+    "shared_prefix": ("shared_prefix_decode", 5),
+}
+FLUSH_BYTES = 512 << 20
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="llama8b_decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="time budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_traffic(kernel_src: str, profile_md: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel source (the summary records the source's sha256)."""
+    path = os.path.join(ROOT, "profiles", profile_md)
+    src = os.path.join(ROOT, "paged_kv_cache_434_b200", "csrc", kernel_src)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(path, encoding="utf-8"):
+        if ":" in line and line.strip().startswith(("kernel_source_sha256", "traffic_bytes_per_launch")):
+            k, v = line.split(":", 1)
+            vals[k.strip().lstrip("- ").strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256") != sha:
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+        except Exception:
+            uuid = None
+        self.target = uuid
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.target:
+            cmd += ["-i", self.target]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- workload accounting
+
+def workload_for(name: str, seed: int):
+    from paged_kv_cache_434_b200 import workloads as W
+    return getattr(W, WORKLOADS[name][0])(seed)
+
+
+def byte_counts(w, out_elt=4):
+    """Algorithmic bytes of one step (unique valid K/V rows once,
+    Q read, O written; the cache write reads and writes each new K/V row)."""
+    from paged_kv_cache_434_b200 import workloads as W
+    kv = W.kv_bytes_touched(w, unique=True)
+    q = w.num_tokens * w.num_heads * w.head_dim * w.elt_bytes
+    o = w.num_tokens * w.num_heads * w.head_dim * out_elt
+    cw = 2 * 2 * w.num_tokens * w.num_kv_heads * w.head_dim * w.elt_bytes
+    return {"kv": kv, "q": q, "o": o, "cache_write": cw, "attention": kv + q + o,
+            "step": kv + q + o + cw}
+
+
+def prefill_flops(w):
+    """Causal-only FLOPs (QK^T and PV, 2 each per MAC) of the q_b > 1 requests."""
+    tot = 0
+    for b in range(w.num_seqs):
+        qb, L = int(w.query_lens[b]), int(w.seq_lens[b])
+        if qb > 1:
+            keys = sum(L - qb + i + 1 for i in range(qb))
+            tot += 4 * w.head_dim * w.num_heads * keys
+    return tot
+
+
+def metric_of(name):
+    if name == "mixed":
+        return "mixed-step query tokens/s per layer", "tokens/s"
+    return "paged decode KV GB/s", "GB/s"
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample(w, pools, seconds: float, rng_seed: int = 0):
+    """Time the oracle on whole rows of the workload until `seconds` pass.
+
+    Returns (units_done, elapsed_s, description) where units are KV bytes
+    (decode workloads) or query rows (mixed step).
+    """
+    import oracle
+    from threadpoolctl import threadpool_limits
+    k_cache, v_cache = pools
+    rng = np.random.default_rng(rng_seed)
+    qsl = w.query_start_loc
+    rows = []
+    if w.is_decode:
+        order = rng.permutation(w.num_seqs)
+        rows = [(int(b), 0) for b in order]
+    else:
+        dec = [b for b in range(w.num_seqs) if w.query_lens[b] == 1]
+        pre = [(b, i) for b in range(w.num_seqs) if w.query_lens[b] > 1
+               for i in range(int(w.query_lens[b]))]
+        rng.shuffle(dec)
+        pi = rng.permutation(len(pre))
+        # same mix of prefill and decode rows as the step
+        for a, b in zip(pi, dec):
+            rows.append(pre[a])
+            rows.append((b, 0))
+    row_kv = 2 * w.num_kv_heads * w.head_dim * w.elt_bytes
+    # fetch the blocks for up to a generous number of rows first (not timed)
+    prepared = []
+    cache = {}
+    for (b, i) in rows[:4096]:
+        if b not in cache:
+            n = (int(w.seq_lens[b]) + w.block_size - 1) // w.block_size
+            ids = torch.from_numpy(w.block_tables[b, :n].astype(np.int64)).to(k_cache.device)
+            cache[b] = (k_cache.index_select(0, ids).cpu(), v_cache.index_select(0, ids).cpu())
+            if len(cache) > 256:
+                break
+        prepared.append((b, i))
+    q = torch.randn(1, w.num_heads, w.head_dim).to(torch.bfloat16 if w.dtype == "bf16"
+                                                     else torch.float32)
+    threads = os.cpu_count() or 1
+    done_units, t0 = 0, time.perf_counter()
+    with threadpool_limits(limits=threads):
+        for (b, i) in prepared:
+            if b not in cache:
+                break
+            kb, vb = cache[b]
+            L, qb = int(w.seq_lens[b]), int(w.query_lens[b])
+            pos = L - qb + i
+            table = np.arange(kb.shape[0])
+            K = oracle.gather(kb.to(torch.float64).numpy(), table, pos + 1)
+            V = oracle.gather(vb.to(torch.float64).numpy(), table, pos + 1)
+            oracle.attend_two_pass(q.to(torch.float64).numpy(), K, V, w.scale, pos)
+            done_units += (pos + 1) * row_kv if w.is_decode else 1
+            if time.perf_counter() - t0 > seconds:
+                break
+    el = time.perf_counter() - t0
+    desc = (f"{'requests' if w.is_decode else 'query rows'} of {w.name} drawn at random, "
+            f"oracle float64 gather + two-pass softmax, {el:.1f} s wall")
+    return done_units, el, desc, threads
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local):
+    import paged_kv_cache_434_b200 as P
+    from paged_kv_cache_434_b200 import workloads as W
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = workload_for(args.workload, args.seed + rank)
+    t = W.make_tensors(w, dev)
+    idx = W.index_tensors(w, dev)
+    T = w.num_tokens
+    decode_only = w.is_decode
+    out = torch.empty(T, w.num_heads, w.head_dim, dtype=torch.float32, device=dev)
+    slots = torch.empty(T, dtype=torch.int64, device=dev)
+    err = P.new_error_word(dev)
+    ws_bytes = (P.decode_workspace_size(w.num_seqs, w.num_heads, w.max_blocks_per_seq,
+                                        t["k_cache"]) if decode_only else
+                P.mixed_step_workspace_size(w.num_seqs, T, w.num_heads, w.max_blocks_per_seq,
+                                            t["k_cache"]))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        P.slot_mapping(idx["block_tables"], idx["query_start_loc"], idx["seq_lens"],
+                       w.block_size, w.num_blocks, T, out=slots, err=err)
+        P.cache_write(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], slots, err=err)
+        mid.record(stream)
+        if decode_only:
+            P.decode(t["q"], t["k_cache"], t["v_cache"], idx["block_tables"], idx["seq_lens"],
+                     w.scale, out=out, workspace=ws, err=err)
+        else:
+            P.mixed_step(t["q"], t["k_cache"], t["v_cache"], idx["block_tables"],
+                         idx["query_start_loc"], idx["seq_lens"], w.scale, out=out,
+                         workspace=ws, err=err)
+
+    mid = torch.cuda.Event(enable_timing=True)
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    if P.read_error(err) != 0:
+        raise RuntimeError("device error bits set during warm-up")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(dev) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    wall0 = time.perf_counter()
+    for (e0, e1, e2) in evs:
+        flush.fill_(1)
+        e0.record(stream)
+        mid = e1
+        step()
+        e2.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop() if clocks else None
+    step_ms = [e0.elapsed_time(e2) for (e0, _, e2) in evs]
+    attn_ms = [e1.elapsed_time(e2) for (_, e1, e2) in evs]
+    total_s = sum(step_ms) / 1e3
+    total_s = max_over_ranks(total_s, world, dev)
+    if P.read_error(err) != 0:
+        raise RuntimeError("device error bits set during the timed steps")
+
+    bc = byte_counts(w)
+    metric, unit = metric_of(args.workload)
+    if args.workload == "mixed":
+        value = T * args.steps * world / total_s
+    else:
+        value = bc["step"] * args.steps * world / total_s / 1e9
+    peaks = load_peaks()
+    attn_s = statistics.mean(attn_ms) / 1e3
+    achieved = bc["attention"] / attn_s / 1e9
+    dominant = "attn_mma_kernel" if w.dtype == "bf16" else "attn_generic_kernel"
+    src = "attn_mma.cu" if w.dtype == "bf16" else "attn_common.cu"
+    roofline = {"bound": "hbm", "kernel": dominant,
+                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)",
+                "timed_over": "the whole attention call (plan + attention + merge launches)",
+                "traffic": kernel_traffic(src, f"{dominant}_{args.workload}.md"),
+                "algorithmic_bytes_per_launch": bc["attention"]}
+    extra = {}
+    if args.workload == "mixed":
+        fl = prefill_flops(w)
+        extra["prefill_flops_per_step"] = fl
+
+    # ---- end to end: host buffers in, result back to the host, each step
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "k_new", "v_new"]
+        host = {n: t[n].cpu().pin_memory() for n in names}
+        host_idx = {n: idx[n].cpu().pin_memory() for n in ("block_tables", "seq_lens",
+                                                            "query_start_loc")}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in list(host.values()) +
+                  list(host_idx.values()))
+        d2h = out_h.numel() * out_h.element_size()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for (a, b) in ev2:
+            flush.fill_(1)
+            a.record(stream)
+            for n in names:
+                t[n].copy_(host[n], non_blocking=True)
+            for n, x in host_idx.items():
+                idx[n].copy_(x, non_blocking=True)
+            mid = torch.cuda.Event(enable_timing=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / 1e3, world, dev)
+        e2e_val = (T * args.steps * world / e2e_s if args.workload == "mixed"
+                   else bc["step"] * args.steps * world / e2e_s / 1e9)
+        e2e = {"value": round(e2e_val, 2), "unit": unit, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_s * 1e3 / args.steps, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        units, el, desc, threads = oracle_sample(w, (t["k_cache"], t["v_cache"]),
+                                                 args.cpu_seconds)
+        v = units / el / (1 if args.workload == "mixed" else 1e9)
+        cpu = {"value": round(v, 4), "unit": unit, "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": round(total_s * 1e3 / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype,
+            "data": "synthetic: seeded N(0,1) Q/K/V rounded to the dtype, seeded lengths and "
+                    "randomly permuted physical blocks",
+            "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_tokens": T,
+                       "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+                       "head_dim": w.head_dim, "block_size": w.block_size,
+                       "num_blocks": w.num_blocks,
+                       "kv_bytes_unique": bc["kv"], "step_bytes": bc["step"],
+                       "l2": "flushed before every step (512 MiB write, outside the events)",
+                       "parallelism": f"replicas x{world} (independent batches per GPU)",
+                       **extra},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 5 * args.steps,
+            "clocks": clk,
+            "wall_s_timed_region": round(wall, 3),
+        }
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world, local):
+    """The CPU oracle timed as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    import paged_kv_cache_434_b200.workloads as W
+    w = workload_for(args.workload, args.seed)
+    metric, unit = metric_of(args.workload)
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    pools = None
+    if dev.type == "cuda":
+        t = W.make_tensors(w, dev)
+        pools = (t["k_cache"], t["v_cache"])
+    else:
+        t = W.make_tensors(w, "cpu", where="host")
+        pools = (t["k_cache"], t["v_cache"])
+    per_step = max(0.5, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    desc = threads = None
+    for k in range(max(args.warmup, 3) + args.steps):
+        units, el, desc, threads = oracle_sample(w, pools, per_step, rng_seed=k)
+        if k >= max(args.warmup, 3):
+            vals.append((units, el))
+    units = sum(u for u, _ in vals)
+    el = sum(e for _, e in vals)
+    value = units / el / (1 if args.workload == "mixed" else 1e9)
+    line = {
+        "impl": "reference", "metric": metric, "value": round(value, 4), "unit": unit,
+        "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(el * 1e3 / max(1, args.steps), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same generator and seed as our arm)",
+        "config": {"workload": w.name},
+        "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": threads,
+                         "kind": "oracle", "sample": f"each step: {desc}"},
+        "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world, local)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

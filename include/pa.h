@@ -1,0 +1,177 @@
+/*
+ * pa.h -- C ABI of the paged-KV attention library (libpa_b200.so, sm_100a).
+ *
+ * Operations (names after the vLLM v1 walkthrough "AI Infra入门干货总结：大模型
+ * 是如何高效推理的"):
+ *   pa_slot_mapping   slot of every new token from the block tables
+ *                     ("Paged Attention": slot = block_idx * block_size + offset,
+ *                     worked example: block_size 16, table [5,8,12], pos 25 -> 137)
+ *   pa_cache_write    reshape_and_cache: scatter each new token's K/V row to
+ *                     its slot ("Reshape & Cache"; "Paged Attention")
+ *   pa_decode         GQA decode attention over the paged cache, FlashAttention
+ *                     online softmax, split-KV partitions merged by log-sum-exp
+ *                     ("Attention (FlashAttention, Scaled Dot-Product Attention)";
+ *                     "总结": Flash-Decoding re-normalises with log-sum-exp)
+ *   pa_mixed_step     causal varlen attention of a flattened continuous-batching
+ *                     step mixing chunked-prefill tokens and decode tokens, every
+ *                     K/V read through the block table (same section: the v1
+ *                     unified varlen call over the paged cache)
+ *
+ * Conventions shared by every call
+ *   - All tensor arguments are DEVICE pointers of the current CUDA device,
+ *     row-major and densely packed, owned by the caller.  The library never
+ *     allocates, frees or retains them, and keeps no state between calls
+ *     other than a per-device cache of launch attributes.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     is asynchronous: it validates on the host, enqueues kernels on `stream`
+ *     and returns.  Host-detectable errors return a non-zero pa_status and
+ *     enqueue nothing.
+ *   - Cache pools: key_cache and value_cache are each
+ *     [num_blocks, block_size, num_kv_heads, head_dim] (one layer), dtype
+ *     cache->dtype.
+ *   - Index arrays are int32 (block_tables, seq_lens, query_start_loc) except
+ *     slot_mapping (int64, as in the page's reshape_and_cache code).
+ *   - Device-detected errors never trap: the offending item is skipped and a
+ *     PA_ERRBIT_* bit is OR-ed into *err_word (an int32 in device memory;
+ *     may be NULL to discard).  pa_read_error() collects it.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, inconsistent shapes        */
+  PA_ERR_UNSUPPORTED = 2,  /* valid but unsupported (dtype, head_dim, ...)       */
+  PA_ERR_WORKSPACE = 3,    /* workspace pointer NULL or smaller than required    */
+  PA_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute ...) */
+  PA_ERR_DEVICE = 5        /* pa_read_error found device error bits set          */
+} pa_status;
+
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Device error bits (OR-ed into *err_word). */
+#define PA_ERRBIT_SLOT_OOB 0x1        /* slot >= num_blocks * block_size           */
+#define PA_ERRBIT_BLOCK_OOB 0x2       /* a needed block_tables entry not in [0,NB) */
+#define PA_ERRBIT_SEQ_TOO_LONG 0x4    /* seq_len > max_blocks_per_seq * block_size */
+#define PA_ERRBIT_QUERY_TOO_LONG 0x8  /* query_len > seq_len (or negative)         */
+#define PA_ERRBIT_TIMEOUT 0x10        /* a bounded device wait gave up             */
+
+/* One layer's cache pools. */
+typedef struct pa_cache_desc {
+  int64_t num_blocks;    /* physical blocks in each pool                 */
+  int32_t block_size;    /* tokens per block: 8, 16, 32, 64, 128 or 256  */
+  int32_t num_kv_heads;  /* >= 1                                        */
+  int32_t head_dim;      /* 64 or 128                                   */
+  int32_t dtype;         /* pa_dtype of pools, q, k and v               */
+} pa_cache_desc;
+
+/* Static description of a status code; never NULL. */
+const char* pa_status_str(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int pa_version(void);
+
+/*
+ * pa_slot_mapping -- slot of every new token of a flattened step.
+ * Request b owns flattened tokens query_start_loc[b] .. query_start_loc[b+1]-1;
+ * its q_b new tokens are its last q_b positions, token i at position
+ * p = seq_lens[b] - q_b + i, and
+ *     slot = block_tables[b][p / block_size] * block_size + p % block_size.
+ *   block_tables    int32 [num_seqs, max_blocks_per_seq]
+ *   query_start_loc int32 [num_seqs + 1], non-decreasing, [num_seqs] == num_tokens
+ *   seq_lens        int32 [num_seqs]
+ *   slot_mapping    int64 [num_tokens] (output)
+ * Tokens of a request whose q_b > seq_len or seq_len > max_blocks_per_seq *
+ * block_size, or whose table entry is outside [0, num_blocks), get slot -1
+ * and set the matching error bit.
+ */
+pa_status pa_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                          const int32_t* query_start_loc, const int32_t* seq_lens,
+                          int32_t num_seqs, int64_t num_tokens, int32_t block_size,
+                          int64_t num_blocks, int64_t* slot_mapping, int32_t* err_word,
+                          void* stream);
+
+/*
+ * pa_cache_write -- reshape_and_cache.
+ * For every t < num_tokens with s = slot_mapping[t] >= 0:
+ *     key_cache[s / block_size][s % block_size][:][:]   = k[t][:][:]
+ *     value_cache[s / block_size][s % block_size][:][:] = v[t][:][:]
+ *   k, v         [num_tokens, num_kv_heads, head_dim], dtype cache->dtype
+ *   slot_mapping int64 [num_tokens]; a negative slot marks padding (skipped)
+ * Bit-exact copy.  s >= num_blocks * block_size is skipped and sets
+ * PA_ERRBIT_SLOT_OOB.  Two tokens with the same slot in one call: undefined.
+ */
+pa_status pa_cache_write(const void* k, const void* v, void* key_cache, void* value_cache,
+                         const int64_t* slot_mapping, int64_t num_tokens,
+                         const pa_cache_desc* cache, int32_t* err_word, void* stream);
+
+/* Bytes of workspace pa_decode needs for these sizes (0 on bad arguments). */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads,
+                                int32_t max_blocks_per_seq, const pa_cache_desc* cache);
+
+/*
+ * pa_decode -- one query per request attends to all seq_lens[b] keys.
+ *   q            [num_seqs, num_heads, head_dim], dtype cache->dtype
+ *   block_tables int32 [num_seqs, max_blocks_per_seq]; entries past
+ *                ceil(seq_lens[b] / block_size) are never read
+ *   seq_lens     int32 [num_seqs]; the new token (already written by
+ *                pa_cache_write) is position seq_lens[b] - 1
+ *   scale        multiplies q.k before the softmax (1/sqrt(head_dim) usually)
+ *   out          [num_seqs, num_heads, head_dim] of out_dtype (PA_F32 or PA_BF16)
+ *   workspace    device buffer of >= pa_decode_workspace_size(...) bytes,
+ *                256-byte aligned; contents need no initialisation.  One
+ *                workspace must not be used by two calls that overlap on the GPU.
+ * Query head h uses KV head h / (num_heads / num_kv_heads) (GQA).
+ * seq_lens[b] == 0 writes a zero row.  Rows of requests with an error bit
+ * (table entry outside the pool, seq_len too long) are left unwritten.
+ */
+pa_status pa_decode(const void* q, const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, const int32_t* seq_lens, float scale,
+                    void* out, int32_t num_seqs, int32_t num_heads, int32_t max_blocks_per_seq,
+                    int32_t out_dtype, const pa_cache_desc* cache, void* workspace,
+                    size_t workspace_bytes, int32_t* err_word, void* stream);
+
+/* Bytes of workspace pa_mixed_step needs (0 on bad arguments). */
+size_t pa_mixed_step_workspace_size(int32_t num_seqs, int64_t num_tokens, int32_t num_heads,
+                                    int32_t max_blocks_per_seq, const pa_cache_desc* cache);
+
+/*
+ * pa_mixed_step -- causal varlen attention of a flattened step.
+ *   q               [num_tokens, num_heads, head_dim]
+ *   query_start_loc int32 [num_seqs + 1] (cu_seqlens of the queries)
+ *   seq_lens        int32 [num_seqs], KV length after this step
+ *   out             [num_tokens, num_heads, head_dim] of out_dtype
+ * Query i of request b (flattened row query_start_loc[b] + i) sits at
+ * position seq_lens[b] - q_b + i and attends to keys 0 .. that position
+ * (causal inside the new tokens, full over the cached prefix).  The new
+ * tokens' K/V must already be in the cache (pa_cache_write).  Requests may
+ * appear in any order and with any mix of q_b == 1 (decode) and q_b > 1
+ * (prefill chunk).  Rows of a request with q_b > seq_len are left unwritten
+ * and set PA_ERRBIT_QUERY_TOO_LONG.  Workspace rules as for pa_decode.
+ */
+pa_status pa_mixed_step(const void* q, const void* key_cache, const void* value_cache,
+                        const int32_t* block_tables, const int32_t* query_start_loc,
+                        const int32_t* seq_lens, float scale, void* out, int32_t num_seqs,
+                        int64_t num_tokens, int32_t num_heads, int32_t max_blocks_per_seq,
+                        int32_t out_dtype, const pa_cache_desc* cache, void* workspace,
+                        size_t workspace_bytes, int32_t* err_word, void* stream);
+
+/*
+ * pa_read_error -- synchronise `stream`, copy *err_word to *host_bits and
+ * reset it to 0.  Returns PA_OK when no bit was set, PA_ERR_DEVICE when some
+ * were, PA_ERR_CUDA if a CUDA call failed (e.g. an earlier kernel faulted).
+ */
+pa_status pa_read_error(int32_t* err_word, int32_t* host_bits, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,31 @@
+"""paged_kv_cache_434_b200 -- attention over a paged KV cache on B200 (sm_100a).
+
+The compute lives in libpa_b200.so (C ABI in include/pa.h); this package is
+its Python binding plus a seeded workload generator:
+
+  slot_mapping   slot of every new token from the block tables
+  cache_write    reshape_and_cache into [num_blocks, block_size, Hkv, D] pools
+  decode         GQA decode attention, online softmax, split-KV + LSE merge
+  mixed_step     causal varlen attention of a chunked-prefill + decode step
+  step           slot_mapping -> cache_write -> attention, the per-layer path
+"""
+
+from .binding import (  # noqa: F401
+    ERRBIT_BLOCK_OOB,
+    ERRBIT_QUERY_TOO_LONG,
+    ERRBIT_SEQ_TOO_LONG,
+    ERRBIT_SLOT_OOB,
+    ERRBIT_TIMEOUT,
+    PagedAttentionError,
+    cache_write,
+    decode,
+    decode_workspace_size,
+    library_path,
+    mixed_step,
+    mixed_step_workspace_size,
+    new_error_word,
+    read_error,
+    slot_mapping,
+    version,
+)
+from .step import step  # noqa: F401

@@ -1,0 +1,248 @@
+"""ctypes binding of libpa_b200.so: argument marshalling only.
+
+Every function takes torch tensors that live on the current CUDA device,
+checks dtype / shape / contiguity, and passes raw device pointers, sizes and
+the current stream to the C ABI declared in include/pa.h.  All arithmetic
+happens in the library's CUDA kernels.  There is no CPU fallback: if the
+library cannot be loaded, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libpa_b200.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_DEVICE = range(6)
+PA_F32, PA_BF16 = 0, 1
+
+ERRBIT_SLOT_OOB = 0x1
+ERRBIT_BLOCK_OOB = 0x2
+ERRBIT_SEQ_TOO_LONG = 0x4
+ERRBIT_QUERY_TOO_LONG = 0x8
+ERRBIT_TIMEOUT = 0x10
+
+EXPORTS = ("pa_status_str", "pa_version", "pa_slot_mapping", "pa_cache_write",
+           "pa_decode_workspace_size", "pa_decode", "pa_mixed_step_workspace_size",
+           "pa_mixed_step", "pa_read_error")
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib().pa_status_str(status).decode() if _LIB is not None else str(status)
+        super().__init__(f"{where}: {msg} (status {status})")
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int64), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("dtype", ctypes.c_int32)]
+
+
+_LIB = None
+_vp, _i32, _i64, _f32, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                              ctypes.c_size_t)
+_desc_p = ctypes.POINTER(CacheDesc)
+
+_SIGNATURES = {
+    "pa_status_str": ([ctypes.c_int], ctypes.c_char_p),
+    "pa_version": ([], ctypes.c_int),
+    "pa_slot_mapping": ([_vp, _i32, _vp, _vp, _i32, _i64, _i32, _i64, _vp, _vp, _vp], ctypes.c_int),
+    "pa_cache_write": ([_vp, _vp, _vp, _vp, _vp, _i64, _desc_p, _vp, _vp], ctypes.c_int),
+    "pa_decode_workspace_size": ([_i32, _i32, _i32, _desc_p], _sz),
+    "pa_decode": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i32, _i32, _i32, _desc_p, _vp, _sz,
+                   _vp, _vp], ctypes.c_int),
+    "pa_mixed_step_workspace_size": ([_i32, _i64, _i32, _i32, _desc_p], _sz),
+    "pa_mixed_step": ([_vp, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i64, _i32, _i32, _i32,
+                       _desc_p, _vp, _sz, _vp, _vp], ctypes.c_int),
+    "pa_read_error": ([_vp, ctypes.POINTER(ctypes.c_int32), _vp], ctypes.c_int),
+}
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"libpa_b200.so not found at {_LIB_PATH}; build it with "
+                "`python -m paged_kv_cache_434_b200.build` (needs nvcc, sm_100a)")
+        lib = ctypes.CDLL(_LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _LIB = lib
+    return _LIB
+
+
+def version() -> int:
+    return _lib().pa_version()
+
+
+# ---------------------------------------------------------------- helpers
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return PA_F32
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None, ndim=None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    return t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _err_ptr(err):
+    if err is None:
+        return None
+    return _cuda(err, "err", torch.int32)
+
+
+def cache_desc(k_cache: torch.Tensor) -> CacheDesc:
+    nb, bs, hkv, d = k_cache.shape
+    return CacheDesc(nb, bs, hkv, d, _dt(k_cache))
+
+
+def _check(status: int, where: str):
+    if status != PA_OK:
+        raise PagedAttentionError(status, where)
+
+
+def new_error_word(device=None) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def read_error(err: torch.Tensor) -> int:
+    """Synchronise the current stream, return the error bits and clear them."""
+    bits = ctypes.c_int32(0)
+    st = _lib().pa_read_error(_cuda(err, "err", torch.int32), ctypes.byref(bits), _stream())
+    if st not in (PA_OK, PA_ERR_DEVICE):
+        raise PagedAttentionError(st, "pa_read_error")
+    return bits.value
+
+
+# ---------------------------------------------------------------- operations
+
+def slot_mapping(block_tables, query_start_loc, seq_lens, block_size: int, num_blocks: int,
+                 num_tokens: int, out=None, err=None):
+    """int64 slot of every new token (see pa_slot_mapping)."""
+    B, W = block_tables.shape
+    if out is None:
+        out = torch.empty(num_tokens, dtype=torch.int64, device=block_tables.device)
+    _check(_lib().pa_slot_mapping(
+        _cuda(block_tables, "block_tables", torch.int32, 2), W,
+        _cuda(query_start_loc, "query_start_loc", torch.int32, 1),
+        _cuda(seq_lens, "seq_lens", torch.int32, 1), B, num_tokens, block_size, num_blocks,
+        _cuda(out, "slot_mapping", torch.int64, 1), _err_ptr(err), _stream()), "pa_slot_mapping")
+    return out
+
+
+def cache_write(k, v, k_cache, v_cache, slot_mapping, err=None):
+    """reshape_and_cache: k_cache[slot // bs, slot % bs] = k[t] (and v)."""
+    desc = cache_desc(k_cache)
+    T = k.shape[0]
+    for name, t in (("k", k), ("v", v)):
+        if t.dim() != 3 or tuple(t.shape[1:]) != (desc.num_kv_heads, desc.head_dim) or \
+                t.shape[0] != T or t.dtype != k_cache.dtype:
+            raise ValueError(f"{name} must be [num_tokens, num_kv_heads, head_dim] of the cache dtype")
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
+        raise ValueError("v_cache must match k_cache")
+    if slot_mapping.shape[0] != T:
+        raise ValueError("slot_mapping must have num_tokens entries")
+    _check(_lib().pa_cache_write(
+        _cuda(k, "k"), _cuda(v, "v"), _cuda(k_cache, "k_cache", ndim=4),
+        _cuda(v_cache, "v_cache", ndim=4), _cuda(slot_mapping, "slot_mapping", torch.int64, 1),
+        T, ctypes.byref(desc), _err_ptr(err), _stream()), "pa_cache_write")
+
+
+def decode_workspace_size(num_seqs, num_heads, max_blocks_per_seq, k_cache) -> int:
+    desc = cache_desc(k_cache)
+    return int(_lib().pa_decode_workspace_size(num_seqs, num_heads, max_blocks_per_seq,
+                                               ctypes.byref(desc)))
+
+
+def mixed_step_workspace_size(num_seqs, num_tokens, num_heads, max_blocks_per_seq, k_cache) -> int:
+    desc = cache_desc(k_cache)
+    return int(_lib().pa_mixed_step_workspace_size(num_seqs, num_tokens, num_heads,
+                                                   max_blocks_per_seq, ctypes.byref(desc)))
+
+
+def _workspace(nbytes, device, workspace):
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace too small: need {nbytes} bytes")
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype):
+    desc = cache_desc(k_cache)
+    if q.dtype != k_cache.dtype or q.dim() != 3 or q.shape[2] != desc.head_dim:
+        raise ValueError("q must be [rows, num_heads, head_dim] of the cache dtype")
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
+        raise ValueError("v_cache must match k_cache")
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    return desc
+
+
+def decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=None,
+           out_dtype=torch.float32, workspace=None, err=None):
+    """Decode attention: out[b, h] over the first seq_lens[b] keys of request b."""
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype)
+    B, H, D = q.shape
+    W = block_tables.shape[1]
+    if out is None:
+        out = torch.empty(B, H, D, dtype=out_dtype, device=q.device)
+    nbytes = decode_workspace_size(B, H, W, k_cache)
+    ws = _workspace(nbytes, q.device, workspace)
+    _check(_lib().pa_decode(
+        _cuda(q, "q"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+        _cuda(block_tables, "block_tables", torch.int32, 2),
+        _cuda(seq_lens, "seq_lens", torch.int32, 1), float(scale), _cuda(out, "out"), B, H, W,
+        _dt(out), ctypes.byref(desc), _cuda(ws, "workspace"), ws.numel() * ws.element_size(),
+        _err_ptr(err), _stream()), "pa_decode")
+    return out
+
+
+def mixed_step(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, scale: float,
+               out=None, out_dtype=torch.float32, workspace=None, err=None):
+    """Causal varlen attention of a flattened step (chunked prefill + decode)."""
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype)
+    T, H, D = q.shape
+    B, W = block_tables.shape
+    if out is None:
+        out = torch.empty(T, H, D, dtype=out_dtype, device=q.device)
+    nbytes = mixed_step_workspace_size(B, T, H, W, k_cache)
+    ws = _workspace(nbytes, q.device, workspace)
+    _check(_lib().pa_mixed_step(
+        _cuda(q, "q"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+        _cuda(block_tables, "block_tables", torch.int32, 2),
+        _cuda(query_start_loc, "query_start_loc", torch.int32, 1),
+        _cuda(seq_lens, "seq_lens", torch.int32, 1), float(scale), _cuda(out, "out"), B, T, H, W,
+        _dt(out), ctypes.byref(desc), _cuda(ws, "workspace"), ws.numel() * ws.element_size(),
+        _err_ptr(err), _stream()), "pa_mixed_step")
+    return out

@@ -1,0 +1,463 @@
+// attn_common.cu -- work planner, CUDA-core attention kernel and the split-KV
+// log-sum-exp merge, shared by pa_decode and pa_mixed_step.
+//
+// What is computed ("AI Infra入门干货总结：大模型是如何高效推理的", section
+// "Attention (FlashAttention, Scaled Dot-Product Attention)"): for every query
+// row r of request b and query head h, with kv = h / (Hq / Hkv),
+//     o = sum_j softmax_j(scale * <q_rh, k_j,kv>) v_j,kv   over j < key_len(r)
+// where key_len(r) = seq_len_b - q_b + i + 1 for the i-th new token of b
+// (causal inside the chunk, full over the cached prefix).  K/V row j lives in
+// physical block block_tables[b][j / block_size] at offset j % block_size.
+//
+// Flash-Decoding ("总结": split the KV axis for SM utilisation, re-normalise
+// across pieces with log-sum-exp): the key range of a row is cut into
+// partitions of P keys; each (row, head group, partition) is one work item
+// producing (m, l, o) with the online softmax (running max m, running sum l,
+// rescale by exp(m_old - m_new), as in the ursb.me Field Note blurb); a second
+// pass merges the partitions: O = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k.
+// Scores are kept in log2 units (scale * log2 e folded in) so exp becomes ex2.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace pa {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WsLayout ws_layout(int64_t num_qrows, int num_heads, int head_dim, int head_groups,
+                   int64_t max_parts, int64_t max_tiles) {
+  WsLayout L{};
+  L.num_qrows = num_qrows;
+  L.max_parts = max_parts;
+  L.max_items = num_qrows * head_groups * max_parts;
+  L.max_tiles = max_tiles;
+  size_t off = 0;
+  L.ctrl = off;
+  off = align_up(off + 64 * sizeof(int32_t), 256);
+  L.qrow_info = off;
+  off = align_up(off + num_qrows * sizeof(int4), 256);
+  L.nparts = off;
+  off = align_up(off + num_qrows * sizeof(int32_t), 256);
+  L.qrow_bad = off;
+  off = align_up(off + num_qrows * sizeof(int32_t), 256);
+  L.items = off;
+  off = align_up(off + L.max_items * sizeof(int4), 256);
+  L.part_ml = off;
+  off = align_up(off + num_qrows * num_heads * max_parts * sizeof(float2), 256);
+  L.part_o = off;
+  off = align_up(off + num_qrows * num_heads * max_parts * head_dim * sizeof(float), 256);
+  L.tiles = off;
+  off = align_up(off + max_tiles * sizeof(int4), 256);
+  L.total = off;
+  return L;
+}
+
+WsView ws_view(void* base, const WsLayout& L) {
+  char* p = static_cast<char*>(base);
+  WsView v;
+  v.ctrl = reinterpret_cast<int32_t*>(p + L.ctrl);
+  v.qrow_info = reinterpret_cast<int4*>(p + L.qrow_info);
+  v.nparts = reinterpret_cast<int32_t*>(p + L.nparts);
+  v.qrow_bad = reinterpret_cast<int32_t*>(p + L.qrow_bad);
+  v.items = reinterpret_cast<int4*>(p + L.items);
+  v.part_ml = reinterpret_cast<float2*>(p + L.part_ml);
+  v.part_o = reinterpret_cast<float*>(p + L.part_o);
+  v.tiles = reinterpret_cast<int4*>(p + L.tiles);
+  v.max_parts = L.max_parts;
+  v.max_items = L.max_items;
+  v.max_tiles = L.max_tiles;
+  return v;
+}
+
+// ======================================================================= planner
+// One CTA.  Pass 1 validates every request, fills the per-row table and sums the
+// work (in 16-key stages); the partition length P is then chosen so that the
+// item count is near target_items and no row needs more than max_parts
+// partitions.  Pass 2 counts items per thread, pass 3 scans and writes them.
+constexpr int kPlanThreads = 1024;
+
+__device__ __forceinline__ void request_rows(const AttnGeom& g, int b, int& r0, int& q_b) {
+  if (g.query_start_loc) {
+    r0 = g.query_start_loc[b];
+    q_b = g.query_start_loc[b + 1] - r0;
+  } else {
+    r0 = b;
+    q_b = 1;
+  }
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs a, WsView ws) {
+  grid_launch_dependents();
+  __shared__ long long s_sum[32];
+  __shared__ int s_max[32];
+  __shared__ int s_scan[32];
+  __shared__ int s_P;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool decode_mode = g.query_start_loc == nullptr;
+  const int64_t max_keys = static_cast<int64_t>(g.max_blocks) * g.block_size;
+
+  // rows no request covers stay unwritten
+  for (int r = tid; r < g.num_qrows; r += kPlanThreads) ws.nparts[r] = -1;
+  __syncthreads();
+
+  long long my_units = 0;
+  int my_max = 0;
+  for (int b = tid; b < g.num_seqs; b += kPlanThreads) {
+    int r0, q_b;
+    request_rows(g, b, r0, q_b);
+    const int L = g.seq_lens[b];
+    int bits = 0;
+    if (r0 < 0 || r0 > g.num_qrows) {
+      if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_QUERY_TOO_LONG);
+      continue;
+    }
+    if (decode_mode) {
+      if (L < 0) bits |= PA_ERRBIT_QUERY_TOO_LONG;
+    } else if (q_b < 0 || q_b > L) {
+      bits |= PA_ERRBIT_QUERY_TOO_LONG;
+    }
+    if (L > max_keys) bits |= PA_ERRBIT_SEQ_TOO_LONG;
+    if (bits && g.err_word) atomicOr(g.err_word, bits);
+    const bool expand = decode_mode || q_b == 1 || a.expand_prefill;
+    for (int i = 0; i < q_b && r0 + i < g.num_qrows; ++i) {
+      const int r = r0 + i;
+      ws.qrow_bad[r] = 0;
+      if (bits) {
+        ws.qrow_info[r] = make_int4(b, 0, 0, 0);
+        ws.nparts[r] = -1;
+        continue;
+      }
+      if (!expand) {
+        ws.qrow_info[r] = make_int4(b, 0, 0, 0);
+        ws.nparts[r] = -2;  // handled by prefill tiles
+        continue;
+      }
+      const int key_len = decode_mode ? L : L - q_b + i + 1;
+      ws.qrow_info[r] = make_int4(b, key_len, 1, 0);
+      const int units = (key_len + kStageTokens - 1) / kStageTokens;
+      my_units += units;
+      my_max = max(my_max, units);
+    }
+  }
+  // block reductions
+  for (int o = 16; o; o >>= 1) {
+    my_units += __shfl_xor_sync(0xffffffffu, my_units, o);
+    my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, o));
+  }
+  if (lane == 0) {
+    s_sum[warp] = my_units;
+    s_max[warp] = my_max;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    long long total = 0;
+    int mx = 0;
+    for (int w = 0; w < kPlanThreads / 32; ++w) {
+      total += s_sum[w];
+      mx = max(mx, s_max[w]);
+    }
+    long long by_target = (total * a.head_groups + a.target_items - 1) / max(a.target_items, 1);
+    long long by_cap = (mx + ws.max_parts - 1) / ws.max_parts;
+    long long P = max(static_cast<long long>(a.min_part_stages), max(by_target, by_cap));
+    s_P = static_cast<int>(max(P, 1LL));
+  }
+  __syncthreads();
+  const int P = s_P;
+
+  // pass 2: items per thread
+  int my_items = 0;
+  for (int b = tid; b < g.num_seqs; b += kPlanThreads) {
+    int r0, q_b;
+    request_rows(g, b, r0, q_b);
+    if (r0 < 0) continue;
+    for (int i = 0; i < q_b && r0 + i < g.num_qrows; ++i) {
+      const int4 info = ws.qrow_info[r0 + i];
+      if (info.z == 0) continue;
+      const int units = (info.y + kStageTokens - 1) / kStageTokens;
+      my_items += (units + P - 1) / P * a.head_groups;
+    }
+  }
+  // exclusive scan over the CTA
+  int incl = my_items;
+  for (int o = 1; o < 32; o <<= 1) {
+    int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) s_scan[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = s_scan[lane];
+    int vi = v;
+    for (int o = 1; o < 32; o <<= 1) {
+      int n = __shfl_up_sync(0xffffffffu, vi, o);
+      if (lane >= o) vi += n;
+    }
+    s_scan[lane] = vi - v;  // exclusive prefix of warp totals
+    if (lane == 31) {
+      ws.ctrl[0] = 0;
+      ws.ctrl[1] = vi;
+      ws.ctrl[2] = P * kStageTokens;
+      ws.ctrl[3] = 0;
+    }
+  }
+  __syncthreads();
+  int pos = s_scan[warp] + incl - my_items;
+
+  // pass 3: write items and partition counts
+  for (int b = tid; b < g.num_seqs; b += kPlanThreads) {
+    int r0, q_b;
+    request_rows(g, b, r0, q_b);
+    if (r0 < 0) continue;
+    for (int i = 0; i < q_b && r0 + i < g.num_qrows; ++i) {
+      const int r = r0 + i;
+      const int4 info = ws.qrow_info[r];
+      if (info.z == 0) continue;
+      const int units = (info.y + kStageTokens - 1) / kStageTokens;
+      const int np = (units + P - 1) / P;
+      ws.nparts[r] = np;
+      for (int p = 0; p < np; ++p)
+        for (int hg = 0; hg < a.head_groups; ++hg) ws.items[pos++] = make_int4(r, hg, p, 0);
+    }
+  }
+}
+
+cudaError_t launch_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws, cudaStream_t s) {
+  plan_kernel<<<1, kPlanThreads, 0, s>>>(g, a, ws);
+  return cudaGetLastError();
+}
+
+// ======================================================================= generic
+// CUDA-core path (any dtype, D in {64,128}, group <= 16): one CTA of 4 warps per
+// item (row, KV head, partition).  Each warp walks every 4th key; the 32 lanes
+// split head_dim, the q.k partial sums are combined with xor shuffles, and
+// each warp keeps its own running (m, l, o) per query head of the group.  The
+// four warps are merged through shared memory at the end of the item.
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T, int V>
+__device__ __forceinline__ void load_row(const T* p, float (&x)[V]) {
+#pragma unroll
+  for (int e = 0; e < V; ++e) x[e] = to_f32(p[e]);
+}
+
+__device__ __forceinline__ void store_out(void* out, int out_dtype, int64_t idx, float v) {
+  if (out_dtype == PA_F32)
+    static_cast<float*>(out)[idx] = v;
+  else
+    static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
+}
+
+constexpr int kGenWarps = 4;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kGenWarps * 32) attn_generic_kernel(AttnGeom g, WsView ws) {
+  constexpr int V = D / 32;
+  __shared__ float s_q[kMaxGroup][D];
+  __shared__ float s_o[kGenWarps][kMaxGroup][D];
+  __shared__ float s_m[kGenWarps][kMaxGroup];
+  __shared__ float s_l[kGenWarps][kMaxGroup];
+  __shared__ int s_item;
+  __shared__ int s_bad;
+  grid_dependency_wait();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = g.num_heads / g.num_kv_heads;
+  const int n_items = ws.ctrl[1];
+  const int P = ws.ctrl[2];
+  const T* q = static_cast<const T*>(g.q);
+  const T* kc = static_cast<const T*>(g.k_cache);
+  const T* vc = static_cast<const T*>(g.v_cache);
+
+  for (;;) {
+    if (tid == 0) {
+      s_item = atomicAdd(&ws.ctrl[0], 1);
+      s_bad = 0;
+    }
+    __syncthreads();
+    const int it = s_item;
+    if (it >= n_items) break;
+    const int4 item = ws.items[it];
+    const int r = item.x, hk = item.y, p = item.z;
+    const int4 info = ws.qrow_info[r];
+    const int b = info.x, key_len = info.y;
+    const int lo = p * P, hi = min(lo + P, key_len);
+    for (int idx = tid; idx < G * D; idx += blockDim.x) {
+      const int gq = idx / D, d = idx % D;
+      s_q[gq][d] = to_f32(q[(static_cast<int64_t>(r) * g.num_heads + hk * G + gq) * D + d]);
+    }
+    __syncthreads();
+
+    float m[kMaxGroup], l[kMaxGroup], o[kMaxGroup][V];
+#pragma unroll
+    for (int gq = 0; gq < kMaxGroup; ++gq) {
+      m[gq] = -INFINITY;
+      l[gq] = 0.f;
+#pragma unroll
+      for (int e = 0; e < V; ++e) o[gq][e] = 0.f;
+    }
+    const int32_t* table = g.block_tables + static_cast<int64_t>(b) * g.max_blocks;
+    bool bad = false;
+    for (int j = lo + warp; j < hi; j += kGenWarps) {
+      const int phys = table[j / g.block_size];
+      if (phys < 0 || phys >= g.num_blocks) {
+        bad = true;
+        continue;
+      }
+      const int64_t row = static_cast<int64_t>(phys) * g.block_size + j % g.block_size;
+      const int64_t off = (row * g.num_kv_heads + hk) * D + lane * V;
+      float kx[V], vx[V];
+      load_row<T, V>(kc + off, kx);
+      load_row<T, V>(vc + off, vx);
+#pragma unroll
+      for (int gq = 0; gq < kMaxGroup; ++gq) {
+        if (gq < G) {
+          float dot = 0.f;
+#pragma unroll
+          for (int e = 0; e < V; ++e) dot = fmaf(s_q[gq][lane * V + e], kx[e], dot);
+#pragma unroll
+          for (int o2 = 16; o2; o2 >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o2);
+          const float s = dot * g.scale_log2;
+          const float m_new = fmaxf(m[gq], s);
+          const float alpha = fast_exp2(m[gq] - m_new);
+          const float pe = fast_exp2(s - m_new);
+          l[gq] = l[gq] * alpha + pe;
+#pragma unroll
+          for (int e = 0; e < V; ++e) o[gq][e] = fmaf(o[gq][e], alpha, pe * vx[e]);
+          m[gq] = m_new;
+        }
+      }
+    }
+    if (bad) s_bad = 1;
+#pragma unroll
+    for (int gq = 0; gq < kMaxGroup; ++gq) {
+      if (gq < G) {
+        if (lane == 0) {
+          s_m[warp][gq] = m[gq];
+          s_l[warp][gq] = l[gq];
+        }
+#pragma unroll
+        for (int e = 0; e < V; ++e) s_o[warp][gq][lane * V + e] = o[gq][e];
+      }
+    }
+    __syncthreads();
+    const bool row_bad = s_bad != 0;
+    if (row_bad) {
+      if (tid == 0) {
+        ws.qrow_bad[r] = 1;
+        if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_BLOCK_OOB);
+      }
+    }
+    const int np = ws.nparts[r];
+    for (int idx = tid; idx < G * D; idx += blockDim.x) {
+      const int gq = idx / D, d = idx % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kGenWarps; ++w) M = fmaxf(M, s_m[w][gq]);
+      float Ls = 0.f, O = 0.f;
+#pragma unroll
+      for (int w = 0; w < kGenWarps; ++w) {
+        const float c = (s_m[w][gq] == -INFINITY) ? 0.f : fast_exp2(s_m[w][gq] - M);
+        Ls = fmaf(s_l[w][gq], c, Ls);
+        O = fmaf(s_o[w][gq][d], c, O);
+      }
+      const int h = hk * G + gq;
+      if (np == 1) {
+        if (!row_bad)
+          store_out(g.out, g.out_dtype, (static_cast<int64_t>(r) * g.num_heads + h) * D + d,
+                    O / Ls);
+      } else {
+        const int64_t slot = (static_cast<int64_t>(r) * g.num_heads + h) * ws.max_parts + p;
+        if (d == 0) ws.part_ml[slot] = make_float2(M, Ls);
+        ws.part_o[slot * D + d] = O;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms,
+                                cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms * 8);
+  cfg.blockDim = dim3(kGenWarps * 32);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (g.dtype == PA_F32) {
+    if (g.head_dim == 64) return cudaLaunchKernelEx(&cfg, attn_generic_kernel<float, 64>, g, ws);
+    return cudaLaunchKernelEx(&cfg, attn_generic_kernel<float, 128>, g, ws);
+  }
+  if (g.head_dim == 64)
+    return cudaLaunchKernelEx(&cfg, attn_generic_kernel<__nv_bfloat16, 64>, g, ws);
+  return cudaLaunchKernelEx(&cfg, attn_generic_kernel<__nv_bfloat16, 128>, g, ws);
+}
+
+// ======================================================================= merge
+// One warp per (row, query head).  Rows with a single partition were written by
+// the attention kernel; rows with none get zeros; invalid rows are skipped.
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(AttnGeom g, WsView ws) {
+  constexpr int V = D / 32;
+  grid_dependency_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (idx >= static_cast<int64_t>(g.num_qrows) * g.num_heads) return;
+  const int r = static_cast<int>(idx / g.num_heads);
+  const int np = ws.nparts[r];
+  if (np == 1 || np < 0 || ws.qrow_bad[r]) return;
+  const int64_t out_base = idx * D + lane * V;
+  if (np == 0) {
+#pragma unroll
+    for (int e = 0; e < V; ++e) store_out(g.out, g.out_dtype, out_base + e, 0.f);
+    return;
+  }
+  const int64_t base = idx * ws.max_parts;
+  float M = -INFINITY;
+  for (int k = lane; k < np; k += 32) M = fmaxf(M, ws.part_ml[base + k].x);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float den = 0.f, acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  for (int k = 0; k < np; ++k) {
+    const float2 ml = ws.part_ml[base + k];
+    const float c = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
+    den = fmaf(ml.y, c, den);
+    const float* po = ws.part_o + (base + k) * D + lane * V;
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = fmaf(po[e], c, acc[e]);
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int e = 0; e < V; ++e) store_out(g.out, g.out_dtype, out_base + e, acc[e] * inv);
+}
+
+cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, cudaStream_t s) {
+  const int64_t warps = static_cast<int64_t>(g.num_qrows) * g.num_heads;
+  if (warps == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((warps + 7) / 8));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (g.head_dim == 64) return cudaLaunchKernelEx(&cfg, merge_kernel<64>, g, ws);
+  return cudaLaunchKernelEx(&cfg, merge_kernel<128>, g, ws);
+}
+
+}  // namespace pa

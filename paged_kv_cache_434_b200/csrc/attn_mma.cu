@@ -1,0 +1,480 @@
+// attn_mma.cu -- bf16 paged attention for query rows that see a long key range
+// (decode rows, split-KV partitions): TMA-staged K/V tiles, one K/V read serving
+// all query heads of a GQA group, tensor-core (mma.sync m16n8k16) products.
+//
+// Math as in attn_common.cu ("AI Infra入门干货总结：大模型是如何高效推理的",
+// "Attention (FlashAttention, Scaled Dot-Product Attention)" and "总结").
+//
+// Layout and work split
+//   * Pools are [num_blocks, block_size, Hkv, D] bf16.  A stage is 16
+//     consecutive keys of one request: for each of the HG KV heads of the
+//     item's head group and each 64-column half of D, a TMA box of
+//     [16 keys x 64 dims] (2 KiB, 128-byte swizzle) is copied from the
+//     physical block the block table names.  16 keys never straddle a
+//     block when block_size >= 16; block_size 8 takes two boxes per stage.
+//   * A persistent CTA = HG consumer warps (warp w owns KV head w of the
+//     group) + 1 producer warp.  The producer pulls items from a global
+//     counter, walks their block tables and keeps NS stages in flight
+//     (full/empty mbarriers); stage descriptors travel with the stage.
+//   * Consumer warp: the G query heads of its KV head are the rows of a
+//     16-row A tile (rows >= G are zero), S = Q K^T uses K as the col-major B
+//     operand (ldmatrix), P V uses V through ldmatrix.trans.  Row max and
+//     row sums are reduced over the 4 lanes of a quad with xor shuffles; the
+//     running (m, l, O) live in registers for the whole item.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace pa {
+
+namespace mmak {
+
+enum : int { kFirst = 1, kLast = 2, kBad = 4, kEnd = 8 };
+
+struct StageInfo {
+  int qrow;
+  int b;
+  int hg;
+  int part;
+  int nvalid;
+  int flags;
+  int pad0, pad1;
+};
+
+template <int D, int HG>
+struct Cfg {
+  static constexpr int NH = D / 64;                     // 64-column halves
+  static constexpr int kTile = 2048;                    // [16 keys x 64 dims] bf16
+  static constexpr int kTensorBytes = HG * NH * kTile;  // K (or V) part of a stage
+  static constexpr int kStageBytes = 2 * kTensorBytes;
+  static constexpr int kBudget = 200 * 1024;
+  static constexpr int NS0 = kBudget / kStageBytes;
+  static constexpr int NS = NS0 > 6 ? 6 : (NS0 < 2 ? 2 : NS0);
+  static constexpr int kThreads = (HG + 1) * 32;
+  static constexpr int kSmem = NS * kStageBytes + 1024 /*align*/ + 1024 /*info+bars*/;
+};
+
+// byte offset of (key, 16-byte chunk) inside one 128B-swizzled [16 x 64] tile
+__device__ __forceinline__ uint32_t swz(int key, int chunk) {
+  return static_cast<uint32_t>(key * 128 + ((chunk ^ (key & 7)) << 4));
+}
+
+}  // namespace mmak
+
+template <int D, int HG>
+__global__ void __launch_bounds__((HG + 1) * 32, 1)
+    attn_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    AttnGeom g, WsView ws, int box_rows) {
+  using C = mmak::Cfg<D, HG>;
+  constexpr int NS = C::NS;
+  constexpr int NH = C::NH;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* stages = smem;
+  mmak::StageInfo* info = reinterpret_cast<mmak::StageInfo*>(smem + NS * C::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(info + NS);
+  uint64_t* empty = full + NS;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], HG);
+    }
+    s_abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  __syncthreads();
+  grid_dependency_wait();
+
+  const int n_items = ws.ctrl[1];
+  const int P = ws.ctrl[2];
+  const int G = g.num_heads / g.num_kv_heads;
+
+  if (warp == HG) {
+    // ------------------------------------------------------------- producer
+    if (lane != 0) return;
+    const uint64_t policy = l2_policy_evict_first();
+    int stage = 0;
+    uint32_t phase = 0;
+    int round = 0;  // completed passes over the ring
+    bool ok = true;
+    for (;;) {
+      const int it = atomicAdd(&ws.ctrl[0], 1);
+      const bool done = it >= n_items;
+      int4 item = make_int4(0, 0, 0, 0), qi = make_int4(0, 0, 0, 0);
+      if (!done) {
+        item = ws.items[it];
+        qi = ws.qrow_info[item.x];
+      }
+      const int lo = item.z * P;
+      const int hi = done ? lo + 1 : min(lo + P, qi.y);
+      const int32_t* table = g.block_tables + static_cast<int64_t>(qi.x) * g.max_blocks;
+      for (int key0 = lo; key0 < hi; key0 += kStageTokens) {
+        if (round > 0 && !mbar_wait_bounded(&empty[stage], phase ^ 1, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        mmak::StageInfo si;
+        si.qrow = item.x;
+        si.b = qi.x;
+        si.hg = item.y;
+        si.part = item.z;
+        si.nvalid = min(kStageTokens, hi - key0);
+        si.flags = done ? mmak::kEnd
+                        : ((key0 == lo ? mmak::kFirst : 0) |
+                           (key0 + kStageTokens >= hi ? mmak::kLast : 0));
+        int rows0 = 0, rows1 = -1;
+        if (!done) {
+          const int phys0 = table[key0 / g.block_size];
+          if (phys0 < 0 || phys0 >= g.num_blocks) si.flags |= mmak::kBad;
+          rows0 = phys0 * g.block_size + key0 % g.block_size;
+          if (box_rows < kStageTokens && si.nvalid > box_rows) {
+            const int phys1 = table[(key0 + box_rows) / g.block_size];
+            if (phys1 < 0 || phys1 >= g.num_blocks) si.flags |= mmak::kBad;
+            rows1 = phys1 * g.block_size + (key0 + box_rows) % g.block_size;
+          }
+        }
+        info[stage] = si;
+        if (done || (si.flags & mmak::kBad)) {
+          mbar_arrive(&full[stage]);
+        } else {
+          const int boxes = rows1 >= 0 ? 2 : 1;
+          const uint32_t box_bytes = static_cast<uint32_t>(box_rows) * 128u;
+          mbar_arrive_expect_tx(&full[stage], 2u * HG * NH * boxes * box_bytes);
+          uint8_t* kbase = stages + stage * C::kStageBytes;
+          uint8_t* vbase = kbase + C::kTensorBytes;
+          const int head0 = item.y * HG;
+#pragma unroll
+          for (int hh = 0; hh < HG; ++hh) {
+#pragma unroll
+            for (int dh = 0; dh < NH; ++dh) {
+              const int toff = (hh * NH + dh) * C::kTile;
+              tma_load_3d_hint(kbase + toff, &tmK, &full[stage], dh * 64, head0 + hh, rows0, policy);
+              tma_load_3d_hint(vbase + toff, &tmV, &full[stage], dh * 64, head0 + hh, rows0, policy);
+              if (rows1 >= 0) {
+                tma_load_3d_hint(kbase + toff + box_bytes, &tmK, &full[stage], dh * 64, head0 + hh,
+                                 rows1, policy);
+                tma_load_3d_hint(vbase + toff + box_bytes, &tmV, &full[stage], dh * 64, head0 + hh,
+                                 rows1, policy);
+              }
+            }
+          }
+        }
+        if (++stage == NS) {
+          stage = 0;
+          phase ^= 1;
+          ++round;
+        }
+      }
+      if (!ok || done) break;
+    }
+    if (!ok) {
+      s_abort = 1;
+      if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------- consumers
+  const int hh = warp;  // KV head within the group
+  const int qr = lane >> 2;      // fragment row (and row + 8)
+  const int qc = (lane & 3) * 2; // fragment column pair
+  uint32_t qa[D / 16][4];
+  float o[D / 8][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  bool bad = false;
+  int stage = 0;
+  uint32_t phase = 0;
+  const __nv_bfloat16* qbase = static_cast<const __nv_bfloat16*>(g.q);
+
+  for (;;) {
+    if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
+      if (g.err_word && lane == 0) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
+      break;
+    }
+    const mmak::StageInfo si = info[stage];
+    if (si.flags & mmak::kEnd) break;
+    const int head = (si.hg * HG + hh) * G;  // first query head of this warp's group
+    if (si.flags & mmak::kFirst) {
+      const __nv_bfloat16* qrow = qbase + (static_cast<int64_t>(si.qrow) * g.num_heads + head) * D;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int c = kk * 16 + qc;
+        qa[kk][0] = qr < G ? *reinterpret_cast<const uint32_t*>(qrow + qr * D + c) : 0u;
+        qa[kk][1] = qr + 8 < G ? *reinterpret_cast<const uint32_t*>(qrow + (qr + 8) * D + c) : 0u;
+        qa[kk][2] = qr < G ? *reinterpret_cast<const uint32_t*>(qrow + qr * D + c + 8) : 0u;
+        qa[kk][3] =
+            qr + 8 < G ? *reinterpret_cast<const uint32_t*>(qrow + (qr + 8) * D + c + 8) : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+      bad = false;
+    }
+    if (si.flags & mmak::kBad) {
+      bad = true;
+    } else {
+      const uint32_t kt = smem_u32(stages + stage * C::kStageBytes) + hh * NH * C::kTile;
+      const uint32_t vt = kt + C::kTensorBytes;
+      // ---- S = Q K^T over 16 keys
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int mi = lane >> 3;
+        const int key = (lane & 7) + ((mi >> 1) << 3);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int dh = kk >> 2, c16 = kk & 3;
+          const int chunk = 2 * c16 + (mi & 1);
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4(kt + dh * C::kTile + mmak::swz(key, chunk), b0, b1, b2, b3);
+          mma_bf16_16816(s0, qa[kk], b0, b1);
+          mma_bf16_16816(s1, qa[kk], b2, b3);
+        }
+      }
+      // ---- mask, scale, online softmax
+      const int nv = si.nvalid;
+      float p[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = qc + (e & 1);
+        p[e] = key < nv ? s0[e] * g.scale_log2 : -INFINITY;
+        p[4 + e] = key + 8 < nv ? s1[e] * g.scale_log2 : -INFINITY;
+      }
+      float mx0 = fmaxf(fmaxf(p[0], p[1]), fmaxf(p[4], p[5]));
+      float mx1 = fmaxf(fmaxf(p[2], p[3]), fmaxf(p[6], p[7]));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float a0 = fast_exp2(m0 - mn0), a1 = fast_exp2(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      uint32_t pa[4];
+      float ps0 = 0.f, ps1 = 0.f;
+      {
+        const float e0 = fast_exp2(p[0] - mn0), e1 = fast_exp2(p[1] - mn0);
+        const float e2 = fast_exp2(p[2] - mn1), e3 = fast_exp2(p[3] - mn1);
+        const float e4 = fast_exp2(p[4] - mn0), e5 = fast_exp2(p[5] - mn0);
+        const float e6 = fast_exp2(p[6] - mn1), e7 = fast_exp2(p[7] - mn1);
+        pa[0] = pack_bf16x2(e0, e1);
+        pa[1] = pack_bf16x2(e2, e3);
+        pa[2] = pack_bf16x2(e4, e5);
+        pa[3] = pack_bf16x2(e6, e7);
+        // the row sums use the same bf16-rounded weights the PV product sees
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(pa);
+        const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+        const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+        ps0 = f0.x + f0.y + f2.x + f2.y;
+        ps1 = f1.x + f1.y + f3.x + f3.y;
+      }
+      l0 = l0 * a0 + ps0;
+      l1 = l1 * a1 + ps1;
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j) {
+        o[j][0] *= a0;
+        o[j][1] *= a0;
+        o[j][2] *= a1;
+        o[j][3] *= a1;
+      }
+      // ---- keys past the end of the request: zero their V rows (P is 0 there,
+      // but the pool may hold non-finite garbage and 0 * inf is NaN)
+      if (nv < kStageTokens) {
+        uint8_t* vrow = stages + stage * C::kStageBytes + C::kTensorBytes + hh * NH * C::kTile;
+        for (int idx = lane; idx < (kStageTokens - nv) * 8 * NH; idx += 32) {
+          const int dh = idx / ((kStageTokens - nv) * 8);
+          const int rem = idx % ((kStageTokens - nv) * 8);
+          const int key = nv + rem / 8, chunk = rem % 8;
+          *reinterpret_cast<uint4*>(vrow + dh * C::kTile + mmak::swz(key, chunk)) =
+              make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+      }
+      // ---- O += P V
+      {
+        const int mi = lane >> 3;
+        const int key = (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+        for (int n2 = 0; n2 < D / 16; ++n2) {
+          const int dh = n2 >> 2, c16 = n2 & 3;
+          const int chunk = 2 * c16 + (mi >> 1);
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4_trans(vt + dh * C::kTile + mmak::swz(key, chunk), b0, b1, b2, b3);
+          mma_bf16_16816(o[2 * n2], pa, b0, b1);
+          mma_bf16_16816(o[2 * n2 + 1], pa, b2, b3);
+        }
+      }
+      if (nv < kStageTokens) fence_proxy_async_smem();
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+
+    if (si.flags & mmak::kLast) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      const int r = si.qrow;
+      if (bad) {
+        if (lane == 0) {
+          ws.qrow_bad[r] = 1;
+          if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_BLOCK_OOB);
+        }
+      } else {
+        const int np = ws.nparts[r];
+        if (np == 1) {
+          const float i0 = 1.f / l0, i1 = 1.f / l1;
+          const int64_t ob = (static_cast<int64_t>(r) * g.num_heads + head) * D;
+          if (g.out_dtype == PA_F32) {
+            float* out = static_cast<float*>(g.out) + ob;
+#pragma unroll
+            for (int j = 0; j < D / 8; ++j) {
+              if (qr < G)
+                *reinterpret_cast<float2*>(out + qr * D + j * 8 + qc) =
+                    make_float2(o[j][0] * i0, o[j][1] * i0);
+              if (qr + 8 < G)
+                *reinterpret_cast<float2*>(out + (qr + 8) * D + j * 8 + qc) =
+                    make_float2(o[j][2] * i1, o[j][3] * i1);
+            }
+          } else {
+            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out) + ob;
+#pragma unroll
+            for (int j = 0; j < D / 8; ++j) {
+              if (qr < G)
+                *reinterpret_cast<uint32_t*>(out + qr * D + j * 8 + qc) =
+                    pack_bf16x2(o[j][0] * i0, o[j][1] * i0);
+              if (qr + 8 < G)
+                *reinterpret_cast<uint32_t*>(out + (qr + 8) * D + j * 8 + qc) =
+                    pack_bf16x2(o[j][2] * i1, o[j][3] * i1);
+            }
+          }
+        } else {
+          const int64_t slot0 = (static_cast<int64_t>(r) * g.num_heads + head) * ws.max_parts + si.part;
+          if (qr < G) {
+            const int64_t sl = slot0 + static_cast<int64_t>(qr) * ws.max_parts;
+            if ((lane & 3) == 0) ws.part_ml[sl] = make_float2(m0, l0);
+            float* po = ws.part_o + sl * D;
+#pragma unroll
+            for (int j = 0; j < D / 8; ++j)
+              *reinterpret_cast<float2*>(po + j * 8 + qc) = make_float2(o[j][0], o[j][1]);
+          }
+          if (qr + 8 < G) {
+            const int64_t sl = slot0 + static_cast<int64_t>(qr + 8) * ws.max_parts;
+            if ((lane & 3) == 0) ws.part_ml[sl] = make_float2(m1, l1);
+            float* po = ws.part_o + sl * D;
+#pragma unroll
+            for (int j = 0; j < D / 8; ++j)
+              *reinterpret_cast<float2*>(po + j * 8 + qc) = make_float2(o[j][2], o[j][3]);
+          }
+        }
+      }
+    }
+    if (++stage == NS) {
+      stage = 0;
+      phase ^= 1;
+    }
+  }
+}
+
+// ----------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [D, Hkv, num_blocks * block_size] bf16 view of a pool, box [64, 1, box_rows].
+static bool make_pool_map(CUtensorMap* m, const void* base, const AttnGeom& g, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(g.head_dim),
+                        static_cast<cuuint64_t>(g.num_kv_heads),
+                        static_cast<cuuint64_t>(g.num_blocks) * g.block_size};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.head_dim) * 2,
+                           static_cast<cuuint64_t>(g.head_dim) * g.num_kv_heads * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool mma_path_supported(const AttnGeom& g) {
+  const int G = g.num_kv_heads > 0 ? g.num_heads / g.num_kv_heads : 0;
+  const bool bs_ok = g.block_size == 8 || (g.block_size % 16 == 0 && g.block_size <= 256);
+  return g.dtype == PA_BF16 && (g.head_dim == 64 || g.head_dim == 128) && G >= 1 &&
+         G <= kMaxGroup && bs_ok && encode_fn() != nullptr &&
+         static_cast<int64_t>(g.num_blocks) * g.block_size < (1LL << 31);
+}
+
+template <int D, int HG>
+static cudaError_t launch_mma_t(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {
+  using C = mmak::Cfg<D, HG>;
+  const int box_rows = g.block_size < kStageTokens ? g.block_size : kStageTokens;
+  CUtensorMap tk, tv;
+  if (!make_pool_map(&tk, g.k_cache, g, box_rows) || !make_pool_map(&tv, g.v_cache, g, box_rows))
+    return cudaErrorInvalidValue;
+  auto kern = attn_mma_kernel<D, HG>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms * per_sm);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tk, tv, g, ws, box_rows);
+}
+
+cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,
+                            cudaStream_t s) {
+  if (g.head_dim == 128) {
+    switch (heads_per_group) {
+      case 8: return launch_mma_t<128, 8>(g, ws, num_sms, s);
+      case 4: return launch_mma_t<128, 4>(g, ws, num_sms, s);
+      case 2: return launch_mma_t<128, 2>(g, ws, num_sms, s);
+      default: return launch_mma_t<128, 1>(g, ws, num_sms, s);
+    }
+  }
+  switch (heads_per_group) {
+    case 8: return launch_mma_t<64, 8>(g, ws, num_sms, s);
+    case 4: return launch_mma_t<64, 4>(g, ws, num_sms, s);
+    case 2: return launch_mma_t<64, 2>(g, ws, num_sms, s);
+    default: return launch_mma_t<64, 1>(g, ws, num_sms, s);
+  }
+}
+
+}  // namespace pa

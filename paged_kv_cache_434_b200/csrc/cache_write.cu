@@ -1,0 +1,107 @@
+// cache_write.cu -- slot mapping and reshape_and_cache for the paged KV pools.
+//
+// "AI Infra入门干货总结：大模型是如何高效推理的", section "Paged Attention":
+// slot_idx = block_idx * block_size + block_offset; the kernel recovers
+// block_idx = slot / block_size and block_offset = slot % block_size.  With the
+// pool laid out [num_blocks, block_size, num_kv_heads, head_dim], the whole
+// [num_kv_heads, head_dim] row of a token is contiguous at element offset
+// slot * num_kv_heads * head_dim, so the scatter is one contiguous row copy per
+// token, done with 16-byte vector loads and stores.
+#include "internal.h"
+
+namespace pa {
+
+// One warp per request: tokens query_start_loc[b] .. [b+1]-1 are the request's
+// last q_b positions.  Invalid requests get slot -1 for all their tokens.
+__global__ void __launch_bounds__(256) slot_mapping_kernel(
+    const int32_t* __restrict__ block_tables, int32_t max_blocks,
+    const int32_t* __restrict__ qsl, const int32_t* __restrict__ seq_lens, int32_t num_seqs,
+    int64_t num_tokens, int32_t block_size, int64_t num_blocks, int64_t* __restrict__ slots,
+    int32_t* __restrict__ err) {
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (b >= num_seqs) return;
+  const int32_t t0 = qsl[b], t1 = qsl[b + 1];
+  const int32_t q_b = t1 - t0;
+  const int32_t L = seq_lens[b];
+  int32_t bits = 0;
+  if (q_b < 0 || q_b > L) bits |= PA_ERRBIT_QUERY_TOO_LONG;
+  if (L > max_blocks * block_size) bits |= PA_ERRBIT_SEQ_TOO_LONG;
+  if (t0 < 0) {
+    if (lane == 0 && err) atomicOr(err, PA_ERRBIT_QUERY_TOO_LONG);
+    return;
+  }
+  const int32_t* table = block_tables + static_cast<int64_t>(b) * max_blocks;
+  for (int32_t i = lane; i < q_b && t0 + static_cast<int64_t>(i) < num_tokens; i += 32) {
+    int64_t slot = -1;
+    if (bits == 0) {
+      const int32_t pos = L - q_b + i;
+      const int32_t phys = table[pos / block_size];
+      if (phys < 0 || phys >= num_blocks) {
+        bits |= PA_ERRBIT_BLOCK_OOB;
+      } else {
+        slot = static_cast<int64_t>(phys) * block_size + pos % block_size;
+      }
+    }
+    slots[t0 + i] = slot;
+  }
+  if (bits && err) atomicOr(err, bits);
+}
+
+// One warp per (token, K|V): copies row_bytes (a multiple of 16) with uint4.
+__global__ void __launch_bounds__(256) cache_write_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ kc,
+    uint4* __restrict__ vc, const int64_t* __restrict__ slots, int64_t num_tokens,
+    int64_t row_vec, int64_t num_slots, int32_t* __restrict__ err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t t = w >> 1;
+  if (t >= num_tokens) return;
+  const int64_t slot = slots[t];
+  if (slot < 0) return;  // padding token
+  if (slot >= num_slots) {
+    if (lane == 0 && (w & 1) == 0 && err) atomicOr(err, PA_ERRBIT_SLOT_OOB);
+    return;
+  }
+  const uint4* src = ((w & 1) ? v : k) + t * row_vec;
+  uint4* dst = ((w & 1) ? vc : kc) + slot * row_vec;
+  int64_t i = lane;
+  // 4 independent 16-byte loads in flight per lane before the stores
+  for (; i + 96 < row_vec; i += 128) {
+    uint4 a = __ldg(src + i), b = __ldg(src + i + 32), c = __ldg(src + i + 64),
+          d = __ldg(src + i + 96);
+    dst[i] = a;
+    dst[i + 32] = b;
+    dst[i + 64] = c;
+    dst[i + 96] = d;
+  }
+  for (; i < row_vec; i += 32) dst[i] = __ldg(src + i);
+}
+
+cudaError_t launch_slot_mapping(const int32_t* block_tables, int32_t max_blocks,
+                                const int32_t* qsl, const int32_t* seq_lens, int32_t num_seqs,
+                                int64_t num_tokens, int32_t block_size, int64_t num_blocks,
+                                int64_t* slots, int32_t* err, cudaStream_t s) {
+  if (num_seqs == 0) return cudaSuccess;
+  const int warps = 8;
+  dim3 grid((num_seqs + warps - 1) / warps);
+  slot_mapping_kernel<<<grid, warps * 32, 0, s>>>(block_tables, max_blocks, qsl, seq_lens,
+                                                  num_seqs, num_tokens, block_size, num_blocks,
+                                                  slots, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cache_write(const void* k, const void* v, void* kc, void* vc,
+                               const int64_t* slots, int64_t num_tokens, int64_t row_bytes,
+                               int64_t num_slots, int32_t* err, cudaStream_t s) {
+  if (num_tokens == 0) return cudaSuccess;
+  const int warps = 8;
+  const int64_t nwarps = 2 * num_tokens;
+  dim3 grid(static_cast<unsigned>((nwarps + warps - 1) / warps));
+  cache_write_kernel<<<grid, warps * 32, 0, s>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(kc),
+      static_cast<uint4*>(vc), slots, num_tokens, row_bytes / 16, num_slots, err);
+  return cudaGetLastError();
+}
+
+}  // namespace pa

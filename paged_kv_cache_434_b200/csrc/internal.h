@@ -1,0 +1,105 @@
+// internal.h -- structures shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/pa.h"
+
+namespace pa {
+
+constexpr int kStageTokens = 16;     // keys per pipeline stage / partition granule
+constexpr int kMaxGroup = 16;        // query heads per KV head handled in one tile
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
+
+// ---------------------------------------------------------------- workspace
+// One attention call's scratch, carved from the caller's workspace buffer.
+//   ctrl      int32[64]   [0] dynamic work counter, [1] number of items,
+//                         [2] partition length in tokens, [3] tile counter,
+//                         [4] number of prefill tiles
+//   qrow_info int4[R]     {request b, key_len, valid, first_key_pos}
+//   nparts    int32[R]    partitions of the row (0: empty -> zero row;
+//                         -1: invalid -> row left unwritten)
+//   qrow_bad  int32[R]    set when a block id outside the pool was met
+//   items     int4[I]     {qrow, head group, partition, 0}
+//   part_ml   float2[R*H*P]   per (row, query head, partition): (m, l),
+//                         m in log2 units (score * scale * log2 e)
+//   part_o    float[R*H*P*D]  unnormalised partial outputs
+//   tiles     int4[Tl]    prefill tiles {request b, kv head, first query row, rows}
+struct WsLayout {
+  size_t ctrl, qrow_info, nparts, qrow_bad, items, part_ml, part_o, tiles, total;
+  int64_t num_qrows, max_parts, max_items, max_tiles;
+};
+
+struct WsView {
+  int32_t* ctrl;
+  int4* qrow_info;
+  int32_t* nparts;
+  int32_t* qrow_bad;
+  int4* items;
+  float2* part_ml;
+  float* part_o;
+  int4* tiles;
+  int64_t max_parts;
+  int64_t max_items;
+  int64_t max_tiles;
+};
+
+WsLayout ws_layout(int64_t num_qrows, int num_heads, int head_dim, int head_groups,
+                   int64_t max_parts, int64_t max_tiles);
+WsView ws_view(void* base, const WsLayout& L);
+
+// ---------------------------------------------------------------- geometry
+struct AttnGeom {
+  const void* q;          // [R, Hq, D]
+  const void* k_cache;    // [NB, bs, Hkv, D]
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  const int32_t* query_start_loc;  // nullptr for decode
+  void* out;              // [R, Hq, D]
+  int64_t num_blocks;
+  int32_t num_seqs;
+  int32_t num_qrows;
+  int32_t num_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t block_size;
+  int32_t max_blocks;
+  int32_t dtype;          // pa_dtype of q / caches
+  int32_t out_dtype;
+  float scale_log2;       // scale * log2(e)
+  int32_t* err_word;
+};
+
+// ---------------------------------------------------------------- planner
+struct PlanArgs {
+  int32_t head_groups;      // items per (row, partition)
+  int32_t heads_per_group;  // KV heads per item
+  int32_t target_items;     // aim for about this many items in total
+  int32_t min_part_stages;  // lower bound of a partition, in 16-key stages
+  int32_t expand_prefill;   // 1: every query of a q_b>1 request is its own row
+};
+
+// ---------------------------------------------------------------- launchers
+// Each returns cudaSuccess or the launch error.
+cudaError_t launch_slot_mapping(const int32_t* block_tables, int32_t max_blocks,
+                                const int32_t* qsl, const int32_t* seq_lens, int32_t num_seqs,
+                                int64_t num_tokens, int32_t block_size, int64_t num_blocks,
+                                int64_t* slots, int32_t* err, cudaStream_t s);
+cudaError_t launch_cache_write(const void* k, const void* v, void* kc, void* vc,
+                               const int64_t* slots, int64_t num_tokens, int64_t row_bytes,
+                               int64_t num_slots, int32_t* err, cudaStream_t s);
+cudaError_t launch_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws, cudaStream_t s);
+cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms,
+                                cudaStream_t s);
+cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,
+                            cudaStream_t s);
+cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, cudaStream_t s);
+
+bool mma_path_supported(const AttnGeom& g);
+int device_num_sms();
+
+}  // namespace pa

@@ -1,0 +1,280 @@
+// pa_api.cu -- the extern "C" entry points declared in include/pa.h.
+//
+// Host side only: validates arguments, sizes and carves the workspace, picks the
+// kernel path and enqueues the launches.  No allocation, no host<->device
+// synchronisation except in pa_read_error.
+#include <cstdio>
+#include <cstring>
+
+#include "internal.h"
+
+namespace pa {
+
+int device_num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+  if (dev < 64 && cache[dev]) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static pa_status check_cache(const pa_cache_desc* c) {
+  if (!c) return PA_ERR_INVALID_ARG;
+  if (c->num_blocks < 1 || c->num_kv_heads < 1) return PA_ERR_INVALID_ARG;
+  const int bs = c->block_size;
+  if (!(bs == 8 || bs == 16 || bs == 32 || bs == 64 || bs == 128 || bs == 256))
+    return PA_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (c->dtype != PA_F32 && c->dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+static int elt_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+
+// Launch plan of one attention call (decode or mixed step); identical in the
+// workspace-size query and in the call itself.
+struct AttnPlan {
+  bool use_mma;
+  int heads_per_group;
+  int head_groups;
+  int num_sms;
+  int64_t num_qrows;
+  int64_t max_parts;
+  int target_items;
+  int64_t max_tiles;
+};
+
+static AttnPlan make_plan(int64_t num_qrows, int num_heads, int max_blocks,
+                          const pa_cache_desc* c, bool bf16_fast_ok) {
+  AttnPlan p{};
+  AttnGeom probe{};
+  probe.num_heads = num_heads;
+  probe.num_kv_heads = c->num_kv_heads;
+  probe.head_dim = c->head_dim;
+  probe.block_size = c->block_size;
+  probe.dtype = c->dtype;
+  probe.num_blocks = c->num_blocks;
+  p.use_mma = bf16_fast_ok && mma_path_supported(probe);
+  if (p.use_mma) {
+    int hg = 8;
+    while (c->num_kv_heads % hg) hg >>= 1;
+    p.heads_per_group = hg;
+  } else {
+    p.heads_per_group = 1;
+  }
+  p.head_groups = c->num_kv_heads / p.heads_per_group;
+  p.num_sms = device_num_sms();
+  if (p.num_sms <= 0) p.num_sms = 148;
+  p.num_qrows = num_qrows;
+  p.target_items = p.num_sms * (p.use_mma ? 8 : 16);
+  const int64_t max_units =
+      (static_cast<int64_t>(max_blocks) * c->block_size + kStageTokens - 1) / kStageTokens;
+  const int64_t denom = num_qrows * p.head_groups;
+  int64_t mp = denom > 0 ? (p.target_items + denom - 1) / denom : 1;
+  if (mp > max_units) mp = max_units;
+  if (mp < 1) mp = 1;
+  p.max_parts = mp;
+  p.max_tiles = 0;
+  return p;
+}
+
+static AttnGeom make_geom(const void* q, const void* kc, const void* vc, const int32_t* bt,
+                          const int32_t* sl, const int32_t* qsl, float scale, void* out,
+                          int32_t num_seqs, int64_t num_qrows, int32_t num_heads,
+                          int32_t max_blocks, int32_t out_dtype, const pa_cache_desc* c,
+                          int32_t* err) {
+  AttnGeom g{};
+  g.q = q;
+  g.k_cache = kc;
+  g.v_cache = vc;
+  g.block_tables = bt;
+  g.seq_lens = sl;
+  g.query_start_loc = qsl;
+  g.out = out;
+  g.num_blocks = c->num_blocks;
+  g.num_seqs = num_seqs;
+  g.num_qrows = static_cast<int32_t>(num_qrows);
+  g.num_heads = num_heads;
+  g.num_kv_heads = c->num_kv_heads;
+  g.head_dim = c->head_dim;
+  g.block_size = c->block_size;
+  g.max_blocks = max_blocks;
+  g.dtype = c->dtype;
+  g.out_dtype = out_dtype;
+  g.scale_log2 = scale * 1.4426950408889634f;
+  g.err_word = err;
+  return g;
+}
+
+static pa_status check_attn_args(int32_t num_seqs, int64_t num_qrows, int32_t num_heads,
+                                  int32_t max_blocks, int32_t out_dtype,
+                                  const pa_cache_desc* c) {
+  pa_status st = check_cache(c);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_qrows < 0 || num_qrows > (1LL << 30) || max_blocks < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_heads < 1 || num_heads % c->num_kv_heads) return PA_ERR_INVALID_ARG;
+  if (num_heads / c->num_kv_heads > kMaxGroup) return PA_ERR_UNSUPPORTED;
+  if (out_dtype != PA_F32 && out_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(max_blocks) * c->block_size > (1LL << 30)) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* workspace,
+                               size_t ws_bytes, int expand_prefill, cudaStream_t s) {
+  const WsLayout L = ws_layout(p.num_qrows, g.num_heads, g.head_dim, p.head_groups, p.max_parts,
+                               p.max_tiles);
+  if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PA_ERR_WORKSPACE;
+  if (g.num_qrows == 0 || g.num_seqs == 0) return PA_OK;
+  const WsView ws = ws_view(workspace, L);
+  PlanArgs a{};
+  a.head_groups = p.head_groups;
+  a.heads_per_group = p.heads_per_group;
+  a.target_items = p.target_items;
+  a.min_part_stages = 2;
+  a.expand_prefill = expand_prefill;
+  if (launch_plan(g, a, ws, s) != cudaSuccess) return PA_ERR_CUDA;
+  cudaError_t e = p.use_mma ? launch_attn_mma(g, ws, p.num_sms, p.heads_per_group, s)
+                            : launch_attn_generic(g, ws, p.num_sms, s);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (launch_merge(g, ws, s) != cudaSuccess) return PA_ERR_CUDA;
+  return PA_OK;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char* pa_status_str(int status) {
+  switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case PA_ERR_CUDA: return "CUDA runtime error";
+    case PA_ERR_DEVICE: return "device reported error bits";
+    default: return "unknown status";
+  }
+}
+
+int pa_version(void) { return 100; }
+
+pa_status pa_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                          const int32_t* query_start_loc, const int32_t* seq_lens,
+                          int32_t num_seqs, int64_t num_tokens, int32_t block_size,
+                          int64_t num_blocks, int64_t* slot_mapping, int32_t* err_word,
+                          void* stream) {
+  if (num_seqs < 0 || num_tokens < 0 || max_blocks_per_seq < 0 || block_size < 1 ||
+      num_blocks < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+  if (!block_tables || !query_start_loc || !seq_lens || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_blocks_per_seq) * block_size > (1LL << 30))
+    return PA_ERR_UNSUPPORTED;
+  cudaError_t e = launch_slot_mapping(block_tables, max_blocks_per_seq, query_start_loc, seq_lens,
+                                      num_seqs, num_tokens, block_size, num_blocks, slot_mapping,
+                                      err_word, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_cache_write(const void* k, const void* v, void* key_cache, void* value_cache,
+                         const int64_t* slot_mapping, int64_t num_tokens,
+                         const pa_cache_desc* cache, int32_t* err_word, void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_INVALID_ARG;
+  const int64_t row_bytes =
+      static_cast<int64_t>(cache->num_kv_heads) * cache->head_dim * elt_bytes(cache->dtype);
+  cudaError_t e = launch_cache_write(k, v, key_cache, value_cache, slot_mapping, num_tokens,
+                                     row_bytes, cache->num_blocks * cache->block_size, err_word,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t max_blocks_per_seq,
+                                const pa_cache_desc* cache) {
+  if (check_attn_args(num_seqs, num_seqs, num_heads, max_blocks_per_seq, PA_F32, cache) != PA_OK)
+    return 0;
+  const AttnPlan p = make_plan(num_seqs, num_heads, max_blocks_per_seq, cache, true);
+  return ws_layout(p.num_qrows, num_heads, cache->head_dim, p.head_groups, p.max_parts,
+                   p.max_tiles)
+      .total;
+}
+
+pa_status pa_decode(const void* q, const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, const int32_t* seq_lens, float scale,
+                    void* out, int32_t num_seqs, int32_t num_heads, int32_t max_blocks_per_seq,
+                    int32_t out_dtype, const pa_cache_desc* cache, void* workspace,
+                    size_t workspace_bytes, int32_t* err_word, void* stream) {
+  pa_status st =
+      check_attn_args(num_seqs, num_seqs, num_heads, max_blocks_per_seq, out_dtype, cache);
+  if (st != PA_OK) return st;
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !key_cache || !value_cache || !block_tables || !seq_lens || !out)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  const AttnPlan p = make_plan(num_seqs, num_heads, max_blocks_per_seq, cache, true);
+  const AttnGeom g = make_geom(q, key_cache, value_cache, block_tables, seq_lens, nullptr, scale,
+                               out, num_seqs, num_seqs, num_heads, max_blocks_per_seq, out_dtype,
+                               cache, err_word);
+  return run_attention(g, p, workspace, workspace_bytes, 1, static_cast<cudaStream_t>(stream));
+}
+
+size_t pa_mixed_step_workspace_size(int32_t num_seqs, int64_t num_tokens, int32_t num_heads,
+                                    int32_t max_blocks_per_seq, const pa_cache_desc* cache) {
+  if (check_attn_args(num_seqs, num_tokens, num_heads, max_blocks_per_seq, PA_F32, cache) !=
+      PA_OK)
+    return 0;
+  const AttnPlan p = make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true);
+  return ws_layout(p.num_qrows, num_heads, cache->head_dim, p.head_groups, p.max_parts,
+                   p.max_tiles)
+      .total;
+}
+
+pa_status pa_mixed_step(const void* q, const void* key_cache, const void* value_cache,
+                        const int32_t* block_tables, const int32_t* query_start_loc,
+                        const int32_t* seq_lens, float scale, void* out, int32_t num_seqs,
+                        int64_t num_tokens, int32_t num_heads, int32_t max_blocks_per_seq,
+                        int32_t out_dtype, const pa_cache_desc* cache, void* workspace,
+                        size_t workspace_bytes, int32_t* err_word, void* stream) {
+  pa_status st =
+      check_attn_args(num_seqs, num_tokens, num_heads, max_blocks_per_seq, out_dtype, cache);
+  if (st != PA_OK) return st;
+  if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+  if (!q || !key_cache || !value_cache || !block_tables || !query_start_loc || !seq_lens || !out)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  const AttnPlan p = make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true);
+  const AttnGeom g = make_geom(q, key_cache, value_cache, block_tables, seq_lens,
+                               query_start_loc, scale, out, num_seqs, num_tokens, num_heads,
+                               max_blocks_per_seq, out_dtype, cache, err_word);
+  return run_attention(g, p, workspace, workspace_bytes, 1, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_read_error(int32_t* err_word, int32_t* host_bits, void* stream) {
+  if (!err_word || !host_bits) return PA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, err_word, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaMemsetAsync(err_word, 0, sizeof(int32_t), s) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
+  *host_bits = h;
+  return h ? PA_ERR_DEVICE : PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,33 @@
+"""One layer's attention step over the paged cache: the three library calls in
+the order the vLLM v1 walkthrough gives them ("AI Infra入门干货总结：大模型是如何
+高效推理的", "Reshape & Cache" then "Attention"): compute the new tokens'
+slots, scatter their K/V into the pools, then attend through the block tables.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import binding
+
+
+def step(q, k_new, v_new, k_cache, v_cache, block_tables, query_start_loc, seq_lens,
+         scale: float, *, decode_only: bool = False, out=None, out_dtype=torch.float32,
+         slots=None, workspace=None, err=None):
+    """Run slot_mapping -> cache_write -> decode / mixed_step on the current stream.
+
+    q: [T, Hq, D]; k_new, v_new: [T, Hkv, D]; query_start_loc: [B+1] int32;
+    seq_lens: [B] int32 (lengths after this step).  With decode_only=True every
+    request has exactly one new token (T == B) and pa_decode is used.
+    Returns out [T, Hq, D].
+    """
+    T = q.shape[0]
+    nb, bs = k_cache.shape[0], k_cache.shape[1]
+    slots = binding.slot_mapping(block_tables, query_start_loc, seq_lens, bs, nb, T, out=slots,
+                                 err=err)
+    binding.cache_write(k_new, v_new, k_cache, v_cache, slots, err=err)
+    if decode_only:
+        return binding.decode(q, k_cache, v_cache, block_tables, seq_lens, scale, out=out,
+                              out_dtype=out_dtype, workspace=workspace, err=err)
+    return binding.mixed_step(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, scale,
+                              out=out, out_dtype=out_dtype, workspace=workspace, err=err)

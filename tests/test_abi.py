@@ -1,0 +1,144 @@
+"""The C-ABI library loads and exports what include/pa.h declares; host-side
+argument validation returns status codes without touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_434_b200 import binding
+    if not os.path.exists(binding.library_path()):
+        from paged_kv_cache_434_b200 import build
+        build.build()
+    return binding._lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("pa_cache_write", "pa_decode", "pa_mixed_step", "pa_slot_mapping",
+              "pa_read_error", "pa_decode_workspace_size", "pa_mixed_step_workspace_size",
+              "pa_status_str", "pa_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(os.path.join(ROOT, "paged_kv_cache_434_b200", "lib", "libpa_b200.so"))
+    missing = [n for n in _declared() if not hasattr(raw, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_export():
+    from paged_kv_cache_434_b200 import binding
+    assert sorted(binding.EXPORTS) == sorted(_declared())
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.pa_status_str(s)
+    assert lib.pa_status_str(99) == b"unknown status"
+    assert lib.pa_version() >= 100
+
+
+def _desc(**kw):
+    from paged_kv_cache_434_b200.binding import CacheDesc
+    d = dict(num_blocks=16, block_size=16, num_kv_heads=2, head_dim=64, dtype=0)
+    d.update(kw)
+    return CacheDesc(**d)
+
+
+def test_cache_write_validation(lib):
+    from paged_kv_cache_434_b200 import binding as B
+    d = _desc()
+    # null pointers
+    assert lib.pa_cache_write(None, None, None, None, None, 4, ctypes.byref(d), None, None) == \
+        B.PA_ERR_INVALID_ARG
+    # zero tokens is a no-op
+    assert lib.pa_cache_write(None, None, None, None, None, 0, ctypes.byref(d), None, None) == B.PA_OK
+    # unsupported geometry
+    for bad in (dict(head_dim=96), dict(block_size=12), dict(dtype=7)):
+        assert lib.pa_cache_write(None, None, None, None, None, 1, ctypes.byref(_desc(**bad)),
+                                  None, None) == B.PA_ERR_UNSUPPORTED
+    assert lib.pa_cache_write(None, None, None, None, None, 1, None, None, None) == \
+        B.PA_ERR_INVALID_ARG
+    # misaligned device pointer (never dereferenced: rejected on the host)
+    assert lib.pa_cache_write(8, 16, 16, 16, 16, 1, ctypes.byref(d), None, None) == \
+        B.PA_ERR_INVALID_ARG
+
+
+def test_attention_validation(lib):
+    from paged_kv_cache_434_b200 import binding as B
+    d = _desc()
+    # num_heads not a multiple of num_kv_heads
+    assert lib.pa_decode(16, 16, 16, 16, 16, 0.1, 16, 2, 3, 4, 0, ctypes.byref(d), 256, 1 << 20,
+                         None, None) == B.PA_ERR_INVALID_ARG
+    # group larger than 16 query heads per KV head
+    assert lib.pa_decode(16, 16, 16, 16, 16, 0.1, 16, 2, 64, 4, 0, ctypes.byref(d), 256, 1 << 20,
+                         None, None) == B.PA_ERR_UNSUPPORTED
+    # bad out dtype
+    assert lib.pa_decode(16, 16, 16, 16, 16, 0.1, 16, 2, 8, 4, 5, ctypes.byref(d), 256, 1 << 20,
+                         None, None) == B.PA_ERR_UNSUPPORTED
+    # null tensors
+    assert lib.pa_decode(None, 16, 16, 16, 16, 0.1, 16, 2, 8, 4, 0, ctypes.byref(d), 256,
+                         1 << 20, None, None) == B.PA_ERR_INVALID_ARG
+    # workspace too small / missing / misaligned
+    assert lib.pa_decode(16, 16, 16, 16, 16, 0.1, 16, 2, 8, 4, 0, ctypes.byref(d), 256, 16,
+                         None, None) == B.PA_ERR_WORKSPACE
+    assert lib.pa_decode(16, 16, 16, 16, 16, 0.1, 16, 2, 8, 4, 0, ctypes.byref(d), None,
+                         1 << 20, None, None) == B.PA_ERR_WORKSPACE
+    assert lib.pa_decode(16, 16, 16, 16, 16, 0.1, 16, 2, 8, 4, 0, ctypes.byref(d), 272,
+                         1 << 20, None, None) == B.PA_ERR_WORKSPACE
+    assert lib.pa_mixed_step(16, 16, 16, 16, None, 16, 0.1, 16, 2, 5, 8, 4, 0, ctypes.byref(d),
+                             256, 1 << 20, None, None) == B.PA_ERR_INVALID_ARG
+    # zero requests is a no-op
+    assert lib.pa_decode(None, None, None, None, None, 0.1, None, 0, 8, 4, 0, ctypes.byref(d),
+                         None, 0, None, None) == B.PA_OK
+
+
+def test_workspace_sizes_are_positive_and_monotone(lib):
+    d = _desc(num_kv_heads=8, head_dim=128, dtype=1)
+    a = lib.pa_decode_workspace_size(64, 32, 512, ctypes.byref(d))
+    b = lib.pa_decode_workspace_size(128, 32, 512, ctypes.byref(d))
+    assert 0 < a <= b
+    assert lib.pa_decode_workspace_size(64, 33, 512, ctypes.byref(d)) == 0
+    m = lib.pa_mixed_step_workspace_size(4098, 8192, 32, 384, ctypes.byref(d))
+    assert m > 0
+
+
+def test_slot_mapping_validation(lib):
+    from paged_kv_cache_434_b200 import binding as B
+    assert lib.pa_slot_mapping(None, 3, None, None, 2, 5, 16, 16, None, None, None) == \
+        B.PA_ERR_INVALID_ARG
+    assert lib.pa_slot_mapping(None, 3, None, None, 0, 0, 16, 16, None, None, None) == B.PA_OK
+    assert lib.pa_slot_mapping(16, 3, 16, 16, 2, 5, 0, 16, 16, None, None) == B.PA_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_cpu_fallback():
+    """Calls on CPU tensors raise instead of computing anything on the host."""
+    import torch
+    import paged_kv_cache_434_b200 as P
+    kc = torch.zeros(4, 16, 2, 64)
+    with pytest.raises(ValueError):
+        P.decode(torch.zeros(1, 8, 64), kc, kc, torch.zeros(1, 1, dtype=torch.int32),
+                 torch.ones(1, dtype=torch.int32), 0.1)
+
+
+def test_product_code_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "paged_kv_cache_434_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in text and "from oracle" not in text, f
