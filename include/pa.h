@@ -164,6 +164,31 @@ pa_status pa_mixed_step(const void* q, const void* key_cache, const void* value_
                         size_t workspace_bytes, int32_t* err_word, void* stream);
 
 /*
+ * pa_decode_no_alloc -- pa_decode without a caller-provided workspace.
+ * The pages have no counterpart: this entry point exists for callers that
+ * can't allocate device memory (a plug-in inside a host engine that owns all
+ * device allocations and hands it no workspace; a runtime that forbids
+ * cudaMalloc after start-up).  Its scratch is a static device array of
+ * PA_DECODE_NO_ALLOC_MAX_BYTES that every GPU loading this library holds
+ * until the process exits; the call itself allocates nothing.
+ *   Arguments, layouts and results: exactly those of pa_decode (same kernels,
+ *   same partition plan), minus workspace / workspace_bytes.
+ *   Returns PA_ERR_WORKSPACE when pa_decode_workspace_size(...) for these
+ *   sizes exceeds PA_DECODE_NO_ALLOC_MAX_BYTES (nothing is launched).
+ *   The first call on a device looks up the array's address on that device
+ *   (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   stream capture.  All calls share the array: two calls whose kernels
+ *   overlap on the GPU race.  Nothing in it needs clearing between calls.
+ */
+#define PA_DECODE_NO_ALLOC_MAX_BYTES (32u << 20) /* 32 MiB of device memory per GPU */
+
+pa_status pa_decode_no_alloc(const void* q, const void* key_cache, const void* value_cache,
+                             const int32_t* block_tables, const int32_t* seq_lens, float scale,
+                             void* out, int32_t num_seqs, int32_t num_heads,
+                             int32_t max_blocks_per_seq, int32_t out_dtype,
+                             const pa_cache_desc* cache, int32_t* err_word, void* stream);
+
+/*
  * pa_read_error -- synchronise `stream`, copy *err_word to *host_bits and
  * reset it to 0.  Returns PA_OK when no bit was set, PA_ERR_DEVICE when some
  * were, PA_ERR_CUDA if a CUDA call failed (e.g. an earlier kernel faulted).

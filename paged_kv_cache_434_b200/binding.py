@@ -27,7 +27,7 @@ ERRBIT_TIMEOUT = 0x10
 
 EXPORTS = ("pa_status_str", "pa_version", "pa_slot_mapping", "pa_cache_write",
            "pa_decode_workspace_size", "pa_decode", "pa_mixed_step_workspace_size",
-           "pa_mixed_step", "pa_read_error")
+           "pa_mixed_step", "pa_read_error", "pa_decode_no_alloc")
 
 
 class PagedAttentionError(RuntimeError):
@@ -60,7 +60,12 @@ _SIGNATURES = {
     "pa_mixed_step": ([_vp, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i64, _i32, _i32, _i32,
                        _desc_p, _vp, _sz, _vp, _vp], ctypes.c_int),
     "pa_read_error": ([_vp, ctypes.POINTER(ctypes.c_int32), _vp], ctypes.c_int),
+    "pa_decode_no_alloc": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i32, _i32, _i32, _desc_p,
+                            _vp, _vp], ctypes.c_int),
 }
+
+# Size of the library's static scratch used by decode_no_alloc (PA_DECODE_NO_ALLOC_MAX_BYTES).
+DECODE_NO_ALLOC_MAX_BYTES = 32 << 20
 
 
 def library_path() -> str:
@@ -245,4 +250,26 @@ def mixed_step(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, sca
         _cuda(seq_lens, "seq_lens", torch.int32, 1), float(scale), _cuda(out, "out"), B, T, H, W,
         _dt(out), ctypes.byref(desc), _cuda(ws, "workspace"), ws.numel() * ws.element_size(),
         _err_ptr(err), _stream()), "pa_mixed_step")
+    return out
+
+
+def decode_no_alloc(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out,
+                    err=None):
+    """pa_decode_no_alloc: decode attention for callers that can't allocate
+    device memory (e.g. a plug-in inside an engine that owns all allocations).
+
+    Same arguments and results as decode(), except that there is no workspace:
+    the library uses its own static device scratch of DECODE_NO_ALLOC_MAX_BYTES
+    and rejects larger problems with PagedAttentionError (PA_ERR_WORKSPACE).
+    `out` must be given, so that this call allocates nothing either.  Calls
+    whose kernels overlap on the GPU share the scratch and race.
+    """
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out.dtype)
+    B, H, D = q.shape
+    W = block_tables.shape[1]
+    _check(_lib().pa_decode_no_alloc(
+        _cuda(q, "q"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
+        _cuda(block_tables, "block_tables", torch.int32, 2),
+        _cuda(seq_lens, "seq_lens", torch.int32, 1), float(scale), _cuda(out, "out"), B, H, W,
+        _dt(out), ctypes.byref(desc), _err_ptr(err), _stream()), "pa_decode_no_alloc")
     return out
