@@ -7,11 +7,13 @@
 //
 // Layout and work split
 //   * Pools are [num_blocks, block_size, Hkv, D] bf16.  A stage is 16
-//     consecutive keys of one request: for each of the HG KV heads of the
-//     item's head group and each 64-column half of D, a TMA box of
-//     [16 keys x 64 dims] (2 KiB, 128-byte swizzle) is copied from the
-//     physical block the block table names.  16 keys never straddle a
-//     block when block_size >= 16; block_size 8 takes two boxes per stage.
+//     consecutive keys of one request.  In shared memory each (64-column
+//     half of D, KV head) pair holds a [16 keys x 64 dims] tile (2 KiB,
+//     128-byte swizzle), tiles of one half stored head after head.  With
+//     block_size >= 16 the tensor map walks (dim, token, head), so ONE TMA box
+//     [64 dims x 16 tokens x HG heads] fills a whole half (16 KiB per copy, 4
+//     copies per stage); with block_size 8 a stage spans two blocks and each
+//     head's tile takes two [64 x 8] boxes from a (dim, head, token) map.
 //   * A persistent CTA = HG consumer warps (warp w owns KV head w of the
 //     group) + 1 producer warp.  The producer pulls items from a global
 //     counter, walks their block tables and keeps NS stages in flight
@@ -68,7 +70,7 @@ __device__ __forceinline__ uint32_t swz(int key, int chunk) {
 template <int D, int HG>
 __global__ void __launch_bounds__((HG + 1) * 32, 1)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                    AttnGeom g, WsView ws, int box_rows) {
+                    AttnGeom g, WsView ws, int box_rows, int heads_per_box) {
   using C = mmak::Cfg<D, HG>;
   constexpr int NS = C::NS;
   constexpr int NH = C::NH;
@@ -153,18 +155,31 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           uint8_t* kbase = stages + stage * C::kStageBytes;
           uint8_t* vbase = kbase + C::kTensorBytes;
           const int head0 = item.y * HG;
-#pragma unroll
-          for (int hh = 0; hh < HG; ++hh) {
+          if (heads_per_box == HG) {
+            // (dim, token, head) map: one box per half and tensor
 #pragma unroll
             for (int dh = 0; dh < NH; ++dh) {
-              const int toff = (hh * NH + dh) * C::kTile;
-              tma_load_3d_hint(kbase + toff, &tmK, &full[stage], dh * 64, head0 + hh, rows0, policy);
-              tma_load_3d_hint(vbase + toff, &tmV, &full[stage], dh * 64, head0 + hh, rows0, policy);
-              if (rows1 >= 0) {
-                tma_load_3d_hint(kbase + toff + box_bytes, &tmK, &full[stage], dh * 64, head0 + hh,
-                                 rows1, policy);
-                tma_load_3d_hint(vbase + toff + box_bytes, &tmV, &full[stage], dh * 64, head0 + hh,
-                                 rows1, policy);
+              const int toff = dh * HG * C::kTile;
+              tma_load_3d_hint(kbase + toff, &tmK, &full[stage], dh * 64, rows0, head0, policy);
+              tma_load_3d_hint(vbase + toff, &tmV, &full[stage], dh * 64, rows0, head0, policy);
+            }
+          } else {
+            // (dim, head, token) map: one box per head, half, tensor and block
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) {
+#pragma unroll
+              for (int dh = 0; dh < NH; ++dh) {
+                const int toff = (dh * HG + hh) * C::kTile;
+                tma_load_3d_hint(kbase + toff, &tmK, &full[stage], dh * 64, head0 + hh, rows0,
+                                 policy);
+                tma_load_3d_hint(vbase + toff, &tmV, &full[stage], dh * 64, head0 + hh, rows0,
+                                 policy);
+                if (rows1 >= 0) {
+                  tma_load_3d_hint(kbase + toff + box_bytes, &tmK, &full[stage], dh * 64,
+                                   head0 + hh, rows1, policy);
+                  tma_load_3d_hint(vbase + toff + box_bytes, &tmV, &full[stage], dh * 64,
+                                   head0 + hh, rows1, policy);
+                }
               }
             }
           }
@@ -224,8 +239,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     if (si.flags & mmak::kBad) {
       bad = true;
     } else {
-      const uint32_t kt = smem_u32(stages + stage * C::kStageBytes) + hh * NH * C::kTile;
+      const uint32_t kt = smem_u32(stages + stage * C::kStageBytes) + hh * C::kTile;
       const uint32_t vt = kt + C::kTensorBytes;
+      constexpr uint32_t kHalf = HG * C::kTile;  // distance between the two halves
       // ---- S = Q K^T over 16 keys
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
       {
@@ -236,7 +252,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           const int dh = kk >> 2, c16 = kk & 3;
           const int chunk = 2 * c16 + (mi & 1);
           uint32_t b0, b1, b2, b3;
-          ldmatrix_x4(kt + dh * C::kTile + mmak::swz(key, chunk), b0, b1, b2, b3);
+          ldmatrix_x4(kt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
           mma_bf16_16816(s0, qa[kk], b0, b1);
           mma_bf16_16816(s1, qa[kk], b2, b3);
         }
@@ -290,12 +306,12 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       // ---- keys past the end of the request: zero their V rows (P is 0 there,
       // but the pool may hold non-finite garbage and 0 * inf is NaN)
       if (nv < kStageTokens) {
-        uint8_t* vrow = stages + stage * C::kStageBytes + C::kTensorBytes + hh * NH * C::kTile;
+        uint8_t* vrow = stages + stage * C::kStageBytes + C::kTensorBytes + hh * C::kTile;
         for (int idx = lane; idx < (kStageTokens - nv) * 8 * NH; idx += 32) {
           const int dh = idx / ((kStageTokens - nv) * 8);
           const int rem = idx % ((kStageTokens - nv) * 8);
           const int key = nv + rem / 8, chunk = rem % 8;
-          *reinterpret_cast<uint4*>(vrow + dh * C::kTile + mmak::swz(key, chunk)) =
+          *reinterpret_cast<uint4*>(vrow + dh * HG * C::kTile + mmak::swz(key, chunk)) =
               make_uint4(0, 0, 0, 0);
         }
         __syncwarp();
@@ -309,7 +325,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           const int dh = n2 >> 2, c16 = n2 & 3;
           const int chunk = 2 * c16 + (mi >> 1);
           uint32_t b0, b1, b2, b3;
-          ldmatrix_x4_trans(vt + dh * C::kTile + mmak::swz(key, chunk), b0, b1, b2, b3);
+          ldmatrix_x4_trans(vt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
           mma_bf16_16816(o[2 * n2], pa, b0, b1);
           mma_bf16_16816(o[2 * n2 + 1], pa, b2, b3);
         }
@@ -407,16 +423,26 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [D, Hkv, num_blocks * block_size] bf16 view of a pool, box [64, 1, box_rows].
-static bool make_pool_map(CUtensorMap* m, const void* base, const AttnGeom& g, int box_rows) {
+// Pool views for TMA.  heads_per_box == 1: (dim, head, token) with box
+// [64, 1, box_rows]; heads_per_box > 1: (dim, token, head) with box
+// [64, 16, heads_per_box] -- the same memory walked with the token stride as
+// the second dimension, so one box holds 16 tokens of several heads.
+static bool make_pool_map(CUtensorMap* m, const void* base, const AttnGeom& g, int box_rows,
+                          int heads_per_box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  const cuuint64_t head_stride = static_cast<cuuint64_t>(g.head_dim) * 2;
+  const cuuint64_t token_stride = head_stride * g.num_kv_heads;
+  const cuuint64_t tokens = static_cast<cuuint64_t>(g.num_blocks) * g.block_size;
+  const bool by_token = heads_per_box > 1;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(g.head_dim),
-                        static_cast<cuuint64_t>(g.num_kv_heads),
-                        static_cast<cuuint64_t>(g.num_blocks) * g.block_size};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.head_dim) * 2,
-                           static_cast<cuuint64_t>(g.head_dim) * g.num_kv_heads * 2};
-  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+                        by_token ? tokens : static_cast<cuuint64_t>(g.num_kv_heads),
+                        by_token ? static_cast<cuuint64_t>(g.num_kv_heads) : tokens};
+  cuuint64_t strides[2] = {by_token ? token_stride : head_stride,
+                           by_token ? head_stride : token_stride};
+  cuuint32_t box[3] = {64, by_token ? static_cast<cuuint32_t>(box_rows) : 1u,
+                       by_token ? static_cast<cuuint32_t>(heads_per_box)
+                                : static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -437,7 +463,12 @@ static cudaError_t launch_mma_t(const AttnGeom& g, const WsView& ws, int num_sms
   using C = mmak::Cfg<D, HG>;
   const int box_rows = g.block_size < kStageTokens ? g.block_size : kStageTokens;
   CUtensorMap tk, tv;
-  if (!make_pool_map(&tk, g.k_cache, g, box_rows) || !make_pool_map(&tv, g.v_cache, g, box_rows))
+  int heads_per_box = (box_rows == kStageTokens && HG > 1) ? HG : 1;
+  if (heads_per_box > 1 && !(make_pool_map(&tk, g.k_cache, g, box_rows, heads_per_box) &&
+                             make_pool_map(&tv, g.v_cache, g, box_rows, heads_per_box)))
+    heads_per_box = 1;  // the driver refused the token-major view: one box per head
+  if (heads_per_box == 1 && !(make_pool_map(&tk, g.k_cache, g, box_rows, 1) &&
+                              make_pool_map(&tv, g.v_cache, g, box_rows, 1)))
     return cudaErrorInvalidValue;
   auto kern = attn_mma_kernel<D, HG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
@@ -456,7 +487,7 @@ static cudaError_t launch_mma_t(const AttnGeom& g, const WsView& ws, int num_sms
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tk, tv, g, ws, box_rows);
+  return cudaLaunchKernelEx(&cfg, kern, tk, tv, g, ws, box_rows, heads_per_box);
 }
 
 cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,
