@@ -43,6 +43,8 @@ WsLayout ws_layout(int64_t num_qrows, int num_heads, int head_dim, int head_grou
   off = align_up(off + num_qrows * sizeof(int32_t), 256);
   L.qrow_bad = off;
   off = align_up(off + num_qrows * sizeof(int32_t), 256);
+  L.merge_rows = off;
+  off = align_up(off + num_qrows * sizeof(int32_t), 256);
   L.items = off;
   off = align_up(off + L.max_items * sizeof(int4), 256);
   L.part_ml = off;
@@ -62,6 +64,7 @@ WsView ws_view(void* base, const WsLayout& L) {
   v.qrow_info = reinterpret_cast<int4*>(p + L.qrow_info);
   v.nparts = reinterpret_cast<int32_t*>(p + L.nparts);
   v.qrow_bad = reinterpret_cast<int32_t*>(p + L.qrow_bad);
+  v.merge_rows = reinterpret_cast<int32_t*>(p + L.merge_rows);
   v.items = reinterpret_cast<int4*>(p + L.items);
   v.part_ml = reinterpret_cast<float2*>(p + L.part_ml);
   v.part_o = reinterpret_cast<float*>(p + L.part_o);
@@ -95,12 +98,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   __shared__ int s_max[32];
   __shared__ int s_scan[32];
   __shared__ int s_P;
+  __shared__ int s_merge;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool decode_mode = g.query_start_loc == nullptr;
   const int64_t max_keys = static_cast<int64_t>(g.max_blocks) * g.block_size;
 
   // rows no request covers stay unwritten
   for (int r = tid; r < g.num_qrows; r += kPlanThreads) ws.nparts[r] = -1;
+  if (tid == 0) s_merge = 0;
   __syncthreads();
 
   long long my_units = 0;
@@ -218,10 +223,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
       const int units = (info.y + kStageTokens - 1) / kStageTokens;
       const int np = (units + P - 1) / P;
       ws.nparts[r] = np;
+      if (np != 1) ws.merge_rows[atomicAdd(&s_merge, 1)] = r;
       for (int p = 0; p < np; ++p)
         for (int hg = 0; hg < a.head_groups; ++hg) ws.items[pos++] = make_int4(r, hg, p, 0);
     }
   }
+  __syncthreads();
+  if (tid == 0) ws.ctrl[5] = s_merge;
 }
 
 cudaError_t launch_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws, cudaStream_t s) {
@@ -405,51 +413,113 @@ cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms
 }
 
 // ======================================================================= merge
-// One warp per (row, query head).  Rows with a single partition were written by
-// the attention kernel; rows with none get zeros; invalid rows are skipped.
+// One CTA of 8 warps per (row, query head).  Rows with a single partition were
+// written by the attention kernel; rows with none get zeros; invalid rows are
+// skipped.  The CTA first reduces M = max_k m_k and the denominator over all
+// partitions, keeping the weights 2^(m_k - M) in shared memory, then each warp
+// accumulates every 8th partition's unnormalised output (lanes own D/32
+// columns, 4 partitions in flight) and the 8 warp sums are combined.
+constexpr int kMergeWarps = 8;
+constexpr int kMergeCached = 2048;  // partition weights kept in shared memory
+
 template <int D>
-__global__ void __launch_bounds__(256) merge_kernel(AttnGeom g, WsView ws) {
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(AttnGeom g, WsView ws) {
   constexpr int V = D / 32;
+  __shared__ float s_c[kMergeCached];
+  __shared__ float s_red[kMergeWarps];
+  __shared__ float s_acc[kMergeWarps][D];
   grid_dependency_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (idx >= static_cast<int64_t>(g.num_qrows) * g.num_heads) return;
-  const int r = static_cast<int>(idx / g.num_heads);
-  const int np = ws.nparts[r];
-  if (np == 1 || np < 0 || ws.qrow_bad[r]) return;
-  const int64_t out_base = idx * D + lane * V;
-  if (np == 0) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t pairs = static_cast<int64_t>(ws.ctrl[5]) * g.num_heads;
+  for (int64_t pi = blockIdx.x; pi < pairs; pi += gridDim.x) {
+    const int r = ws.merge_rows[pi / g.num_heads];
+    const int64_t idx = static_cast<int64_t>(r) * g.num_heads + pi % g.num_heads;
+    const int np = ws.nparts[r];
+    if (np == 1 || np < 0 || ws.qrow_bad[r]) continue;
+    const int64_t out_base = idx * D;
+    if (np == 0) {
+      for (int d = tid; d < D; d += blockDim.x) store_out(g.out, g.out_dtype, out_base + d, 0.f);
+      continue;
+    }
+    const int64_t base = idx * ws.max_parts;
+    // M
+    float M = -INFINITY;
+    for (int k = tid; k < np; k += blockDim.x) M = fmaxf(M, ws.part_ml[base + k].x);
 #pragma unroll
-    for (int e = 0; e < V; ++e) store_out(g.out, g.out_dtype, out_base + e, 0.f);
-    return;
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) s_red[warp] = M;
+    __syncthreads();
+    M = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, s_red[w]);
+    __syncthreads();
+    // denominator and weights
+    float den = 0.f;
+    for (int k = tid; k < np; k += blockDim.x) {
+      const float2 ml = ws.part_ml[base + k];
+      const float c = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
+      if (k < kMergeCached) s_c[k] = c;
+      den = fmaf(ml.y, c, den);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane == 0) s_red[warp] = den;
+    __syncthreads();
+    den = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) den += s_red[w];
+    // weighted sum of the partial outputs
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    const float* po = ws.part_o + base * D + lane * V;
+    int k = warp;
+    for (; k + 3 * kMergeWarps < np; k += 4 * kMergeWarps) {
+      float x[4][V], c[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int kk = k + u * kMergeWarps;
+        c[u] = kk < kMergeCached ? s_c[kk]
+                                 : (ws.part_ml[base + kk].x == -INFINITY
+                                        ? 0.f
+                                        : fast_exp2(ws.part_ml[base + kk].x - M));
+#pragma unroll
+        for (int e = 0; e < V; ++e) x[u][e] = po[static_cast<int64_t>(kk) * D + e];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] = fmaf(x[u][e], c[u], acc[e]);
+    }
+    for (; k < np; k += kMergeWarps) {
+      const float c = k < kMergeCached ? s_c[k]
+                                       : (ws.part_ml[base + k].x == -INFINITY
+                                              ? 0.f
+                                              : fast_exp2(ws.part_ml[base + k].x - M));
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[e] = fmaf(po[static_cast<int64_t>(k) * D + e], c, acc[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < V; ++e) s_acc[warp][lane * V + e] = acc[e];
+    __syncthreads();
+    const float inv = 1.f / den;
+    for (int d = tid; d < D; d += blockDim.x) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMergeWarps; ++w) sum += s_acc[w][d];
+      store_out(g.out, g.out_dtype, out_base + d, sum * inv);
+    }
+    __syncthreads();  // s_c / s_red / s_acc are reused by the next pair
   }
-  const int64_t base = idx * ws.max_parts;
-  float M = -INFINITY;
-  for (int k = lane; k < np; k += 32) M = fmaxf(M, ws.part_ml[base + k].x);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float den = 0.f, acc[V];
-#pragma unroll
-  for (int e = 0; e < V; ++e) acc[e] = 0.f;
-  for (int k = 0; k < np; ++k) {
-    const float2 ml = ws.part_ml[base + k];
-    const float c = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
-    den = fmaf(ml.y, c, den);
-    const float* po = ws.part_o + (base + k) * D + lane * V;
-#pragma unroll
-    for (int e = 0; e < V; ++e) acc[e] = fmaf(po[e], c, acc[e]);
-  }
-  const float inv = 1.f / den;
-#pragma unroll
-  for (int e = 0; e < V; ++e) store_out(g.out, g.out_dtype, out_base + e, acc[e] * inv);
 }
 
-cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, cudaStream_t s) {
-  const int64_t warps = static_cast<int64_t>(g.num_qrows) * g.num_heads;
-  if (warps == 0) return cudaSuccess;
+cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {
+  int64_t blocks = static_cast<int64_t>(g.num_qrows) * g.num_heads;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((warps + 7) / 8));
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(kMergeWarps * 32);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -18,18 +18,19 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 // One attention call's scratch, carved from the caller's workspace buffer.
 //   ctrl      int32[64]   [0] dynamic work counter, [1] number of items,
 //                         [2] partition length in tokens, [3] tile counter,
-//                         [4] number of prefill tiles
+//                         [4] number of prefill tiles, [5] rows to merge
 //   qrow_info int4[R]     {request b, key_len, valid, first_key_pos}
 //   nparts    int32[R]    partitions of the row (0: empty -> zero row;
 //                         -1: invalid -> row left unwritten)
 //   qrow_bad  int32[R]    set when a block id outside the pool was met
+//   merge_rows int32[R]   rows the merge pass must write (0 or >1 partitions)
 //   items     int4[I]     {qrow, head group, partition, 0}
 //   part_ml   float2[R*H*P]   per (row, query head, partition): (m, l),
 //                         m in log2 units (score * scale * log2 e)
 //   part_o    float[R*H*P*D]  unnormalised partial outputs
 //   tiles     int4[Tl]    prefill tiles {request b, kv head, first query row, rows}
 struct WsLayout {
-  size_t ctrl, qrow_info, nparts, qrow_bad, items, part_ml, part_o, tiles, total;
+  size_t ctrl, qrow_info, nparts, qrow_bad, merge_rows, items, part_ml, part_o, tiles, total;
   int64_t num_qrows, max_parts, max_items, max_tiles;
 };
 
@@ -38,6 +39,7 @@ struct WsView {
   int4* qrow_info;
   int32_t* nparts;
   int32_t* qrow_bad;
+  int32_t* merge_rows;
   int4* items;
   float2* part_ml;
   float* part_o;
@@ -97,7 +99,7 @@ cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms
                                 cudaStream_t s);
 cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,
                             cudaStream_t s);
-cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, cudaStream_t s);
+cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s);
 
 bool mma_path_supported(const AttnGeom& g);
 int device_num_sms();

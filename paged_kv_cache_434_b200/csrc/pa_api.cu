@@ -143,7 +143,7 @@ static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* works
   cudaError_t e = p.use_mma ? launch_attn_mma(g, ws, p.num_sms, p.heads_per_group, s)
                             : launch_attn_generic(g, ws, p.num_sms, s);
   if (e != cudaSuccess) return PA_ERR_CUDA;
-  if (launch_merge(g, ws, s) != cudaSuccess) return PA_ERR_CUDA;
+  if (launch_merge(g, ws, p.num_sms, s) != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }
 
