@@ -81,6 +81,10 @@ WsView ws_view(void* base, const WsLayout& L) {
 // item count is near target_items and no row needs more than max_parts
 // partitions.  Pass 2 counts items per thread, pass 3 scans and writes them.
 constexpr int kPlanThreads = 1024;
+constexpr int kMaxPrefill = 512;  // prefill requests served by tensor-core tiles per call
+constexpr int kTileBins = 2048;   // longest-first ordering of tiles by 128-key tile count
+
+__device__ __forceinline__ int tile_bin(int n_kv) { return n_kv < kTileBins ? n_kv : kTileBins - 1; }
 
 __device__ __forceinline__ void request_rows(const AttnGeom& g, int b, int& r0, int& q_b) {
   if (g.query_start_loc) {
@@ -99,13 +103,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   __shared__ int s_scan[32];
   __shared__ int s_P;
   __shared__ int s_merge;
+  __shared__ int s_npref;
+  __shared__ int s_pref[kMaxPrefill];
+  __shared__ int s_hist[kTileBins];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool decode_mode = g.query_start_loc == nullptr;
   const int64_t max_keys = static_cast<int64_t>(g.max_blocks) * g.block_size;
 
   // rows no request covers stay unwritten
   for (int r = tid; r < g.num_qrows; r += kPlanThreads) ws.nparts[r] = -1;
-  if (tid == 0) s_merge = 0;
+  if (tid == 0) {
+    s_merge = 0;
+    s_npref = 0;
+  }
+  for (int i = tid; i < kTileBins; i += kPlanThreads) s_hist[i] = 0;
   __syncthreads();
 
   long long my_units = 0;
@@ -126,7 +137,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     }
     if (L > max_keys) bits |= PA_ERRBIT_SEQ_TOO_LONG;
     if (bits && g.err_word) atomicOr(g.err_word, bits);
-    const bool expand = decode_mode || q_b == 1 || a.expand_prefill;
+    bool expand = decode_mode || q_b == 1 || a.expand_prefill;
+    if (!expand && !bits) {
+      const int slot = atomicAdd(&s_npref, 1);
+      if (slot < kMaxPrefill)
+        s_pref[slot] = b;
+      else
+        expand = true;  // beyond the tile list's capacity: per-row path
+    }
     for (int i = 0; i < q_b && r0 + i < g.num_qrows; ++i) {
       const int r = r0 + i;
       ws.qrow_bad[r] = 0;
@@ -171,6 +189,75 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   }
   __syncthreads();
   const int P = s_P;
+
+  // ---- prefill requests on tensor-core tiles: validate their block tables
+  // cooperatively, then list tiles longest-first (histogram over 128-key tile counts)
+  const int npref = min(s_npref, kMaxPrefill);
+  __shared__ int s_badpref;
+  int n_tiles_total = 0;
+  for (int pi = 0; pi < npref; ++pi) {
+    const int b = s_pref[pi];
+    const int L = g.seq_lens[b];
+    const int nblk = (L + g.block_size - 1) / g.block_size;
+    if (tid == 0) s_badpref = 0;
+    __syncthreads();
+    const int32_t* table = g.block_tables + static_cast<int64_t>(b) * g.max_blocks;
+    for (int k = tid; k < nblk; k += kPlanThreads) {
+      const int phys = table[k];
+      if (phys < 0 || phys >= g.num_blocks) s_badpref = 1;
+    }
+    __syncthreads();
+    if (s_badpref) {
+      if (tid == 0) {
+        s_pref[pi] = -1;
+        if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_BLOCK_OOB);
+      }
+      int r0, q_b;
+      request_rows(g, b, r0, q_b);
+      for (int i = tid; i < q_b && r0 + i < g.num_qrows; i += kPlanThreads) ws.nparts[r0 + i] = -1;
+    } else {
+      int r0, q_b;
+      request_rows(g, b, r0, q_b);
+      const int ntb = (q_b + a.tile_tokens - 1) / a.tile_tokens;
+      for (int idx = tid; idx < ntb * g.num_kv_heads; idx += kPlanThreads) {
+        const int tb = idx / g.num_kv_heads;
+        const int last = min((tb + 1) * a.tile_tokens, q_b) - 1;
+        const int n_kv = (L - q_b + last) / 128 + 1;
+        atomicAdd(&s_hist[tile_bin(n_kv)], 1);
+      }
+      n_tiles_total += ntb * g.num_kv_heads;
+    }
+    __syncthreads();
+  }
+  if (npref > 0) {
+    // descending exclusive scan of the histogram: bins with more key tiles first
+    if (tid == 0) {
+      int acc = 0;
+      for (int bin = kTileBins - 1; bin >= 0; --bin) {
+        const int c = s_hist[bin];
+        s_hist[bin] = acc;
+        acc += c;
+      }
+    }
+    __syncthreads();
+    for (int pi = 0; pi < npref; ++pi) {
+      const int b = s_pref[pi];
+      if (b < 0) continue;
+      int r0, q_b;
+      request_rows(g, b, r0, q_b);
+      const int L = g.seq_lens[b];
+      const int ntb = (q_b + a.tile_tokens - 1) / a.tile_tokens;
+      for (int idx = tid; idx < ntb * g.num_kv_heads; idx += kPlanThreads) {
+        const int tb = idx / g.num_kv_heads, hk = idx % g.num_kv_heads;
+        const int tok0 = tb * a.tile_tokens;
+        const int ntok = min(a.tile_tokens, q_b - tok0);
+        const int n_kv = (L - q_b + tok0 + ntok - 1) / 128 + 1;
+        const int at = atomicAdd(&s_hist[tile_bin(n_kv)], 1);
+        if (at < ws.max_tiles) ws.tiles[at] = make_int4(b, hk, tok0, ntok);
+      }
+    }
+  }
+  if (tid == 0) ws.ctrl[4] = static_cast<int>(min(static_cast<int64_t>(n_tiles_total), ws.max_tiles));
 
   // pass 2: items per thread
   int my_items = 0;

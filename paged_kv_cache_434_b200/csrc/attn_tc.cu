@@ -1,0 +1,537 @@
+// attn_tc.cu -- tensor-core (tcgen05 / TMEM) tiles for the chunked-prefill
+// requests of a mixed continuous-batching step.
+//
+// What is computed ("AI Infra入门干货总结：大模型是如何高效推理的", section
+// "Attention (FlashAttention, Scaled Dot-Product Attention)"): for the q_b new
+// tokens of a request with seq_len L (q_b > 1), query i at position
+// L - q_b + i attends causally to keys 0 .. L - q_b + i through the block table
+// (the v1 unified varlen path reads every K/V from the paged cache).  The
+// online softmax keeps a running max m and sum l and rescales the output by
+// exp(m_old - m_new); here the rescale is skipped while the new row max stays
+// within 2^8 of the one in use (the weights then stay below 256, which bf16
+// and fp32 represent exactly enough), an exact reformulation.
+//
+// Tile = 128 query rows x all keys they see, processed 128 keys at a time.
+// The 128 rows are 128/G consecutive tokens x the G query heads of one KV
+// head (GQA): one K/V tile read serves the whole group.
+//
+// CTA (persistent, one per SM, 10 warps):
+//   warp 9   scheduler: takes the next tile from the planner's longest-first
+//            list, publishes it in a 2-slot ring, TMA-loads the Q tile
+//            (double-buffered, 128-byte swizzle) for it.
+//   warps 0-3  two loader groups of 64 threads; group g fills K/V stage g for
+//            every other 128-key tile with 16-byte cp.async copies gathered
+//            through the block table into the 128B-swizzled layout the MMA
+//            reads (blocks of 16 keys are too small for efficient TMA boxes).
+//   warp 8   allocates TMEM; one thread issues the MMAs: S = Q K^T into one of
+//            two TMEM S buffers (M=128, N=128, K=D), then O += P V into the
+//            TMEM O accumulator (N=D, K=128, V read as an MN-major operand).
+//   warps 4-7  softmax: thread i owns query row i = TMEM lane i, reads its S
+//            row straight from TMEM (row max and sum need no shuffles),
+//            writes bf16 P to shared memory for the PV MMA, rescales O in
+//            TMEM when the max moved, and finally writes O / l.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace pa {
+namespace tck {
+
+constexpr int kRows = 128;     // query rows per tile
+constexpr int kKeys = 128;     // keys per KV tile
+constexpr int kThreads = 320;  // 10 warps
+constexpr int kHalfBytes = 128 * 128;  // [128 rows x 64 bf16]
+constexpr float kRescaleLog2 = 8.f;
+
+struct Item {
+  int b, hk, tok0, ntok;  // request, KV head, first token (within the request), tokens
+  int n_kv;               // 128-key tiles to visit (0: end of work)
+  int first_pos;          // position of the first token
+  int row0;               // flattened row of the first token
+  int L;                  // seq_len of the request
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int NH = D / 64;
+  static constexpr int kQBytes = NH * kHalfBytes;
+  static constexpr int kPBytes = 2 * kHalfBytes;   // 128 rows x 128 keys
+  static constexpr int kKVBytes = NH * kHalfBytes; // one K (or V) tile
+  static constexpr int kStageBytes = 2 * kKVBytes;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffP = 2 * kQBytes;
+  static constexpr int kOffKV = kOffP + kPBytes;
+  static constexpr int kOffMeta = kOffKV + 2 * kStageBytes;
+  static constexpr int kSmem = kOffMeta + 1024 + 1024;  // meta + alignment slack
+};
+
+// barriers in the meta area
+struct Meta {
+  Item ring[2];
+  uint64_t item_full[2], item_empty[2];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t kv_full[2], kv_empty[2];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full, o_ready, o_empty, drain;
+  uint32_t tmem_base;
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity) {
+  bool ok = mbar_wait_bounded(bar, parity, kWaitLimitNs);
+  return __all_sync(0xffffffffu, ok);
+}
+
+}  // namespace tck
+
+template <int D>
+__global__ void __launch_bounds__(tck::kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, AttnGeom g, WsView ws) {
+  using namespace tck;
+  using C = Cfg<D>;
+  constexpr int NH = C::NH;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Meta* meta = reinterpret_cast<Meta*>(smem + C::kOffMeta);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = g.num_heads / g.num_kv_heads;
+  const int Tq = kRows / G;  // tokens per tile
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&meta->item_full[i], 1);
+      mbar_init(&meta->item_empty[i], 64 + 64 + 1 + 128);
+      mbar_init(&meta->q_full[i], 1);
+      mbar_init(&meta->q_empty[i], 1);
+      mbar_init(&meta->kv_full[i], 64);
+      mbar_init(&meta->kv_empty[i], 1);
+      mbar_init(&meta->s_full[i], 1);
+      mbar_init(&meta->s_empty[i], 128);
+    }
+    mbar_init(&meta->p_full, 128);
+    mbar_init(&meta->o_ready, 1);
+    mbar_init(&meta->o_empty, 128);
+    mbar_init(&meta->drain, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmQ);
+  }
+  if (warp == 8) {
+    tmem_alloc(&meta->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  grid_dependency_wait();
+  const uint32_t tmem = meta->tmem_base;
+  const int n_tiles = ws.ctrl[4];
+  const uint32_t sQ = smem_u32(smem + C::kOffQ);
+  const uint32_t sP = smem_u32(smem + C::kOffP);
+  const uint32_t sKV = smem_u32(smem + C::kOffKV);
+
+  if (warp == 9) {
+    // ---------------------------------------------------------- scheduler
+    if (lane == 0) {
+      for (int n = 0;; ++n) {
+        const int it = atomicAdd(&ws.ctrl[3], 1);
+        Item info{};
+        if (it < n_tiles) {
+          const int4 t = ws.tiles[it];
+          const int qs = g.query_start_loc[t.x];
+          const int qb = g.query_start_loc[t.x + 1] - qs;
+          info.b = t.x;
+          info.hk = t.y;
+          info.tok0 = t.z;
+          info.ntok = t.w;
+          info.L = g.seq_lens[t.x];
+          info.first_pos = info.L - qb + t.z;
+          info.row0 = qs + t.z;
+          info.n_kv = (info.first_pos + t.w - 1) / kKeys + 1;
+        }
+        const int slot = n & 1;
+        if (n >= 2 && !mbar_wait_bounded(&meta->item_empty[slot], ((n >> 1) - 1) & 1,
+                                         kWaitLimitNs)) {
+          if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
+          break;
+        }
+        meta->ring[slot] = info;
+        mbar_arrive(&meta->item_full[slot]);
+        if (info.n_kv == 0) break;
+        const int qbuf = n & 1;
+        if (n >= 2 && !mbar_wait_bounded(&meta->q_empty[qbuf], ((n >> 1) - 1) & 1,
+                                         kWaitLimitNs)) {
+          if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(&meta->q_full[qbuf], C::kQBytes);
+#pragma unroll
+        for (int dh = 0; dh < NH; ++dh)
+          tma_load_3d(smem + C::kOffQ + qbuf * C::kQBytes + dh * kHalfBytes, &tmQ,
+                      &meta->q_full[qbuf], dh * 64, info.hk * G, info.row0);
+      }
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------- loaders
+    const int grp = warp >> 1;        // loader group = stage it fills
+    const int tg = tid & 63;          // thread within the group
+    const __nv_bfloat16* kc = static_cast<const __nv_bfloat16*>(g.k_cache);
+    const __nv_bfloat16* vc = static_cast<const __nv_bfloat16*>(g.v_cache);
+    const uint32_t kst = sKV + grp * C::kStageBytes;
+    const uint32_t vst = kst + C::kKVBytes;
+    int tile_base = 0, mine = 0;
+    bool ok = true;
+    for (int n = 0; ok; ++n) {
+      const int slot = n & 1;
+      if (!wait_warp(&meta->item_full[slot], (n >> 1) & 1)) break;
+      const Item info = meta->ring[slot];
+      mbar_arrive(&meta->item_empty[slot]);
+      if (info.n_kv == 0) break;
+      const int32_t* table = g.block_tables + static_cast<int64_t>(info.b) * g.max_blocks;
+      for (int j = 0; j < info.n_kv; ++j) {
+        const int t = tile_base + j;
+        if ((t & 1) != grp) continue;
+        if (mine >= 1 && !wait_warp(&meta->kv_empty[grp], (mine - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        ++mine;
+#pragma unroll
+        for (int half_keys = 0; half_keys < 2; ++half_keys) {
+          const int key = tg + 64 * half_keys;
+          const int kpos = j * kKeys + key;
+          const __nv_bfloat16* ksrc = kc;
+          const __nv_bfloat16* vsrc = vc;
+          uint32_t bytes = 0;
+          if (kpos < info.L) {
+            const int phys = table[kpos / g.block_size];
+            if (phys >= 0 && phys < g.num_blocks) {
+              const int64_t row = static_cast<int64_t>(phys) * g.block_size + kpos % g.block_size;
+              const int64_t off = (row * g.num_kv_heads + info.hk) * D;
+              ksrc = kc + off;
+              vsrc = vc + off;
+              bytes = 16;
+            }
+          }
+#pragma unroll
+          for (int dh = 0; dh < NH; ++dh) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t o = dh * kHalfBytes + swz(key, c);
+              cp_async16(kst + o, ksrc + (bytes ? dh * 64 + c * 8 : 0), bytes);
+              cp_async16(vst + o, vsrc + (bytes ? dh * 64 + c * 8 : 0), bytes);
+            }
+          }
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        mbar_arrive(&meta->kv_full[grp]);
+      }
+      tile_base += info.n_kv;
+    }
+    cp_async_wait<0>();
+    if (!ok && g.err_word && tg == 0) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
+  } else if (warp == 8) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t id_qk = idesc_bf16_f32(kRows, kKeys, 0, 0);
+      const uint32_t id_pv = idesc_bf16_f32(kRows, D, 0, 1);
+      const uint32_t tO = tmem + 256;
+      int tile_base = 0, p_count = 0;
+      bool ok = true;
+      auto pv = [&](int t, int j, int n) -> bool {
+        if (!mbar_wait_bounded(&meta->p_full, p_count & 1, kWaitLimitNs)) return false;
+        ++p_count;
+        if (j == 0 && n >= 1 && !mbar_wait_bounded(&meta->o_empty, (n - 1) & 1, kWaitLimitNs))
+          return false;
+        tc_fence_after();
+        const uint32_t vst = sKV + (t & 1) * C::kStageBytes + C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          const uint64_t a = smem_desc(sP + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024, 2);
+          const uint64_t bd = smem_desc(vst + kk * 2048, kHalfBytes, 1024, 2);
+          umma_bf16(tO, a, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&meta->o_ready);
+        umma_commit(&meta->kv_empty[t & 1]);
+        return true;
+      };
+      for (int n = 0; ok; ++n) {
+        const int slot = n & 1;
+        if (!mbar_wait_bounded(&meta->item_full[slot], (n >> 1) & 1, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        const Item info = meta->ring[slot];
+        mbar_arrive(&meta->item_empty[slot]);
+        if (info.n_kv == 0) break;
+        const int qbuf = n & 1;
+        if (!mbar_wait_bounded(&meta->q_full[qbuf], (n >> 1) & 1, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        const uint32_t qb = sQ + qbuf * C::kQBytes;
+        for (int j = 0; j < info.n_kv && ok; ++j) {
+          const int t = tile_base + j;
+          if (!mbar_wait_bounded(&meta->kv_full[t & 1], (t >> 1) & 1, kWaitLimitNs) ||
+              (t >= 2 && !mbar_wait_bounded(&meta->s_empty[t & 1], ((t >> 1) - 1) & 1,
+                                            kWaitLimitNs))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kst = sKV + (t & 1) * C::kStageBytes;
+          const uint32_t tS = tmem + (t & 1) * 128;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            umma_bf16(tS, smem_desc(qb + off, 16, 1024, 2), smem_desc(kst + off, 16, 1024, 2),
+                      id_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&meta->s_full[t & 1]);
+          if (j == info.n_kv - 1) umma_commit(&meta->q_empty[qbuf]);
+          if (j >= 1 && !pv(t - 1, j - 1, n)) ok = false;
+        }
+        if (ok && !pv(tile_base + info.n_kv - 1, info.n_kv - 1, n)) ok = false;
+        tile_base += info.n_kv;
+      }
+      // every MMA issued so far has completed before TMEM is released
+      umma_commit(&meta->drain);
+      mbar_wait_bounded(&meta->drain, 0, kWaitLimitNs);
+      if (!ok && g.err_word) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
+    }
+  } else {
+    // ---------------------------------------------------------- softmax (warps 4-7)
+    const int row = tid - 128;                     // query row = TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tO = tmem + lane_addr + 256;
+    int tile_base = 0, o_count = 0;
+    bool ok = true;
+    for (int n = 0; ok; ++n) {
+      const int slot = n & 1;
+      if (!wait_warp(&meta->item_full[slot], (n >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      const Item info = meta->ring[slot];
+      mbar_arrive(&meta->item_empty[slot]);
+      if (info.n_kv == 0) break;
+      const int tok = row / G;
+      const int pos = info.first_pos + tok;  // this row's position
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < info.n_kv; ++j) {
+        const int t = tile_base + j;
+        const uint32_t tS = tmem + lane_addr + (t & 1) * 128;
+        if (!wait_warp(&meta->s_full[t & 1], (t >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool masked = j * kKeys + kKeys - 1 > info.first_pos;
+        const int lim = pos - j * kKeys;  // keys c <= lim are visible
+        // pass 1: row max of the scaled scores
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tS + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float s = __uint_as_float(r[e]);
+            if (!masked || c * 32 + e <= lim) mx = fmaxf(mx, s);
+          }
+        }
+        mx *= g.scale_log2;
+        const bool rescale = mx > m + kRescaleLog2;
+        const float m_use = rescale ? mx : m;
+        const float alpha = rescale ? fast_exp2(m - m_use) : 1.f;
+        // the previous PV must be done before P is overwritten and O rescaled
+        if (j >= 1) {
+          if (!wait_warp(&meta->o_ready, o_count & 1)) {
+            ok = false;
+            break;
+          }
+          ++o_count;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld32(tO + c * 32, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              tmem_st32(tO + c * 32, r);
+            }
+            tmem_st_wait();
+          }
+        }
+        // pass 2: P = 2^(s * scale_log2 - m_use) as bf16 into shared memory
+        float psum = 0.f;
+        const uint32_t prow = sP + row * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tS + c * 32, r);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float p0 = fast_exp2(fmaf(__uint_as_float(r[e]), g.scale_log2, -m_use));
+            float p1 = fast_exp2(fmaf(__uint_as_float(r[e + 1]), g.scale_log2, -m_use));
+            if (masked) {
+              if (c * 32 + e > lim) p0 = 0.f;
+              if (c * 32 + e + 1 > lim) p1 = 0.f;
+            }
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e >> 1]));
+            psum += f.x + f.y;
+          }
+          // keys 32c .. 32c+31 -> half c/2, chunks (c&1)*4 .. +3 of this row
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int chunk = (c & 1) * 4 + q4;
+            const uint32_t addr = prow - row * 128 + (c >> 1) * kHalfBytes + swz(row, chunk);
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[q4 * 4]),
+                         "r"(pk[q4 * 4 + 1]), "r"(pk[q4 * 4 + 2]), "r"(pk[q4 * 4 + 3])
+                         : "memory");
+          }
+        }
+        l = l * alpha + psum;
+        m = m_use;
+        tc_fence_before();
+        mbar_arrive(&meta->s_empty[t & 1]);
+        fence_proxy_async_smem();
+        mbar_arrive(&meta->p_full);
+      }
+      if (!ok) break;
+      // epilogue: O / l for the rows of real tokens
+      if (!wait_warp(&meta->o_ready, o_count & 1)) {
+        ok = false;
+        break;
+      }
+      ++o_count;
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const bool store = tok < info.ntok;
+      const int64_t obase =
+          (static_cast<int64_t>(info.row0 + tok) * g.num_heads + info.hk * G + row % G) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + c * 32, r);
+        tmem_ld_wait();
+        if (store) {
+          if (g.out_dtype == PA_F32) {
+            float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(g.out) + obase + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              o4[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                                  __uint_as_float(r[4 * e + 2]) * inv,
+                                  __uint_as_float(r[4 * e + 3]) * inv);
+          } else {
+            uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + obase + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              o4[e] = make_uint4(
+                  pack_bf16x2(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
+                  pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
+                  pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
+                  pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&meta->o_empty);
+      tile_base += info.n_kv;
+    }
+    if (!ok && g.err_word && row == 0) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFnTc)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFnTc encode_fn_tc() {
+  static EncodeTiledFnTc fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFnTc>(p);
+  }
+  return fn;
+}
+
+bool tc_path_supported(const AttnGeom& g) {
+  const int G = g.num_kv_heads > 0 ? g.num_heads / g.num_kv_heads : 0;
+  return g.dtype == PA_BF16 && (g.head_dim == 64 || g.head_dim == 128) && G >= 1 && G <= 16 &&
+         (tck::kRows % G) == 0 && encode_fn_tc() != nullptr;
+}
+
+int tc_tokens_per_tile(const AttnGeom& g) {
+  return tck::kRows / (g.num_heads / g.num_kv_heads);
+}
+
+template <int D>
+static cudaError_t launch_tc_t(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {
+  using C = tck::Cfg<D>;
+  const int G = g.num_heads / g.num_kv_heads;
+  // q viewed as (dim, head, token); one box = 64 dims x G heads x 128/G tokens
+  CUtensorMap tq;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(g.num_heads),
+                        static_cast<cuuint64_t>(g.num_qrows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(D) * 2 * g.num_heads};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(tck::kRows / G)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (encode_fn_tc()(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(g.q), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  auto kern = attn_tc_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms);
+  cfg.blockDim = dim3(tck::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tq, g, ws);
+}
+
+cudaError_t launch_attn_tc(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {
+  if (g.head_dim == 128) return launch_tc_t<128>(g, ws, num_sms, s);
+  return launch_tc_t<64>(g, ws, num_sms, s);
+}
+
+}  // namespace pa

@@ -83,6 +83,7 @@ struct PlanArgs {
   int32_t target_items;     // aim for about this many items in total
   int32_t min_part_stages;  // lower bound of a partition, in 16-key stages
   int32_t expand_prefill;   // 1: every query of a q_b>1 request is its own row
+  int32_t tile_tokens;      // tokens per prefill tile (when expand_prefill == 0)
 };
 
 // ---------------------------------------------------------------- launchers
@@ -100,8 +101,11 @@ cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms
 cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,
                             cudaStream_t s);
 cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s);
+cudaError_t launch_attn_tc(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s);
 
 bool mma_path_supported(const AttnGeom& g);
+bool tc_path_supported(const AttnGeom& g);
+int tc_tokens_per_tile(const AttnGeom& g);
 int device_num_sms();
 
 }  // namespace pa

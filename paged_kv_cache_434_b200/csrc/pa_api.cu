@@ -40,6 +40,8 @@ static int elt_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
 // workspace-size query and in the call itself.
 struct AttnPlan {
   bool use_mma;
+  bool use_tc;       // prefill requests (q_b > 1) on tcgen05 tiles
+  int tile_tokens;
   int heads_per_group;
   int head_groups;
   int num_sms;
@@ -50,7 +52,8 @@ struct AttnPlan {
 };
 
 static AttnPlan make_plan(int64_t num_qrows, int num_heads, int max_blocks,
-                          const pa_cache_desc* c, bool bf16_fast_ok) {
+                          const pa_cache_desc* c, bool bf16_fast_ok, int num_seqs = 0,
+                          bool mixed = false) {
   AttnPlan p{};
   AttnGeom probe{};
   probe.num_heads = num_heads;
@@ -79,7 +82,11 @@ static AttnPlan make_plan(int64_t num_qrows, int num_heads, int max_blocks,
   if (mp > max_units) mp = max_units;
   if (mp < 1) mp = 1;
   p.max_parts = mp;
-  p.max_tiles = 0;
+  p.use_tc = mixed && bf16_fast_ok && tc_path_supported(probe);
+  p.tile_tokens = p.use_tc ? tc_tokens_per_tile(probe) : 0;
+  p.max_tiles = p.use_tc ? ((num_qrows + p.tile_tokens - 1) / p.tile_tokens + num_seqs) *
+                               static_cast<int64_t>(c->num_kv_heads)
+                         : 0;
   return p;
 }
 
@@ -126,7 +133,7 @@ static pa_status check_attn_args(int32_t num_seqs, int64_t num_qrows, int32_t nu
 }
 
 static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* workspace,
-                               size_t ws_bytes, int expand_prefill, cudaStream_t s) {
+                               size_t ws_bytes, cudaStream_t s) {
   const WsLayout L = ws_layout(p.num_qrows, g.num_heads, g.head_dim, p.head_groups, p.max_parts,
                                p.max_tiles);
   if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -138,8 +145,10 @@ static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* works
   a.heads_per_group = p.heads_per_group;
   a.target_items = p.target_items;
   a.min_part_stages = 2;
-  a.expand_prefill = expand_prefill;
+  a.expand_prefill = p.use_tc ? 0 : 1;
+  a.tile_tokens = p.tile_tokens;
   if (launch_plan(g, a, ws, s) != cudaSuccess) return PA_ERR_CUDA;
+  if (p.use_tc && launch_attn_tc(g, ws, p.num_sms, s) != cudaSuccess) return PA_ERR_CUDA;
   cudaError_t e = p.use_mma ? launch_attn_mma(g, ws, p.num_sms, p.heads_per_group, s)
                             : launch_attn_generic(g, ws, p.num_sms, s);
   if (e != cudaSuccess) return PA_ERR_CUDA;
@@ -230,7 +239,7 @@ pa_status pa_decode(const void* q, const void* key_cache, const void* value_cach
   const AttnGeom g = make_geom(q, key_cache, value_cache, block_tables, seq_lens, nullptr, scale,
                                out, num_seqs, num_seqs, num_heads, max_blocks_per_seq, out_dtype,
                                cache, err_word);
-  return run_attention(g, p, workspace, workspace_bytes, 1, static_cast<cudaStream_t>(stream));
+  return run_attention(g, p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 size_t pa_mixed_step_workspace_size(int32_t num_seqs, int64_t num_tokens, int32_t num_heads,
@@ -238,7 +247,8 @@ size_t pa_mixed_step_workspace_size(int32_t num_seqs, int64_t num_tokens, int32_
   if (check_attn_args(num_seqs, num_tokens, num_heads, max_blocks_per_seq, PA_F32, cache) !=
       PA_OK)
     return 0;
-  const AttnPlan p = make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true);
+  const AttnPlan p =
+      make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true, num_seqs, true);
   return ws_layout(p.num_qrows, num_heads, cache->head_dim, p.head_groups, p.max_parts,
                    p.max_tiles)
       .total;
@@ -258,11 +268,12 @@ pa_status pa_mixed_step(const void* q, const void* key_cache, const void* value_
     return PA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
     return PA_ERR_INVALID_ARG;
-  const AttnPlan p = make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true);
+  const AttnPlan p =
+      make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true, num_seqs, true);
   const AttnGeom g = make_geom(q, key_cache, value_cache, block_tables, seq_lens,
                                query_start_loc, scale, out, num_seqs, num_tokens, num_heads,
                                max_blocks_per_seq, out_dtype, cache, err_word);
-  return run_attention(g, p, workspace, workspace_bytes, 1, static_cast<cudaStream_t>(stream));
+  return run_attention(g, p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 pa_status pa_read_error(int32_t* err_word, int32_t* host_bits, void* stream) {

@@ -90,6 +90,17 @@ def test_mixed_random_shapes(cuda_device, dtype, bs, D):
     _check_all(w, cuda_device)
 
 
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 4), (32, 2)])
+@pytest.mark.parametrize("D", [64, 128])
+def test_mixed_gqa_packings(cuda_device, hq, hkv, D):
+    # prefill tiles pack 128/G tokens x G query heads; cover G = 1, 2, 8, 16,
+    # chunks shorter and longer than a tile, a cached prefix not a multiple of 128
+    lens = [300, 129, 1, 77, 520, 64]
+    qlens = [150, 129, 1, 1, 8, 17]
+    w = W.custom("mixed_gqa", lens, qlens, hq, hkv, D, 16, "bf16", seed=hq + hkv + D)
+    _check_all(w, cuda_device)
+
+
 def test_bf16_output_variant(cuda_device):
     w = W.custom("bf16_out", [5, 77, 300, 1], [1, 1, 1, 1], 32, 8, 128, 16, "bf16", seed=4)
     _check_all(w, cuda_device, out_dtype=torch.bfloat16)
