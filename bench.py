@@ -39,6 +39,7 @@ WORKLOADS = {
     "long_context": ("long_context_decode", 3),
     "mixed": ("mixed_step", 4),
     "shared_prefix": ("shared_prefix_decode", 5),
+    "mixed_prefill": ("mixed_step_prefill_only", 4),
 }
 FLUSH_BYTES = 512 << 20
 
@@ -186,8 +187,8 @@ def workload_for(name: str, seed: int):
 
 
 def byte_counts(w, out_elt=4):
-    """Algorithmic bytes of one step (unique valid K/V rows once,
-    Q read, O written; the cache write reads and writes each new K/V row)."""
+    """Algorithmic bytes of one step: unique valid K/V rows once, Q read, O
+    written; the cache write reads and writes each new K/V row."""
     from paged_kv_cache_434_b200 import workloads as W
     kv = W.kv_bytes_touched(w, unique=True)
     q = w.num_tokens * w.num_heads * w.head_dim * w.elt_bytes
@@ -209,7 +210,7 @@ def prefill_flops(w):
 
 
 def metric_of(name):
-    if name == "mixed":
+    if name in ("mixed", "mixed_prefill"):
         return "mixed-step query tokens/s per layer", "tokens/s"
     return "paged decode KV GB/s", "GB/s"
 
@@ -278,6 +279,51 @@ def oracle_sample(w, pools, seconds: float, rng_seed: int = 0):
 
 
 # ---------------------------------------------------------------- our arm
+
+def time_prefill_tiles(P, w, t, idx, flush, stream, steps, peaks, flops):
+    """Time the tensor-core prefill tiles alone: a mixed step over only the
+    q_b > 1 requests of the batch (same pools and block tables).  The timed
+    call still includes the planner and two near-empty launches."""
+    qsl = w.query_start_loc
+    pre = [b for b in range(w.num_seqs) if w.query_lens[b] > 1]
+    if not pre:
+        return None
+    rows = np.concatenate([np.arange(qsl[b], qsl[b + 1]) for b in pre])
+    dev = t["q"].device
+    q_sub = t["q"][torch.from_numpy(rows).to(dev)].contiguous()
+    qlens = w.query_lens[pre]
+    qsl_sub = torch.from_numpy(np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)).to(dev)
+    lens_sub = torch.from_numpy(w.seq_lens[pre].copy()).to(dev)
+    tables_sub = torch.from_numpy(np.ascontiguousarray(w.block_tables[pre])).to(dev)
+    out = torch.empty(q_sub.shape, dtype=torch.float32, device=dev)
+    nbytes = P.mixed_step_workspace_size(len(pre), q_sub.shape[0], w.num_heads,
+                                         tables_sub.shape[1], t["k_cache"])
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+    def call():
+        P.mixed_step(q_sub, t["k_cache"], t["v_cache"], tables_sub, qsl_sub, lens_sub, w.scale,
+                     out=out, workspace=ws)
+    for _ in range(3):
+        call()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(min(steps, 50))]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        flush.fill_(1)
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    sec = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+    tf = flops / sec / 1e12
+    return {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": round(tf, 1),
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(tf / peaks["bf16_tflops"], 4),
+            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16_tflops, burst: timed alone)",
+            "timed_over": "pa_mixed_step on the prefill requests only (planner + tiles)",
+            "ms": round(sec * 1e3, 4), "algorithmic_flops_per_launch": flops,
+            "traffic": None}
+
 
 def run_ours(args, rank, world, local):
     import paged_kv_cache_434_b200 as P
@@ -349,7 +395,7 @@ def run_ours(args, rank, world, local):
 
     bc = byte_counts(w)
     metric, unit = metric_of(args.workload)
-    if args.workload == "mixed":
+    if args.workload in ("mixed", "mixed_prefill"):
         value = T * args.steps * world / total_s
     else:
         value = bc["step"] * args.steps * world / total_s / 1e9
@@ -366,9 +412,11 @@ def run_ours(args, rank, world, local):
                 "traffic": kernel_traffic(src, f"{dominant}_{args.workload}.md"),
                 "algorithmic_bytes_per_launch": bc["attention"]}
     extra = {}
-    if args.workload == "mixed":
+    prefill_roofline = None
+    if args.workload in ("mixed", "mixed_prefill"):
         fl = prefill_flops(w)
         extra["prefill_flops_per_step"] = fl
+        prefill_roofline = time_prefill_tiles(P, w, t, idx, flush, stream, args.steps, peaks, fl)
 
     # ---- end to end: host buffers in, result back to the host, each step
     e2e = None
@@ -399,7 +447,7 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / 1e3, world, dev)
-        e2e_val = (T * args.steps * world / e2e_s if args.workload == "mixed"
+        e2e_val = (T * args.steps * world / e2e_s if args.workload in ("mixed", "mixed_prefill")
                    else bc["step"] * args.steps * world / e2e_s / 1e9)
         e2e = {"value": round(e2e_val, 2), "unit": unit, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_s * 1e3 / args.steps, 4)}
@@ -408,7 +456,7 @@ def run_ours(args, rank, world, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         units, el, desc, threads = oracle_sample(w, (t["k_cache"], t["v_cache"]),
                                                  args.cpu_seconds)
-        v = units / el / (1 if args.workload == "mixed" else 1e9)
+        v = units / el / (1 if args.workload in ("mixed", "mixed_prefill") else 1e9)
         cpu = {"value": round(v, 4), "unit": unit, "cores": threads, "kind": "oracle",
                "sample": desc}
 
@@ -430,6 +478,7 @@ def run_ours(args, rank, world, local):
                        "parallelism": f"replicas x{world} (independent batches per GPU)",
                        **extra},
             "roofline": roofline,
+            **({"prefill_roofline": prefill_roofline} if prefill_roofline else {}),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 5 * args.steps,
@@ -465,7 +514,7 @@ def run_reference(args, rank, world, local):
             vals.append((units, el))
     units = sum(u for u, _ in vals)
     el = sum(e for _, e in vals)
-    value = units / el / (1 if args.workload == "mixed" else 1e9)
+    value = units / el / (1 if args.workload in ("mixed", "mixed_prefill") else 1e9)
     line = {
         "impl": "reference", "metric": metric, "value": round(value, 4), "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),

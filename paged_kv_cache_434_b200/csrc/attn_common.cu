@@ -76,13 +76,23 @@ WsView ws_view(void* base, const WsLayout& L) {
 }
 
 // ======================================================================= planner
-// One CTA.  Pass 1 validates every request, fills the per-row table and sums the
-// work (in 16-key stages); the partition length P is then chosen so that the
-// item count is near target_items and no row needs more than max_parts
-// partitions.  Pass 2 counts items per thread, pass 3 scans and writes them.
+// One CTA of 1024 threads, all loops parallel:
+//   0. every row starts "unassigned" (left unwritten);
+//   1. requests in parallel: validation (error bits), rows of small requests
+//      filled inline, larger per-row requests and prefill-tile requests listed;
+//   1b. listed per-row requests: their rows filled cooperatively;
+//   1c. prefill-tile requests: block table validated cooperatively, tiles
+//      counted per 128-key-tile bin;
+//   the partition length P is then chosen so that the item count is near
+//   target_items and no row needs more than max_parts partitions;
+//   2./3. rows in parallel: items counted, scanned, written; rows whose result
+//      the merge pass writes (0 or > 1 partitions) listed;
+//   4. tiles scattered longest-first (descending bin order).
 constexpr int kPlanThreads = 1024;
 constexpr int kMaxPrefill = 512;  // prefill requests served by tensor-core tiles per call
 constexpr int kTileBins = 2048;   // longest-first ordering of tiles by 128-key tile count
+constexpr int kInlineRows = 8;    // requests with at most this many rows: one thread
+constexpr int kMaxBig = 1024;     // larger per-row requests: whole CTA, one at a time
 
 __device__ __forceinline__ int tile_bin(int n_kv) { return n_kv < kTileBins ? n_kv : kTileBins - 1; }
 
@@ -96,76 +106,136 @@ __device__ __forceinline__ void request_rows(const AttnGeom& g, int b, int& r0, 
   }
 }
 
+__device__ __forceinline__ void fill_row(const AttnGeom& g, const WsView& ws, bool decode_mode,
+                                         int b, int r, int i, int q_b, int L,
+                                         long long& units_sum, int& units_max) {
+  const int key_len = decode_mode ? L : L - q_b + i + 1;
+  ws.qrow_info[r] = make_int4(b, key_len, 1, 0);
+  const int units = (key_len + kStageTokens - 1) / kStageTokens;
+  units_sum += units;
+  units_max = max(units_max, units);
+}
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs a, WsView ws) {
   grid_launch_dependents();
   __shared__ long long s_sum[32];
   __shared__ int s_max[32];
   __shared__ int s_scan[32];
-  __shared__ int s_P;
-  __shared__ int s_merge;
-  __shared__ int s_npref;
+  __shared__ int s_P, s_merge, s_npref, s_nbig, s_badpref;
   __shared__ int s_pref[kMaxPrefill];
+  __shared__ int s_big[kMaxBig];
   __shared__ int s_hist[kTileBins];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool decode_mode = g.query_start_loc == nullptr;
   const int64_t max_keys = static_cast<int64_t>(g.max_blocks) * g.block_size;
 
-  // rows no request covers stay unwritten
-  for (int r = tid; r < g.num_qrows; r += kPlanThreads) ws.nparts[r] = -1;
+  // 0. rows no request covers stay unwritten
+  for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
+    ws.nparts[r] = -1;
+    ws.qrow_bad[r] = 0;
+    ws.qrow_info[r] = make_int4(-1, 0, 0, 0);
+  }
   if (tid == 0) {
     s_merge = 0;
     s_npref = 0;
+    s_nbig = 0;
   }
   for (int i = tid; i < kTileBins; i += kPlanThreads) s_hist[i] = 0;
   __syncthreads();
 
+  // 1. requests
   long long my_units = 0;
   int my_max = 0;
   for (int b = tid; b < g.num_seqs; b += kPlanThreads) {
     int r0, q_b;
     request_rows(g, b, r0, q_b);
     const int L = g.seq_lens[b];
-    int bits = 0;
     if (r0 < 0 || r0 > g.num_qrows) {
       if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_QUERY_TOO_LONG);
       continue;
     }
+    int bits = 0;
     if (decode_mode) {
       if (L < 0) bits |= PA_ERRBIT_QUERY_TOO_LONG;
     } else if (q_b < 0 || q_b > L) {
       bits |= PA_ERRBIT_QUERY_TOO_LONG;
     }
     if (L > max_keys) bits |= PA_ERRBIT_SEQ_TOO_LONG;
-    if (bits && g.err_word) atomicOr(g.err_word, bits);
-    bool expand = decode_mode || q_b == 1 || a.expand_prefill;
-    if (!expand && !bits) {
+    if (bits) {
+      if (g.err_word) atomicOr(g.err_word, bits);
+      continue;  // its rows stay unwritten
+    }
+    const bool tile = !(decode_mode || q_b == 1 || a.expand_prefill);
+    if (tile) {
       const int slot = atomicAdd(&s_npref, 1);
-      if (slot < kMaxPrefill)
+      if (slot < kMaxPrefill) {
         s_pref[slot] = b;
-      else
-        expand = true;  // beyond the tile list's capacity: per-row path
+        continue;
+      }  // beyond the tile list's capacity: per-row path below
     }
-    for (int i = 0; i < q_b && r0 + i < g.num_qrows; ++i) {
-      const int r = r0 + i;
-      ws.qrow_bad[r] = 0;
-      if (bits) {
-        ws.qrow_info[r] = make_int4(b, 0, 0, 0);
-        ws.nparts[r] = -1;
+    const int nrows = min(q_b, g.num_qrows - r0);
+    if (nrows > kInlineRows) {
+      const int slot = atomicAdd(&s_nbig, 1);
+      if (slot < kMaxBig) {
+        s_big[slot] = b;
         continue;
       }
-      if (!expand) {
-        ws.qrow_info[r] = make_int4(b, 0, 0, 0);
-        ws.nparts[r] = -2;  // handled by prefill tiles
-        continue;
-      }
-      const int key_len = decode_mode ? L : L - q_b + i + 1;
-      ws.qrow_info[r] = make_int4(b, key_len, 1, 0);
-      const int units = (key_len + kStageTokens - 1) / kStageTokens;
-      my_units += units;
-      my_max = max(my_max, units);
     }
+    for (int i = 0; i < nrows; ++i)
+      fill_row(g, ws, decode_mode, b, r0 + i, i, q_b, L, my_units, my_max);
   }
-  // block reductions
+  __syncthreads();
+
+  // 1b. large per-row requests, cooperatively
+  const int nbig = min(s_nbig, kMaxBig);
+  for (int k = 0; k < nbig; ++k) {
+    const int b = s_big[k];
+    int r0, q_b;
+    request_rows(g, b, r0, q_b);
+    const int L = g.seq_lens[b];
+    const int nrows = min(q_b, g.num_qrows - r0);
+    for (int i = tid; i < nrows; i += kPlanThreads)
+      fill_row(g, ws, decode_mode, b, r0 + i, i, q_b, L, my_units, my_max);
+  }
+
+  // 1c. prefill requests on tensor-core tiles: block tables validated
+  // cooperatively, rows marked, tiles counted per bin
+  const int npref = min(s_npref, kMaxPrefill);
+  int n_tiles_total = 0;
+  for (int pi = 0; pi < npref; ++pi) {
+    const int b = s_pref[pi];
+    const int L = g.seq_lens[b];
+    const int nblk = (L + g.block_size - 1) / g.block_size;
+    if (tid == 0) s_badpref = 0;
+    __syncthreads();
+    const int32_t* table = g.block_tables + static_cast<int64_t>(b) * g.max_blocks;
+    for (int k = tid; k < nblk; k += kPlanThreads) {
+      const int phys = table[k];
+      if (phys < 0 || phys >= g.num_blocks) s_badpref = 1;
+    }
+    __syncthreads();
+    int r0, q_b;
+    request_rows(g, b, r0, q_b);
+    if (s_badpref) {
+      if (tid == 0) {
+        s_pref[pi] = -1;
+        if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_BLOCK_OOB);
+      }
+    } else {
+      for (int i = tid; i < q_b && r0 + i < g.num_qrows; i += kPlanThreads)
+        ws.nparts[r0 + i] = -2;  // written by the tile kernel
+      const int ntb = (q_b + a.tile_tokens - 1) / a.tile_tokens;
+      for (int idx = tid; idx < ntb * g.num_kv_heads; idx += kPlanThreads) {
+        const int tb = idx / g.num_kv_heads;
+        const int last = min((tb + 1) * a.tile_tokens, q_b) - 1;
+        atomicAdd(&s_hist[tile_bin((L - q_b + last) / 128 + 1)], 1);
+      }
+      n_tiles_total += ntb * g.num_kv_heads;
+    }
+    __syncthreads();
+  }
+
+  // partition length
   for (int o = 16; o; o >>= 1) {
     my_units += __shfl_xor_sync(0xffffffffu, my_units, o);
     my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, o));
@@ -190,89 +260,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   __syncthreads();
   const int P = s_P;
 
-  // ---- prefill requests on tensor-core tiles: validate their block tables
-  // cooperatively, then list tiles longest-first (histogram over 128-key tile counts)
-  const int npref = min(s_npref, kMaxPrefill);
-  __shared__ int s_badpref;
-  int n_tiles_total = 0;
-  for (int pi = 0; pi < npref; ++pi) {
-    const int b = s_pref[pi];
-    const int L = g.seq_lens[b];
-    const int nblk = (L + g.block_size - 1) / g.block_size;
-    if (tid == 0) s_badpref = 0;
-    __syncthreads();
-    const int32_t* table = g.block_tables + static_cast<int64_t>(b) * g.max_blocks;
-    for (int k = tid; k < nblk; k += kPlanThreads) {
-      const int phys = table[k];
-      if (phys < 0 || phys >= g.num_blocks) s_badpref = 1;
-    }
-    __syncthreads();
-    if (s_badpref) {
-      if (tid == 0) {
-        s_pref[pi] = -1;
-        if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_BLOCK_OOB);
-      }
-      int r0, q_b;
-      request_rows(g, b, r0, q_b);
-      for (int i = tid; i < q_b && r0 + i < g.num_qrows; i += kPlanThreads) ws.nparts[r0 + i] = -1;
-    } else {
-      int r0, q_b;
-      request_rows(g, b, r0, q_b);
-      const int ntb = (q_b + a.tile_tokens - 1) / a.tile_tokens;
-      for (int idx = tid; idx < ntb * g.num_kv_heads; idx += kPlanThreads) {
-        const int tb = idx / g.num_kv_heads;
-        const int last = min((tb + 1) * a.tile_tokens, q_b) - 1;
-        const int n_kv = (L - q_b + last) / 128 + 1;
-        atomicAdd(&s_hist[tile_bin(n_kv)], 1);
-      }
-      n_tiles_total += ntb * g.num_kv_heads;
-    }
-    __syncthreads();
-  }
-  if (npref > 0) {
-    // descending exclusive scan of the histogram: bins with more key tiles first
-    if (tid == 0) {
-      int acc = 0;
-      for (int bin = kTileBins - 1; bin >= 0; --bin) {
-        const int c = s_hist[bin];
-        s_hist[bin] = acc;
-        acc += c;
-      }
-    }
-    __syncthreads();
-    for (int pi = 0; pi < npref; ++pi) {
-      const int b = s_pref[pi];
-      if (b < 0) continue;
-      int r0, q_b;
-      request_rows(g, b, r0, q_b);
-      const int L = g.seq_lens[b];
-      const int ntb = (q_b + a.tile_tokens - 1) / a.tile_tokens;
-      for (int idx = tid; idx < ntb * g.num_kv_heads; idx += kPlanThreads) {
-        const int tb = idx / g.num_kv_heads, hk = idx % g.num_kv_heads;
-        const int tok0 = tb * a.tile_tokens;
-        const int ntok = min(a.tile_tokens, q_b - tok0);
-        const int n_kv = (L - q_b + tok0 + ntok - 1) / 128 + 1;
-        const int at = atomicAdd(&s_hist[tile_bin(n_kv)], 1);
-        if (at < ws.max_tiles) ws.tiles[at] = make_int4(b, hk, tok0, ntok);
-      }
-    }
-  }
-  if (tid == 0) ws.ctrl[4] = static_cast<int>(min(static_cast<int64_t>(n_tiles_total), ws.max_tiles));
-
-  // pass 2: items per thread
+  // 2. items per thread (rows in parallel)
   int my_items = 0;
-  for (int b = tid; b < g.num_seqs; b += kPlanThreads) {
-    int r0, q_b;
-    request_rows(g, b, r0, q_b);
-    if (r0 < 0) continue;
-    for (int i = 0; i < q_b && r0 + i < g.num_qrows; ++i) {
-      const int4 info = ws.qrow_info[r0 + i];
-      if (info.z == 0) continue;
-      const int units = (info.y + kStageTokens - 1) / kStageTokens;
-      my_items += (units + P - 1) / P * a.head_groups;
-    }
+  for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
+    const int4 info = ws.qrow_info[r];
+    if (info.z == 0) continue;
+    const int units = (info.y + kStageTokens - 1) / kStageTokens;
+    my_items += (units + P - 1) / P * a.head_groups;
   }
-  // exclusive scan over the CTA
   int incl = my_items;
   for (int o = 1; o < 32; o <<= 1) {
     int n = __shfl_up_sync(0xffffffffu, incl, o);
@@ -298,25 +293,50 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   __syncthreads();
   int pos = s_scan[warp] + incl - my_items;
 
-  // pass 3: write items and partition counts
-  for (int b = tid; b < g.num_seqs; b += kPlanThreads) {
-    int r0, q_b;
-    request_rows(g, b, r0, q_b);
-    if (r0 < 0) continue;
-    for (int i = 0; i < q_b && r0 + i < g.num_qrows; ++i) {
-      const int r = r0 + i;
-      const int4 info = ws.qrow_info[r];
-      if (info.z == 0) continue;
-      const int units = (info.y + kStageTokens - 1) / kStageTokens;
-      const int np = (units + P - 1) / P;
-      ws.nparts[r] = np;
-      if (np != 1) ws.merge_rows[atomicAdd(&s_merge, 1)] = r;
-      for (int p = 0; p < np; ++p)
-        for (int hg = 0; hg < a.head_groups; ++hg) ws.items[pos++] = make_int4(r, hg, p, 0);
+  // 3. items, partition counts, rows to merge
+  for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
+    const int4 info = ws.qrow_info[r];
+    if (info.z == 0) continue;
+    const int units = (info.y + kStageTokens - 1) / kStageTokens;
+    const int np = (units + P - 1) / P;
+    ws.nparts[r] = np;
+    if (np != 1) ws.merge_rows[atomicAdd(&s_merge, 1)] = r;
+    for (int p = 0; p < np; ++p)
+      for (int hg = 0; hg < a.head_groups; ++hg) ws.items[pos++] = make_int4(r, hg, p, 0);
+  }
+
+  // 4. tiles, longest first
+  if (npref > 0) {
+    if (tid == 0) {
+      int acc = 0;
+      for (int bin = kTileBins - 1; bin >= 0; --bin) {
+        const int c = s_hist[bin];
+        s_hist[bin] = acc;
+        acc += c;
+      }
+    }
+    __syncthreads();
+    for (int pi = 0; pi < npref; ++pi) {
+      const int b = s_pref[pi];
+      if (b < 0) continue;
+      int r0, q_b;
+      request_rows(g, b, r0, q_b);
+      const int L = g.seq_lens[b];
+      const int ntb = (q_b + a.tile_tokens - 1) / a.tile_tokens;
+      for (int idx = tid; idx < ntb * g.num_kv_heads; idx += kPlanThreads) {
+        const int tb = idx / g.num_kv_heads, hk = idx % g.num_kv_heads;
+        const int tok0 = tb * a.tile_tokens;
+        const int ntok = min(a.tile_tokens, q_b - tok0);
+        const int at = atomicAdd(&s_hist[tile_bin((L - q_b + tok0 + ntok - 1) / 128 + 1)], 1);
+        if (at < ws.max_tiles) ws.tiles[at] = make_int4(b, hk, tok0, ntok);
+      }
     }
   }
   __syncthreads();
-  if (tid == 0) ws.ctrl[5] = s_merge;
+  if (tid == 0) {
+    ws.ctrl[4] = static_cast<int>(min(static_cast<int64_t>(n_tiles_total), ws.max_tiles));
+    ws.ctrl[5] = s_merge;
+  }
 }
 
 cudaError_t launch_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws, cudaStream_t s) {

@@ -15,15 +15,19 @@
 // The 128 rows are 128/G consecutive tokens x the G query heads of one KV
 // head (GQA): one K/V tile read serves the whole group.
 //
-// CTA (persistent, one per SM, 10 warps):
-//   warp 9   scheduler: takes the next tile from the planner's longest-first
+// CTA (persistent, one per SM, 8 warps -- two per SM sub-partition, so the
+// softmax threads can hold a whole 128-column S row in registers):
+//   warp 3   scheduler: takes the next tile from the planner's longest-first
 //            list, publishes it in a 2-slot ring, TMA-loads the Q tile
 //            (double-buffered, 128-byte swizzle) for it.
-//   warps 0-3  two loader groups of 64 threads; group g fills K/V stage g for
-//            every other 128-key tile with 16-byte cp.async copies gathered
-//            through the block table into the 128B-swizzled layout the MMA
-//            reads (blocks of 16 keys are too small for efficient TMA boxes).
-//   warp 8   allocates TMEM; one thread issues the MMAs: S = Q K^T into one of
+//   warps 0-1  loaders: warp 0 fills the K stages, warp 1 the V stages (two
+//            each), with 16-byte cp.async copies gathered through the block
+//            table into the 128B-swizzled layout the MMA reads (blocks of 16
+//            keys are too small for efficient TMA boxes).  A K stage is free
+//            again once its QK^T is done, a V stage once its PV is done; each
+//            loader keeps two tiles in flight and announces a tile when it has
+//            issued the next one.
+//   warp 2   allocates TMEM; one thread issues the MMAs: S = Q K^T into one of
 //            two TMEM S buffers (M=128, N=128, K=D), then O += P V into the
 //            TMEM O accumulator (N=D, K=128, V read as an MN-major operand).
 //   warps 4-7  softmax: thread i owns query row i = TMEM lane i, reads its S
@@ -43,7 +47,7 @@ namespace tck {
 
 constexpr int kRows = 128;     // query rows per tile
 constexpr int kKeys = 128;     // keys per KV tile
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 256;  // 8 warps
 constexpr int kHalfBytes = 128 * 128;  // [128 rows x 64 bf16]
 constexpr float kRescaleLog2 = 8.f;
 
@@ -61,11 +65,11 @@ struct Cfg {
   static constexpr int kQBytes = NH * kHalfBytes;
   static constexpr int kPBytes = 2 * kHalfBytes;   // 128 rows x 128 keys
   static constexpr int kKVBytes = NH * kHalfBytes; // one K (or V) tile
-  static constexpr int kStageBytes = 2 * kKVBytes;
   static constexpr int kOffQ = 0;
   static constexpr int kOffP = 2 * kQBytes;
-  static constexpr int kOffKV = kOffP + kPBytes;
-  static constexpr int kOffMeta = kOffKV + 2 * kStageBytes;
+  static constexpr int kOffK = kOffP + kPBytes;     // two K stages
+  static constexpr int kOffV = kOffK + 2 * kKVBytes; // two V stages
+  static constexpr int kOffMeta = kOffV + 2 * kKVBytes;
   static constexpr int kSmem = kOffMeta + 1024 + 1024;  // meta + alignment slack
 };
 
@@ -74,7 +78,7 @@ struct Meta {
   Item ring[2];
   uint64_t item_full[2], item_empty[2];
   uint64_t q_full[2], q_empty[2];
-  uint64_t kv_full[2], kv_empty[2];
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full, o_ready, o_empty, drain;
   uint32_t tmem_base;
@@ -103,16 +107,17 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
   Meta* meta = reinterpret_cast<Meta*>(smem + C::kOffMeta);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = g.num_heads / g.num_kv_heads;
-  const int Tq = kRows / G;  // tokens per tile
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&meta->item_full[i], 1);
-      mbar_init(&meta->item_empty[i], 64 + 64 + 1 + 128);
+      mbar_init(&meta->item_empty[i], 32 + 32 + 1 + 128);
       mbar_init(&meta->q_full[i], 1);
       mbar_init(&meta->q_empty[i], 1);
-      mbar_init(&meta->kv_full[i], 64);
-      mbar_init(&meta->kv_empty[i], 1);
+      mbar_init(&meta->k_full[i], 32);
+      mbar_init(&meta->k_empty[i], 1);
+      mbar_init(&meta->v_full[i], 32);
+      mbar_init(&meta->v_empty[i], 1);
       mbar_init(&meta->s_full[i], 1);
       mbar_init(&meta->s_empty[i], 128);
     }
@@ -123,7 +128,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&tmQ);
   }
-  if (warp == 8) {
+  if (warp == 2) {
     tmem_alloc(&meta->tmem_base, 512);
     tmem_relinquish();
   }
@@ -135,9 +140,10 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
   const int n_tiles = ws.ctrl[4];
   const uint32_t sQ = smem_u32(smem + C::kOffQ);
   const uint32_t sP = smem_u32(smem + C::kOffP);
-  const uint32_t sKV = smem_u32(smem + C::kOffKV);
+  const uint32_t sK = smem_u32(smem + C::kOffK);
+  const uint32_t sV = smem_u32(smem + C::kOffV);
 
-  if (warp == 9) {
+  if (warp == 3) {
     // ---------------------------------------------------------- scheduler
     if (lane == 0) {
       for (int n = 0;; ++n) {
@@ -178,68 +184,82 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
                       &meta->q_full[qbuf], dh * 64, info.hk * G, info.row0);
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 2) {
     // ---------------------------------------------------------- loaders
-    const int grp = warp >> 1;        // loader group = stage it fills
-    const int tg = tid & 63;          // thread within the group
-    const __nv_bfloat16* kc = static_cast<const __nv_bfloat16*>(g.k_cache);
-    const __nv_bfloat16* vc = static_cast<const __nv_bfloat16*>(g.v_cache);
-    const uint32_t kst = sKV + grp * C::kStageBytes;
-    const uint32_t vst = kst + C::kKVBytes;
-    int tile_base = 0, mine = 0;
+    const bool is_v = warp == 1;
+    const int tg = lane;
+    const int bshift = __ffs(g.block_size) - 1;  // block sizes are powers of two
+    const __nv_bfloat16* src_pool = static_cast<const __nv_bfloat16*>(is_v ? g.v_cache : g.k_cache);
+    const uint32_t sbase = is_v ? sV : sK;
+    uint64_t* full = is_v ? meta->v_full : meta->k_full;
+    uint64_t* empty = is_v ? meta->v_empty : meta->k_empty;
+    int tile_base = 0, pending = -1;
     bool ok = true;
     for (int n = 0; ok; ++n) {
       const int slot = n & 1;
-      if (!wait_warp(&meta->item_full[slot], (n >> 1) & 1)) break;
+      if (!wait_warp(&meta->item_full[slot], (n >> 1) & 1)) {
+        ok = false;
+        break;
+      }
       const Item info = meta->ring[slot];
       mbar_arrive(&meta->item_empty[slot]);
       if (info.n_kv == 0) break;
       const int32_t* table = g.block_tables + static_cast<int64_t>(info.b) * g.max_blocks;
       for (int j = 0; j < info.n_kv; ++j) {
         const int t = tile_base + j;
-        if ((t & 1) != grp) continue;
-        if (mine >= 1 && !wait_warp(&meta->kv_empty[grp], (mine - 1) & 1)) {
+        if (t >= 2 && !wait_warp(&empty[t & 1], ((t >> 1) - 1) & 1)) {
           ok = false;
           break;
         }
-        ++mine;
+        const uint32_t dst = sbase + (t & 1) * C::kKVBytes;
+        // block-table lookups first: lane l resolves keys l, l+32, l+64, l+96 to
+        // their pool rows (-1: past the request or outside the pool)
+        int prow[4];
 #pragma unroll
-        for (int half_keys = 0; half_keys < 2; ++half_keys) {
-          const int key = tg + 64 * half_keys;
-          const int kpos = j * kKeys + key;
-          const __nv_bfloat16* ksrc = kc;
-          const __nv_bfloat16* vsrc = vc;
-          uint32_t bytes = 0;
+        for (int q = 0; q < 4; ++q) {
+          const int kpos = j * kKeys + tg + 32 * q;
+          prow[q] = -1;
           if (kpos < info.L) {
-            const int phys = table[kpos / g.block_size];
-            if (phys >= 0 && phys < g.num_blocks) {
-              const int64_t row = static_cast<int64_t>(phys) * g.block_size + kpos % g.block_size;
-              const int64_t off = (row * g.num_kv_heads + info.hk) * D;
-              ksrc = kc + off;
-              vsrc = vc + off;
-              bytes = 16;
-            }
-          }
-#pragma unroll
-          for (int dh = 0; dh < NH; ++dh) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const uint32_t o = dh * kHalfBytes + swz(key, c);
-              cp_async16(kst + o, ksrc + (bytes ? dh * 64 + c * 8 : 0), bytes);
-              cp_async16(vst + o, vsrc + (bytes ? dh * 64 + c * 8 : 0), bytes);
-            }
+            const int phys = table[kpos >> bshift];
+            if (phys >= 0 && phys < g.num_blocks)
+              prow[q] = (phys << bshift) + (kpos & (g.block_size - 1));
           }
         }
+        // lane l then copies 16-byte chunk l % (8 * NH) of a key, several keys per
+        // instruction, so every warp instruction reads whole 128-byte rows
+        constexpr int kChunks = 8 * NH;          // 16-byte chunks per key row
+        constexpr int kKeysPerInst = 32 / kChunks;
+        const int chunk = tg % kChunks, dh = chunk >> 3, c = chunk & 7;
+#pragma unroll
+        for (int i = 0; i < kKeys / kKeysPerInst; ++i) {
+          const int key = i * kKeysPerInst + tg / kChunks;
+          const int r = __shfl_sync(0xffffffffu, prow[(i * kKeysPerInst) >> 5], key & 31);
+          const __nv_bfloat16* src = src_pool;
+          uint32_t bytes = 0;
+          if (r >= 0) {
+            src = src_pool + (static_cast<int64_t>(r) * g.num_kv_heads + info.hk) * D + dh * 64 + c * 8;
+            bytes = 16;
+          }
+          cp_async16(dst + dh * kHalfBytes + swz(key, c), src, bytes);
+        }
         cp_async_commit();
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(&meta->kv_full[grp]);
+        if (pending >= 0) {
+          // the previous tile's copies are complete once at most this group is in flight
+          cp_async_wait<1>();
+          fence_proxy_async_smem();
+          mbar_arrive(&full[pending & 1]);
+        }
+        pending = t;
       }
       tile_base += info.n_kv;
     }
     cp_async_wait<0>();
+    if (pending >= 0) {
+      fence_proxy_async_smem();
+      mbar_arrive(&full[pending & 1]);
+    }
     if (!ok && g.err_word && tg == 0) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
-  } else if (warp == 8) {
+  } else if (warp == 2) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(kRows, kKeys, 0, 0);
@@ -252,8 +272,9 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         ++p_count;
         if (j == 0 && n >= 1 && !mbar_wait_bounded(&meta->o_empty, (n - 1) & 1, kWaitLimitNs))
           return false;
+        if (!mbar_wait_bounded(&meta->v_full[t & 1], (t >> 1) & 1, kWaitLimitNs)) return false;
         tc_fence_after();
-        const uint32_t vst = sKV + (t & 1) * C::kStageBytes + C::kKVBytes;
+        const uint32_t vst = sV + (t & 1) * C::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
           const uint64_t a = smem_desc(sP + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024, 2);
@@ -261,7 +282,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
           umma_bf16(tO, a, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&meta->o_ready);
-        umma_commit(&meta->kv_empty[t & 1]);
+        umma_commit(&meta->v_empty[t & 1]);
         return true;
       };
       for (int n = 0; ok; ++n) {
@@ -281,14 +302,14 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         const uint32_t qb = sQ + qbuf * C::kQBytes;
         for (int j = 0; j < info.n_kv && ok; ++j) {
           const int t = tile_base + j;
-          if (!mbar_wait_bounded(&meta->kv_full[t & 1], (t >> 1) & 1, kWaitLimitNs) ||
+          if (!mbar_wait_bounded(&meta->k_full[t & 1], (t >> 1) & 1, kWaitLimitNs) ||
               (t >= 2 && !mbar_wait_bounded(&meta->s_empty[t & 1], ((t >> 1) - 1) & 1,
                                             kWaitLimitNs))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t kst = sKV + (t & 1) * C::kStageBytes;
+          const uint32_t kst = sK + (t & 1) * C::kKVBytes;
           const uint32_t tS = tmem + (t & 1) * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -297,6 +318,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
                       id_qk, kk > 0 ? 1u : 0u);
           }
           umma_commit(&meta->s_full[t & 1]);
+          umma_commit(&meta->k_empty[t & 1]);
           if (j == info.n_kv - 1) umma_commit(&meta->q_empty[qbuf]);
           if (j >= 1 && !pv(t - 1, j - 1, n)) ok = false;
         }
@@ -337,19 +359,25 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         tc_fence_after();
         const bool masked = j * kKeys + kKeys - 1 > info.first_pos;
         const int lim = pos - j * kKeys;  // keys c <= lim are visible
-        // pass 1: row max of the scaled scores
+        // the whole S row in one round trip: 4 loads of 32 columns, one wait
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&meta->s_empty[t & 1]);  // S buffer free for the MMA of tile t + 2
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e > lim) sr[c][e] = 0xff800000u;  // -inf
+        }
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tS + c * 32, r);
-          tmem_ld_wait();
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float s = __uint_as_float(r[e]);
-            if (!masked || c * 32 + e <= lim) mx = fmaxf(mx, s);
-          }
-        }
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
         mx *= g.scale_log2;
         const bool rescale = mx > m + kRescaleLog2;
         const float m_use = rescale ? mx : m;
@@ -363,44 +391,36 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
           ++o_count;
           tc_fence_after();
           if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
+            // rare after the first tiles: 32 columns at a time keeps registers low
+#pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
-              uint32_t r[32];
-              tmem_ld32(tO + c * 32, r);
+              uint32_t orr[32];
+              tmem_ld32(tO + c * 32, orr);
               tmem_ld_wait();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-              tmem_st32(tO + c * 32, r);
+              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+              tmem_st32(tO + c * 32, orr);
             }
             tmem_st_wait();
           }
         }
-        // pass 2: P = 2^(s * scale_log2 - m_use) as bf16 into shared memory
+        // P = 2^(s * scale_log2 - m_use) as bf16 into shared memory (masked keys
+        // hold -inf and give 0)
         float psum = 0.f;
-        const uint32_t prow = sP + row * 128;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tS + c * 32, r);
-          tmem_ld_wait();
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            float p0 = fast_exp2(fmaf(__uint_as_float(r[e]), g.scale_log2, -m_use));
-            float p1 = fast_exp2(fmaf(__uint_as_float(r[e + 1]), g.scale_log2, -m_use));
-            if (masked) {
-              if (c * 32 + e > lim) p0 = 0.f;
-              if (c * 32 + e + 1 > lim) p1 = 0.f;
-            }
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][e]), g.scale_log2, -m_use));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][e + 1]), g.scale_log2, -m_use));
+            psum += p0 + p1;
             pk[e >> 1] = pack_bf16x2(p0, p1);
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e >> 1]));
-            psum += f.x + f.y;
           }
-          // keys 32c .. 32c+31 -> half c/2, chunks (c&1)*4 .. +3 of this row
+          // keys 32c .. 32c+31 -> half c/2, 16-byte chunks (c&1)*4 .. +3 of this row
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
-            const int chunk = (c & 1) * 4 + q4;
-            const uint32_t addr = prow - row * 128 + (c >> 1) * kHalfBytes + swz(row, chunk);
+            const uint32_t addr = sP + (c >> 1) * kHalfBytes + swz(row, (c & 1) * 4 + q4);
             asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[q4 * 4]),
                          "r"(pk[q4 * 4 + 1]), "r"(pk[q4 * 4 + 2]), "r"(pk[q4 * 4 + 3])
                          : "memory");
@@ -409,7 +429,6 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         l = l * alpha + psum;
         m = m_use;
         tc_fence_before();
-        mbar_arrive(&meta->s_empty[t & 1]);
         fence_proxy_async_smem();
         mbar_arrive(&meta->p_full);
       }
@@ -459,7 +478,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -489,7 +508,8 @@ static EncodeTiledFnTc encode_fn_tc() {
 bool tc_path_supported(const AttnGeom& g) {
   const int G = g.num_kv_heads > 0 ? g.num_heads / g.num_kv_heads : 0;
   return g.dtype == PA_BF16 && (g.head_dim == 64 || g.head_dim == 128) && G >= 1 && G <= 16 &&
-         (tck::kRows % G) == 0 && encode_fn_tc() != nullptr;
+         (tck::kRows % G) == 0 && encode_fn_tc() != nullptr &&
+         static_cast<int64_t>(g.num_blocks) * g.block_size < (1LL << 31);
 }
 
 int tc_tokens_per_tile(const AttnGeom& g) {

@@ -6,7 +6,7 @@
 
 #include <cuda_runtime.h>
 
-#include "../../include/pa.h"
+#include "pa.h"  // include/ is on the include path
 
 namespace pa {
 

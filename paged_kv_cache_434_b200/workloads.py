@@ -175,6 +175,14 @@ def shared_prefix_decode(seed: int = 0, num_seqs: int = 128, prefix_tokens: int 
                     seed, shared_prefix_blocks=pblocks)
 
 
+def mixed_step_prefill_only(seed: int = 0, chunk: int = 2048, prefix: int = 4096) -> Workload:
+    """Only the two chunked-prefill requests of mixed_step(): a 2048-token
+    chunk after a 4096-token cached prefix and a fresh 2048-token prompt."""
+    lens = np.array([prefix + chunk, chunk], dtype=np.int32)
+    qlens = np.array([chunk, chunk], dtype=np.int32)
+    return custom("mixed_prefill_chunks_bf16", lens, qlens, 32, 8, 128, 16, "bf16", seed)
+
+
 CONFIGS = {
     1: tiny_decode,
     2: llama8b_decode,
