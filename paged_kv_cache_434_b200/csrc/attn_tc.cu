@@ -207,40 +207,45 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
       const int32_t* table = g.block_tables + static_cast<int64_t>(info.b) * g.max_blocks;
       for (int j = 0; j < info.n_kv; ++j) {
         const int t = tile_base + j;
+        const uint32_t dst = sbase + (t & 1) * C::kKVBytes;
+        // Lanes are paired (D = 128) or grouped by four (D = 64) on a key so
+        // that one warp instruction copies whole 32-byte sectors of 16 (8)
+        // keys.  Each lane first resolves its keys' pool rows through the block
+        // table (-1: past the request or outside the pool), then copies fixed
+        // chunk offsets of those rows into the 128B-swizzled tile.
+        constexpr int kChunks = 8 * NH;                 // 16-byte chunks per key row
+        constexpr int kKPI = D == 128 ? 16 : 8;          // keys per warp instruction
+        constexpr int kLPK = 32 / kKPI;                  // lanes per key
+        constexpr int kKeysPerLane = kKeys / kKPI;
+        constexpr int kCPL = kChunks / kLPK;             // chunks per lane per key
+        const int ksub = tg / kLPK, csub = tg % kLPK;
+        const __nv_bfloat16* rowp[kKeysPerLane];
+#pragma unroll
+        for (int q = 0; q < kKeysPerLane; ++q) {
+          const int kpos = j * kKeys + q * kKPI + ksub;
+          rowp[q] = nullptr;
+          if (kpos < info.L) {
+            const int phys = table[kpos >> bshift];
+            if (phys >= 0 && phys < g.num_blocks)
+              rowp[q] = src_pool + ((static_cast<int64_t>(phys << bshift) + (kpos & (g.block_size - 1))) *
+                                        g.num_kv_heads + info.hk) * D;
+          }
+        }
         if (t >= 2 && !wait_warp(&empty[t & 1], ((t >> 1) - 1) & 1)) {
           ok = false;
           break;
         }
-        const uint32_t dst = sbase + (t & 1) * C::kKVBytes;
-        // block-table lookups first: lane l resolves keys l, l+32, l+64, l+96 to
-        // their pool rows (-1: past the request or outside the pool)
-        int prow[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int kpos = j * kKeys + tg + 32 * q;
-          prow[q] = -1;
-          if (kpos < info.L) {
-            const int phys = table[kpos >> bshift];
-            if (phys >= 0 && phys < g.num_blocks)
-              prow[q] = (phys << bshift) + (kpos & (g.block_size - 1));
-          }
-        }
-        // lane l then copies 16-byte chunk l % (8 * NH) of a key, several keys per
-        // instruction, so every warp instruction reads whole 128-byte rows
-        constexpr int kChunks = 8 * NH;          // 16-byte chunks per key row
-        constexpr int kKeysPerInst = 32 / kChunks;
-        const int chunk = tg % kChunks, dh = chunk >> 3, c = chunk & 7;
+        for (int q = 0; q < kKeysPerLane; ++q) {
+          const int key = q * kKPI + ksub;
+          const uint32_t rbase = dst + key * 128;
+          const bool valid = rowp[q] != nullptr;
 #pragma unroll
-        for (int i = 0; i < kKeys / kKeysPerInst; ++i) {
-          const int key = i * kKeysPerInst + tg / kChunks;
-          const int r = __shfl_sync(0xffffffffu, prow[(i * kKeysPerInst) >> 5], key & 31);
-          const __nv_bfloat16* src = src_pool;
-          uint32_t bytes = 0;
-          if (r >= 0) {
-            src = src_pool + (static_cast<int64_t>(r) * g.num_kv_heads + info.hk) * D + dh * 64 + c * 8;
-            bytes = 16;
+          for (int p = 0; p < kCPL; ++p) {
+            const int chunk = p * kLPK + csub, dh = chunk >> 3, c = chunk & 7;
+            cp_async16(rbase + dh * kHalfBytes + ((c ^ (key & 7)) << 4),
+                       valid ? rowp[q] + chunk * 8 : src_pool, valid ? 16u : 0u);
           }
-          cp_async16(dst + dh * kHalfBytes + swz(key, c), src, bytes);
         }
         cp_async_commit();
         if (pending >= 0) {
@@ -412,8 +417,9 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
+            // half of the exponentials on the XU (ex2.approx), half on the FMA pipe
             const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][e]), g.scale_log2, -m_use));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][e + 1]), g.scale_log2, -m_use));
+            const float p1 = exp2_poly(fmaf(__uint_as_float(sr[c][e + 1]), g.scale_log2, -m_use));
             psum += p0 + p1;
             pk[e >> 1] = pack_bf16x2(p0, p1);
           }
