@@ -20,8 +20,8 @@
 //   warp 3   scheduler: takes the next tile from the planner's longest-first
 //            list, publishes it in a 2-slot ring, TMA-loads the Q tile
 //            (double-buffered, 128-byte swizzle) for it.
-//   warps 0-1  loaders: warp 0 fills the K stages, warp 1 the V stages (two
-//            each), with 16-byte cp.async copies gathered through the block
+//   warps 0-1  loaders: warp 0 fills the K stages (three), warp 1 the V stages
+//            (two), with 16-byte cp.async copies gathered through the block
 //            table into the 128B-swizzled layout the MMA reads (blocks of 16
 //            keys are too small for efficient TMA boxes).  A K stage is free
 //            again once its QK^T is done, a V stage once its PV is done; each
@@ -29,11 +29,14 @@
 //            issued the next one.
 //   warp 2   allocates TMEM; one thread issues the MMAs: S = Q K^T into one of
 //            two TMEM S buffers (M=128, N=128, K=D), then O += P V into the
-//            TMEM O accumulator (N=D, K=128, V read as an MN-major operand).
+//            TMEM O accumulator (N=D, K=128) with P read from TMEM and V as an
+//            MN-major shared-memory operand.  MMAs of one thread execute in
+//            issue order, and each PV is issued before the QK^T that reuses
+//            its S buffer.
 //   warps 4-7  softmax: thread i owns query row i = TMEM lane i, reads its S
 //            row straight from TMEM (row max and sum need no shuffles),
-//            writes bf16 P to shared memory for the PV MMA, rescales O in
-//            TMEM when the max moved, and finally writes O / l.
+//            writes bf16 P over the first 64 columns of the same S buffer,
+//            rescales O in TMEM when the max moved, and finally writes O / l.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -63,13 +66,12 @@ template <int D>
 struct Cfg {
   static constexpr int NH = D / 64;
   static constexpr int kQBytes = NH * kHalfBytes;
-  static constexpr int kPBytes = 2 * kHalfBytes;   // 128 rows x 128 keys
   static constexpr int kKVBytes = NH * kHalfBytes; // one K (or V) tile
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffP = 2 * kQBytes;
-  static constexpr int kOffK = kOffP + kPBytes;     // two K stages
-  static constexpr int kOffV = kOffK + 2 * kKVBytes; // two V stages
-  static constexpr int kOffMeta = kOffV + 2 * kKVBytes;
+  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr int kOffQ = 0;                   // two Q buffers
+  static constexpr int kOffK = 2 * kQBytes;
+  static constexpr int kOffV = kOffK + kKStages * kKVBytes;
+  static constexpr int kOffMeta = kOffV + kVStages * kKVBytes;
   static constexpr int kSmem = kOffMeta + 1024 + 1024;  // meta + alignment slack
 };
 
@@ -78,8 +80,8 @@ struct Meta {
   Item ring[2];
   uint64_t item_full[2], item_empty[2];
   uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
+  uint64_t s_full[2];
   uint64_t p_full, o_ready, o_empty, drain;
   uint32_t tmem_base;
 };
@@ -114,12 +116,13 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
       mbar_init(&meta->item_empty[i], 32 + 32 + 1 + 128);
       mbar_init(&meta->q_full[i], 1);
       mbar_init(&meta->q_empty[i], 1);
-      mbar_init(&meta->k_full[i], 32);
-      mbar_init(&meta->k_empty[i], 1);
       mbar_init(&meta->v_full[i], 32);
       mbar_init(&meta->v_empty[i], 1);
       mbar_init(&meta->s_full[i], 1);
-      mbar_init(&meta->s_empty[i], 128);
+    }
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&meta->k_full[i], 32);
+      mbar_init(&meta->k_empty[i], 1);
     }
     mbar_init(&meta->p_full, 128);
     mbar_init(&meta->o_ready, 1);
@@ -139,7 +142,6 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
   const uint32_t tmem = meta->tmem_base;
   const int n_tiles = ws.ctrl[4];
   const uint32_t sQ = smem_u32(smem + C::kOffQ);
-  const uint32_t sP = smem_u32(smem + C::kOffP);
   const uint32_t sK = smem_u32(smem + C::kOffK);
   const uint32_t sV = smem_u32(smem + C::kOffV);
 
@@ -193,6 +195,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
     const uint32_t sbase = is_v ? sV : sK;
     uint64_t* full = is_v ? meta->v_full : meta->k_full;
     uint64_t* empty = is_v ? meta->v_empty : meta->k_empty;
+    const int nst = is_v ? C::kVStages : C::kKStages;
     int tile_base = 0, pending = -1;
     bool ok = true;
     for (int n = 0; ok; ++n) {
@@ -207,7 +210,8 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
       const int32_t* table = g.block_tables + static_cast<int64_t>(info.b) * g.max_blocks;
       for (int j = 0; j < info.n_kv; ++j) {
         const int t = tile_base + j;
-        const uint32_t dst = sbase + (t & 1) * C::kKVBytes;
+        const int st = t % nst, use = t / nst;  // stage and how often it was used before
+        const uint32_t dst = sbase + st * C::kKVBytes;
         // Lanes are paired (D = 128) or grouped by four (D = 64) on a key so
         // that one warp instruction copies whole 32-byte sectors of 16 (8)
         // keys.  Each lane first resolves its keys' pool rows through the block
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
                                         g.num_kv_heads + info.hk) * D;
           }
         }
-        if (t >= 2 && !wait_warp(&empty[t & 1], ((t >> 1) - 1) & 1)) {
+        if (use >= 1 && !wait_warp(&empty[st], (use - 1) & 1)) {
           ok = false;
           break;
         }
@@ -252,7 +256,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
           // the previous tile's copies are complete once at most this group is in flight
           cp_async_wait<1>();
           fence_proxy_async_smem();
-          mbar_arrive(&full[pending & 1]);
+          mbar_arrive(&full[pending % nst]);
         }
         pending = t;
       }
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
     cp_async_wait<0>();
     if (pending >= 0) {
       fence_proxy_async_smem();
-      mbar_arrive(&full[pending & 1]);
+      mbar_arrive(&full[pending % nst]);
     }
     if (!ok && g.err_word && tg == 0) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
   } else if (warp == 2) {
@@ -280,11 +284,11 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         if (!mbar_wait_bounded(&meta->v_full[t & 1], (t >> 1) & 1, kWaitLimitNs)) return false;
         tc_fence_after();
         const uint32_t vst = sV + (t & 1) * C::kKVBytes;
+        const uint32_t tP = tmem + (t & 1) * 128;  // P packed two bf16 per column
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint64_t a = smem_desc(sP + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024, 2);
           const uint64_t bd = smem_desc(vst + kk * 2048, kHalfBytes, 1024, 2);
-          umma_bf16(tO, a, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tO, tP + kk * 8, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&meta->o_ready);
         umma_commit(&meta->v_empty[t & 1]);
@@ -307,14 +311,12 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         const uint32_t qb = sQ + qbuf * C::kQBytes;
         for (int j = 0; j < info.n_kv && ok; ++j) {
           const int t = tile_base + j;
-          if (!mbar_wait_bounded(&meta->k_full[t & 1], (t >> 1) & 1, kWaitLimitNs) ||
-              (t >= 2 && !mbar_wait_bounded(&meta->s_empty[t & 1], ((t >> 1) - 1) & 1,
-                                            kWaitLimitNs))) {
+          if (!mbar_wait_bounded(&meta->k_full[t % 3], (t / 3) & 1, kWaitLimitNs)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t kst = sK + (t & 1) * C::kKVBytes;
+          const uint32_t kst = sK + (t % 3) * C::kKVBytes;
           const uint32_t tS = tmem + (t & 1) * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -323,7 +325,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
                       id_qk, kk > 0 ? 1u : 0u);
           }
           umma_commit(&meta->s_full[t & 1]);
-          umma_commit(&meta->k_empty[t & 1]);
+          umma_commit(&meta->k_empty[t % 3]);
           if (j == info.n_kv - 1) umma_commit(&meta->q_empty[qbuf]);
           if (j >= 1 && !pv(t - 1, j - 1, n)) ok = false;
         }
@@ -369,8 +371,6 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
         tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&meta->s_empty[t & 1]);  // S buffer free for the MMA of tile t + 2
         if (masked) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -409,33 +409,29 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
             tmem_st_wait();
           }
         }
-        // P = 2^(s * scale_log2 - m_use) as bf16 into shared memory (masked keys
-        // hold -inf and give 0)
+        // P = 2^(s * scale_log2 - m_use) as bf16 over columns 0..63 of this S
+        // buffer (masked keys hold -inf and give 0)
         float psum = 0.f;
+        uint32_t pk[2][32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            // half of the exponentials on the XU (ex2.approx), half on the FMA pipe
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][e]), g.scale_log2, -m_use));
-            const float p1 = exp2_poly(fmaf(__uint_as_float(sr[c][e + 1]), g.scale_log2, -m_use));
+            // three exponentials in four on the XU (ex2.approx), one on the FMA pipe
+            const float x0 = fmaf(__uint_as_float(sr[c][e]), g.scale_log2, -m_use);
+            const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), g.scale_log2, -m_use);
+            const float p0 = fast_exp2(x0);
+            const float p1 = (e & 2) ? exp2_poly(x1) : fast_exp2(x1);
             psum += p0 + p1;
-            pk[e >> 1] = pack_bf16x2(p0, p1);
-          }
-          // keys 32c .. 32c+31 -> half c/2, 16-byte chunks (c&1)*4 .. +3 of this row
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const uint32_t addr = sP + (c >> 1) * kHalfBytes + swz(row, (c & 1) * 4 + q4);
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[q4 * 4]),
-                         "r"(pk[q4 * 4 + 1]), "r"(pk[q4 * 4 + 2]), "r"(pk[q4 * 4 + 3])
-                         : "memory");
+            pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
           }
         }
+        tmem_st32(tS, pk[0]);
+        tmem_st32(tS + 32, pk[1]);
+        tmem_st_wait();
         l = l * alpha + psum;
         m = m_use;
         tc_fence_before();
-        fence_proxy_async_smem();
         mbar_arrive(&meta->p_full);
       }
       if (!ok) break;
