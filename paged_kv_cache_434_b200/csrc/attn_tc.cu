@@ -11,32 +11,33 @@
 // within 2^8 of the one in use (the weights then stay below 256, which bf16
 // and fp32 represent exactly enough), an exact reformulation.
 //
-// Tile = 128 query rows x all keys they see, processed 128 keys at a time.
-// The 128 rows are 128/G consecutive tokens x the G query heads of one KV
-// head (GQA): one K/V tile read serves the whole group.
+// A work item is a pair of 128-row query tiles A and B (each 128/G
+// consecutive tokens x the G query heads of one KV head) that share every
+// 128-key K/V tile: one K/V read serves 256 query rows, which halves the
+// bytes per FLOP that must come from L2.
 //
-// CTA (persistent, one per SM, 8 warps -- two per SM sub-partition, so the
-// softmax threads can hold a whole 128-column S row in registers):
-//   warp 3   scheduler: takes the next tile from the planner's longest-first
-//            list, publishes it in a 2-slot ring, TMA-loads the Q tile
-//            (double-buffered, 128-byte swizzle) for it.
+// CTA (persistent, one per SM, 8 warps):
+//   warp 3   scheduler: takes the next item from the planner's longest-first
+//            list, publishes it in a 2-slot ring and TMA-loads the 256 query
+//            rows (128-byte swizzle) once the previous item's QK^T are done.
 //   warps 0-1  loaders: warp 0 fills the K stages (three), warp 1 the V stages
 //            (two), with 16-byte cp.async copies gathered through the block
 //            table into the 128B-swizzled layout the MMA reads (blocks of 16
 //            keys are too small for efficient TMA boxes).  A K stage is free
-//            again once its QK^T is done, a V stage once its PV is done; each
-//            loader keeps two tiles in flight and announces a tile when it has
-//            issued the next one.
-//   warp 2   allocates TMEM; one thread issues the MMAs: S = Q K^T into one of
-//            two TMEM S buffers (M=128, N=128, K=D), then O += P V into the
-//            TMEM O accumulator (N=D, K=128) with P read from TMEM and V as an
-//            MN-major shared-memory operand.  MMAs of one thread execute in
-//            issue order, and each PV is issued before the QK^T that reuses
-//            its S buffer.
-//   warps 4-7  softmax: thread i owns query row i = TMEM lane i, reads its S
-//            row straight from TMEM (row max and sum need no shuffles),
+//            again once its QK^T are done, a V stage once its PVs are done;
+//            each loader keeps two tiles in flight and announces a tile when
+//            it has issued the next one.
+//   warp 2   allocates TMEM (S_A, S_B, O_A, O_B: 128 columns each); one thread
+//            issues S_X = Q_X K^T (M=128, N=128, K=D) and O_X += P_X V (N=D,
+//            K=128, P from TMEM, V an MN-major shared-memory operand) in the
+//            order QK_A(t), QK_B(t), PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1),
+//            ... so that the tensor core works on one tile while the softmax
+//            handles the other.  MMAs of one thread complete in issue order.
+//   warps 4-7  softmax: thread i owns row i of A and of B (TMEM lane i), reads
+//            its S row straight from TMEM (row max and sum need no shuffles),
 //            writes bf16 P over the first 64 columns of the same S buffer,
-//            rescales O in TMEM when the max moved, and finally writes O / l.
+//            rescales O in TMEM when the max moved (S_X(t) being complete
+//            implies PV_X(t-1) is), and finally writes O / l.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -65,24 +66,23 @@ struct Item {
 template <int D>
 struct Cfg {
   static constexpr int NH = D / 64;
-  static constexpr int kQBytes = NH * kHalfBytes;
-  static constexpr int kKVBytes = NH * kHalfBytes; // one K (or V) tile
+  static constexpr int kQTile = NH * kHalfBytes;     // one 128-row query tile
+  static constexpr int kKVBytes = NH * kHalfBytes;   // one K (or V) tile
   static constexpr int kKStages = 3, kVStages = 2;
-  static constexpr int kOffQ = 0;                   // two Q buffers
-  static constexpr int kOffK = 2 * kQBytes;
+  static constexpr int kOffQ = 0;                    // 256 query rows: per half, A then B
+  static constexpr int kOffK = 2 * kQTile;
   static constexpr int kOffV = kOffK + kKStages * kKVBytes;
   static constexpr int kOffMeta = kOffV + kVStages * kKVBytes;
   static constexpr int kSmem = kOffMeta + 1024 + 1024;  // meta + alignment slack
 };
 
-// barriers in the meta area
 struct Meta {
   Item ring[2];
   uint64_t item_full[2], item_empty[2];
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full, q_empty;
   uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
-  uint64_t s_full[2];
-  uint64_t p_full, o_ready, o_empty, drain;
+  uint64_t s_full[2], p_full[2], o_ready[2];  // [tile A, tile B]
+  uint64_t o_empty, drain;
   uint32_t tmem_base;
 };
 
@@ -109,23 +109,24 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
   Meta* meta = reinterpret_cast<Meta*>(smem + C::kOffMeta);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = g.num_heads / g.num_kv_heads;
+  const int Tq = kRows / G;  // tokens per query tile
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&meta->item_full[i], 1);
       mbar_init(&meta->item_empty[i], 32 + 32 + 1 + 128);
-      mbar_init(&meta->q_full[i], 1);
-      mbar_init(&meta->q_empty[i], 1);
       mbar_init(&meta->v_full[i], 32);
       mbar_init(&meta->v_empty[i], 1);
       mbar_init(&meta->s_full[i], 1);
+      mbar_init(&meta->p_full[i], 128);
+      mbar_init(&meta->o_ready[i], 1);
     }
     for (int i = 0; i < 3; ++i) {
       mbar_init(&meta->k_full[i], 32);
       mbar_init(&meta->k_empty[i], 1);
     }
-    mbar_init(&meta->p_full, 128);
-    mbar_init(&meta->o_ready, 1);
+    mbar_init(&meta->q_full, 1);
+    mbar_init(&meta->q_empty, 1);
     mbar_init(&meta->o_empty, 128);
     mbar_init(&meta->drain, 1);
     fence_mbar_init();
@@ -173,17 +174,16 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         meta->ring[slot] = info;
         mbar_arrive(&meta->item_full[slot]);
         if (info.n_kv == 0) break;
-        const int qbuf = n & 1;
-        if (n >= 2 && !mbar_wait_bounded(&meta->q_empty[qbuf], ((n >> 1) - 1) & 1,
-                                         kWaitLimitNs)) {
+        // the 256 query rows: box [64 dims x G heads x 2Tq tokens] per half
+        if (n >= 1 && !mbar_wait_bounded(&meta->q_empty, (n - 1) & 1, kWaitLimitNs)) {
           if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
           break;
         }
-        mbar_arrive_expect_tx(&meta->q_full[qbuf], C::kQBytes);
+        mbar_arrive_expect_tx(&meta->q_full, 2 * C::kQTile);
 #pragma unroll
         for (int dh = 0; dh < NH; ++dh)
-          tma_load_3d(smem + C::kOffQ + qbuf * C::kQBytes + dh * kHalfBytes, &tmQ,
-                      &meta->q_full[qbuf], dh * 64, info.hk * G, info.row0);
+          tma_load_3d(smem + C::kOffQ + dh * 2 * kHalfBytes, &tmQ, &meta->q_full, dh * 64,
+                      info.hk * G, info.row0);
       }
     }
   } else if (warp < 2) {
@@ -273,26 +273,38 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(kRows, kKeys, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(kRows, D, 0, 1);
-      const uint32_t tO = tmem + 256;
-      int tile_base = 0, p_count = 0;
+      int tile_base = 0;
+      int sfa = 0, sfb = 0;  // P tiles consumed per query tile (p_full parity)
       bool ok = true;
-      auto pv = [&](int t, int j, int n) -> bool {
-        if (!mbar_wait_bounded(&meta->p_full, p_count & 1, kWaitLimitNs)) return false;
-        ++p_count;
-        if (j == 0 && n >= 1 && !mbar_wait_bounded(&meta->o_empty, (n - 1) & 1, kWaitLimitNs))
-          return false;
-        if (!mbar_wait_bounded(&meta->v_full[t & 1], (t >> 1) & 1, kWaitLimitNs)) return false;
+      // S_X = Q_X K_t^T, X = 0 (A) or 1 (B)
+      auto qk = [&](int X, int t) {
+        const uint32_t qx = sQ + X * (kRows * 128);
+        const uint32_t kst = sK + (t % 3) * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = (kk >> 2) * 2 * kHalfBytes + (kk & 3) * 32;
+          const uint32_t ko = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          umma_bf16(tmem + X * 128, smem_desc(qx + qo, 16, 1024, 2), smem_desc(kst + ko, 16, 1024, 2),
+                    id_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&meta->s_full[X]);
+      };
+      // O_X += P_X V_t
+      auto pv = [&](int X, int t, bool first) -> bool {
+        int& cnt = X ? sfb : sfa;
+        if (!mbar_wait_bounded(&meta->p_full[X], cnt & 1, kWaitLimitNs)) return false;
+        ++cnt;
         tc_fence_after();
         const uint32_t vst = sV + (t & 1) * C::kKVBytes;
-        const uint32_t tP = tmem + (t & 1) * 128;  // P packed two bf16 per column
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint64_t bd = smem_desc(vst + kk * 2048, kHalfBytes, 1024, 2);
-          umma_bf16_tmem_a(tO, tP + kk * 8, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&meta->o_ready);
-        umma_commit(&meta->v_empty[t & 1]);
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          umma_bf16_tmem_a(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
+                           smem_desc(vst + kk * 2048, kHalfBytes, 1024, 2), id_pv,
+                           (!first || kk > 0) ? 1u : 0u);
         return true;
+      };
+      auto wait_k = [&](int t) {
+        return mbar_wait_bounded(&meta->k_full[t % 3], (t / 3) & 1, kWaitLimitNs);
       };
       for (int n = 0; ok; ++n) {
         const int slot = n & 1;
@@ -303,33 +315,48 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         const Item info = meta->ring[slot];
         mbar_arrive(&meta->item_empty[slot]);
         if (info.n_kv == 0) break;
-        const int qbuf = n & 1;
-        if (!mbar_wait_bounded(&meta->q_full[qbuf], (n >> 1) & 1, kWaitLimitNs)) {
+        const bool hasB = info.ntok > Tq;
+        if (!mbar_wait_bounded(&meta->q_full, n & 1, kWaitLimitNs) || !wait_k(tile_base) ||
+            (n >= 1 && !mbar_wait_bounded(&meta->o_empty, (n - 1) & 1, kWaitLimitNs))) {
           ok = false;
           break;
         }
-        const uint32_t qb = sQ + qbuf * C::kQBytes;
+        tc_fence_after();
+        qk(0, tile_base);
+        if (hasB) qk(1, tile_base);
+        umma_commit(&meta->k_empty[tile_base % 3]);
         for (int j = 0; j < info.n_kv && ok; ++j) {
           const int t = tile_base + j;
-          if (!mbar_wait_bounded(&meta->k_full[t % 3], (t / 3) & 1, kWaitLimitNs)) {
+          const bool more = j + 1 < info.n_kv;
+          if (!mbar_wait_bounded(&meta->v_full[t & 1], (t >> 1) & 1, kWaitLimitNs) ||
+              !pv(0, t, j == 0)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t kst = sK + (t % 3) * C::kKVBytes;
-          const uint32_t tS = tmem + (t & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            umma_bf16(tS, smem_desc(qb + off, 16, 1024, 2), smem_desc(kst + off, 16, 1024, 2),
-                      id_qk, kk > 0 ? 1u : 0u);
+          if (!more) umma_commit(&meta->o_ready[0]);
+          if (more) {
+            if (!wait_k(t + 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            qk(0, t + 1);
           }
-          umma_commit(&meta->s_full[t & 1]);
-          umma_commit(&meta->k_empty[t % 3]);
-          if (j == info.n_kv - 1) umma_commit(&meta->q_empty[qbuf]);
-          if (j >= 1 && !pv(t - 1, j - 1, n)) ok = false;
+          if (hasB) {
+            if (!pv(1, t, j == 0)) {
+              ok = false;
+              break;
+            }
+            if (!more) umma_commit(&meta->o_ready[1]);
+          }
+          umma_commit(&meta->v_empty[t & 1]);
+          if (more) {
+            if (hasB) qk(1, t + 1);
+            umma_commit(&meta->k_empty[(t + 1) % 3]);
+          } else {
+            umma_commit(&meta->q_empty);
+          }
         }
-        if (ok && !pv(tile_base + info.n_kv - 1, info.n_kv - 1, n)) ok = false;
         tile_base += info.n_kv;
       }
       // every MMA issued so far has completed before TMEM is released
@@ -339,10 +366,10 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- softmax (warps 4-7)
-    const int row = tid - 128;                     // query row = TMEM lane
+    const int row = tid - 128;  // query row of A and of B = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tO = tmem + lane_addr + 256;
-    int tile_base = 0, o_count = 0;
+    int cnt[2] = {0, 0};        // S tiles consumed per query tile (s_full parity)
+    int items_x[2] = {0, 0};    // items that had query tile A / B (o_ready parity)
     bool ok = true;
     for (int n = 0; ok; ++n) {
       const int slot = n & 1;
@@ -353,50 +380,45 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
       const Item info = meta->ring[slot];
       mbar_arrive(&meta->item_empty[slot]);
       if (info.n_kv == 0) break;
-      const int tok = row / G;
-      const int pos = info.first_pos + tok;  // this row's position
-      float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < info.n_kv; ++j) {
-        const int t = tile_base + j;
-        const uint32_t tS = tmem + lane_addr + (t & 1) * 128;
-        if (!wait_warp(&meta->s_full[t & 1], (t >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const bool masked = j * kKeys + kKeys - 1 > info.first_pos;
-        const int lim = pos - j * kKeys;  // keys c <= lim are visible
-        // the whole S row in one round trip: 4 loads of 32 columns, one wait
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-        tmem_ld_wait();
-        if (masked) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c * 32 + e > lim) sr[c][e] = 0xff800000u;  // -inf
-        }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
-        mx *= g.scale_log2;
-        const bool rescale = mx > m + kRescaleLog2;
-        const float m_use = rescale ? mx : m;
-        const float alpha = rescale ? fast_exp2(m - m_use) : 1.f;
-        // the previous PV must be done before P is overwritten and O rescaled
-        if (j >= 1) {
-          if (!wait_warp(&meta->o_ready, o_count & 1)) {
+      const int nX = info.ntok > Tq ? 2 : 1;
+      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      for (int j = 0; j < info.n_kv && ok; ++j) {
+#pragma unroll 1
+        for (int X = 0; X < nX; ++X) {
+          const uint32_t tS = tmem + lane_addr + X * 128;
+          const uint32_t tO = tmem + lane_addr + 256 + X * 128;
+          if (!wait_warp(&meta->s_full[X], cnt[X] & 1)) {
             ok = false;
             break;
           }
-          ++o_count;
+          ++cnt[X];
           tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
-            // rare after the first tiles: 32 columns at a time keeps registers low
+          const int pos = info.first_pos + X * Tq + row / G;  // this row's position
+          const bool masked = j * kKeys + kKeys - 1 > info.first_pos + X * Tq;
+          const int lim = pos - j * kKeys;  // keys c <= lim are visible
+          // the whole S row in one round trip: 4 loads of 32 columns, one wait
+          uint32_t sr[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+          tmem_ld_wait();
+          if (masked) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (c * 32 + e > lim) sr[c][e] = 0xff800000u;  // -inf
+          }
+          float mx = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+          mx *= g.scale_log2;
+          const bool rescale = mx > m[X] + kRescaleLog2;
+          const float m_use = rescale ? mx : m[X];
+          const float alpha = rescale ? fast_exp2(m[X] - m_use) : 1.f;
+          // S_X(t) complete implies PV_X(t-1) complete: O_X is stable here
+          if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
               uint32_t orr[32];
@@ -408,72 +430,75 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
             }
             tmem_st_wait();
           }
-        }
-        // P = 2^(s * scale_log2 - m_use) as bf16 over columns 0..63 of this S
-        // buffer (masked keys hold -inf and give 0)
-        float psum = 0.f;
-        uint32_t pk[2][32];
+          // P = 2^(s * scale_log2 - m_use) as bf16 over columns 0..63 of S_X
+          float psum = 0.f;
+          uint32_t pk[2][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 4; ++c) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            // three exponentials in four on the XU (ex2.approx), one on the FMA pipe
-            const float x0 = fmaf(__uint_as_float(sr[c][e]), g.scale_log2, -m_use);
-            const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), g.scale_log2, -m_use);
-            const float p0 = fast_exp2(x0);
-            const float p1 = (e & 2) ? exp2_poly(x1) : fast_exp2(x1);
-            psum += p0 + p1;
-            pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+            for (int e = 0; e < 32; e += 2) {
+              // three exponentials in four on the XU (ex2.approx), one on the FMA pipe
+              const float x0 = fmaf(__uint_as_float(sr[c][e]), g.scale_log2, -m_use);
+              const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), g.scale_log2, -m_use);
+              const float p0 = fast_exp2(x0);
+              const float p1 = (e & 2) ? exp2_poly(x1) : fast_exp2(x1);
+              psum += p0 + p1;
+              pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+            }
           }
+          tmem_st32(tS, pk[0]);
+          tmem_st32(tS + 32, pk[1]);
+          tmem_st_wait();
+          l[X] = l[X] * alpha + psum;
+          m[X] = m_use;
+          tc_fence_before();
+          mbar_arrive(&meta->p_full[X]);
         }
-        tmem_st32(tS, pk[0]);
-        tmem_st32(tS + 32, pk[1]);
-        tmem_st_wait();
-        l = l * alpha + psum;
-        m = m_use;
-        tc_fence_before();
-        mbar_arrive(&meta->p_full);
       }
       if (!ok) break;
-      // epilogue: O / l for the rows of real tokens
-      if (!wait_warp(&meta->o_ready, o_count & 1)) {
-        ok = false;
-        break;
-      }
-      ++o_count;
-      tc_fence_after();
-      const float inv = 1.f / l;
-      const bool store = tok < info.ntok;
-      const int64_t obase =
-          (static_cast<int64_t>(info.row0 + tok) * g.num_heads + info.hk * G + row % G) * D;
+      // epilogue: O_X / l_X for the rows of real tokens
+      for (int X = 0; X < nX; ++X) {
+        if (!wait_warp(&meta->o_ready[X], items_x[X]++ & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tO = tmem + lane_addr + 256 + X * 128;
+        const int tok = X * Tq + row / G;
+        const float inv = 1.f / l[X];
+        const bool store = tok < info.ntok;
+        const int64_t obase =
+            (static_cast<int64_t>(info.row0 + tok) * g.num_heads + info.hk * G + row % G) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + c * 32, r);
-        tmem_ld_wait();
-        if (store) {
-          if (g.out_dtype == PA_F32) {
-            float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(g.out) + obase + c * 32);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+          tmem_ld_wait();
+          if (store) {
+            if (g.out_dtype == PA_F32) {
+              float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(g.out) + obase + c * 32);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              o4[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
-                                  __uint_as_float(r[4 * e + 2]) * inv,
-                                  __uint_as_float(r[4 * e + 3]) * inv);
-          } else {
-            uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + obase + c * 32);
+              for (int e = 0; e < 8; ++e)
+                o4[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                                    __uint_as_float(r[4 * e + 2]) * inv,
+                                    __uint_as_float(r[4 * e + 3]) * inv);
+            } else {
+              uint4* o4 =
+                  reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + obase + c * 32);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              o4[e] = make_uint4(
-                  pack_bf16x2(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
-                  pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
-                  pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
-                  pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
+              for (int e = 0; e < 4; ++e)
+                o4[e] = make_uint4(
+                    pack_bf16x2(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
+                    pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
+                    pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
+                    pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
+            }
           }
         }
       }
+      if (!ok) break;
       tc_fence_before();
       mbar_arrive(&meta->o_empty);
-      tile_base += info.n_kv;
     }
     if (!ok && g.err_word && row == 0) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
   }
@@ -515,20 +540,20 @@ bool tc_path_supported(const AttnGeom& g) {
 }
 
 int tc_tokens_per_tile(const AttnGeom& g) {
-  return tck::kRows / (g.num_heads / g.num_kv_heads);
+  return 2 * tck::kRows / (g.num_heads / g.num_kv_heads);  // a pair of query tiles
 }
 
 template <int D>
 static cudaError_t launch_tc_t(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {
   using C = tck::Cfg<D>;
   const int G = g.num_heads / g.num_kv_heads;
-  // q viewed as (dim, head, token); one box = 64 dims x G heads x 128/G tokens
+  // q viewed as (dim, head, token); one box = 64 dims x G heads x 256/G tokens
   CUtensorMap tq;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(g.num_heads),
                         static_cast<cuuint64_t>(g.num_qrows)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                            static_cast<cuuint64_t>(D) * 2 * g.num_heads};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(tck::kRows / G)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(2 * tck::kRows / G)};
   cuuint32_t estr[3] = {1, 1, 1};
   if (encode_fn_tc()(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(g.q), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
