@@ -408,11 +408,16 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
               for (int e = 0; e < 32; ++e)
                 if (c * 32 + e > lim) sr[c][e] = 0xff800000u;  // -inf
           }
-          float mx = -INFINITY;
+          // row max: four independent chains of 3-input maxima
+          float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+            for (int e = 0; e < 32; e += 8)
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mq[k] = fmax3(mq[k], __uint_as_float(sr[c][e + 2 * k]), __uint_as_float(sr[c][e + 2 * k + 1]));
+          float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
           mx *= g.scale_log2;
           const bool rescale = mx > m[X] + kRescaleLog2;
           const float m_use = rescale ? mx : m[X];
@@ -430,22 +435,30 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
             }
             tmem_st_wait();
           }
-          // P = 2^(s * scale_log2 - m_use) as bf16 over columns 0..63 of S_X
-          float psum = 0.f;
+          // P = 2^(s * scale_log2 - m_use) as bf16 over columns 0..63 of S_X;
+          // scaling and the row sum on packed f32x2 pairs, four sum chains
+          const uint64_t sl2 = f2_pack(g.scale_log2, g.scale_log2);
+          const uint64_t nm2 = f2_pack(-m_use, -m_use);
+          uint64_t acc[4] = {0, 0, 0, 0};
           uint32_t pk[2][32];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sl2, nm2),
+                        x0, x1);
               // three exponentials in four on the XU (ex2.approx), one on the FMA pipe
-              const float x0 = fmaf(__uint_as_float(sr[c][e]), g.scale_log2, -m_use);
-              const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), g.scale_log2, -m_use);
               const float p0 = fast_exp2(x0);
               const float p1 = (e & 2) ? exp2_poly(x1) : fast_exp2(x1);
-              psum += p0 + p1;
+              acc[(e >> 1) & 3] = f2_add(acc[(e >> 1) & 3], f2_pack(p0, p1));
               pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
             }
           }
+          float a0, a1, b0, b1;
+          f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+          f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
+          const float psum = (a0 + b0) + (a1 + b1);
           tmem_st32(tS, pk[0]);
           tmem_st32(tS + 32, pk[1]);
           tmem_st_wait();
