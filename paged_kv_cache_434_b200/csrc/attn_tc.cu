@@ -16,7 +16,8 @@
 // 128-key K/V tile: one K/V read serves 256 query rows, which halves the
 // bytes per FLOP that must come from L2.
 //
-// CTA (persistent, one per SM, 8 warps):
+// CTA (persistent, one per SM, 12 warps in three warpgroups; the first gives
+// registers to the two softmax warpgroups: 128 x 104 + 256 x 200 = 384 x 168):
 //   warp 3   scheduler: takes the next item from the planner's longest-first
 //            list, publishes it in a 2-slot ring and TMA-loads the 256 query
 //            rows (128-byte swizzle) once the previous item's QK^T are done.
@@ -33,11 +34,12 @@
 //            order QK_A(t), QK_B(t), PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1),
 //            ... so that the tensor core works on one tile while the softmax
 //            handles the other.  MMAs of one thread complete in issue order.
-//   warps 4-7  softmax: thread i owns row i of A and of B (TMEM lane i), reads
-//            its S row straight from TMEM (row max and sum need no shuffles),
-//            writes bf16 P over the first 64 columns of the same S buffer,
-//            rescales O in TMEM when the max moved (S_X(t) being complete
-//            implies PV_X(t-1) is), and finally writes O / l.
+//   warps 4-7 (tile A) and 8-11 (tile B)  softmax, the two tiles concurrently:
+//            thread i owns row i (TMEM lane i), reads its S row straight from
+//            TMEM (row max and sum need no shuffles), writes bf16 P over the
+//            first 64 columns of the same S buffer, rescales O in TMEM when the
+//            max moved (S_X(t) being complete implies PV_X(t-1) is), and
+//            finally writes O / l.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -51,7 +53,7 @@ namespace tck {
 
 constexpr int kRows = 128;     // query rows per tile
 constexpr int kKeys = 128;     // keys per KV tile
-constexpr int kThreads = 256;  // 8 warps
+constexpr int kThreads = 384;  // 12 warps
 constexpr int kHalfBytes = 128 * 128;  // [128 rows x 64 bf16]
 constexpr float kRescaleLog2 = 8.f;
 
@@ -114,7 +116,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&meta->item_full[i], 1);
-      mbar_init(&meta->item_empty[i], 32 + 32 + 1 + 128);
+      mbar_init(&meta->item_empty[i], 32 + 32 + 1 + 256);
       mbar_init(&meta->v_full[i], 32);
       mbar_init(&meta->v_empty[i], 1);
       mbar_init(&meta->s_full[i], 1);
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
     }
     mbar_init(&meta->q_full, 1);
     mbar_init(&meta->q_empty, 1);
-    mbar_init(&meta->o_empty, 128);
+    mbar_init(&meta->o_empty, 256);
     mbar_init(&meta->drain, 1);
     fence_mbar_init();
     prefetch_tmap(&tmQ);
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
 
   if (warp == 3) {
     // ---------------------------------------------------------- scheduler
+    regs_dec<104>();
     if (lane == 0) {
       for (int n = 0;; ++n) {
         const int it = atomicAdd(&ws.ctrl[3], 1);
@@ -188,6 +191,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
     }
   } else if (warp < 2) {
     // ---------------------------------------------------------- loaders
+    regs_dec<104>();
     const bool is_v = warp == 1;
     const int tg = lane;
     const int bshift = __ffs(g.block_size) - 1;  // block sizes are powers of two
@@ -270,6 +274,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
     if (!ok && g.err_word && tg == 0) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
   } else if (warp == 2) {
     // ---------------------------------------------------------- MMA issuer
+    regs_dec<104>();
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16_f32(kRows, kKeys, 0, 0);
       const uint32_t id_pv = idesc_bf16_f32(kRows, D, 0, 1);
@@ -365,11 +370,15 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
       if (!ok && g.err_word) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
     }
   } else {
-    // ---------------------------------------------------------- softmax (warps 4-7)
-    const int row = tid - 128;  // query row of A and of B = TMEM lane
+    // ---------------------------------------------------------- softmax
+    regs_inc<200>();
+    const int X = warp >= 8 ? 1 : 0;  // query tile of this warpgroup
+    const int row = (tid - 128) & 127;  // query row = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    int cnt[2] = {0, 0};        // S tiles consumed per query tile (s_full parity)
-    int items_x[2] = {0, 0};    // items that had query tile A / B (o_ready parity)
+    const uint32_t tS = tmem + lane_addr + X * 128;
+    const uint32_t tO = tmem + lane_addr + 256 + X * 128;
+    int cnt = 0;      // S tiles consumed (s_full parity)
+    int items_x = 0;  // items that had this query tile (o_ready parity)
     bool ok = true;
     for (int n = 0; ok; ++n) {
       const int slot = n & 1;
@@ -380,18 +389,15 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
       const Item info = meta->ring[slot];
       mbar_arrive(&meta->item_empty[slot]);
       if (info.n_kv == 0) break;
-      const int nX = info.ntok > Tq ? 2 : 1;
-      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-      for (int j = 0; j < info.n_kv && ok; ++j) {
-#pragma unroll 1
-        for (int X = 0; X < nX; ++X) {
-          const uint32_t tS = tmem + lane_addr + X * 128;
-          const uint32_t tO = tmem + lane_addr + 256 + X * 128;
-          if (!wait_warp(&meta->s_full[X], cnt[X] & 1)) {
+      const bool active = X == 0 || info.ntok > Tq;  // tile B may be empty
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; active && j < info.n_kv && ok; ++j) {
+        {
+          if (!wait_warp(&meta->s_full[X], cnt & 1)) {
             ok = false;
             break;
           }
-          ++cnt[X];
+          ++cnt;
           tc_fence_after();
           const int pos = info.first_pos + X * Tq + row / G;  // this row's position
           const bool masked = j * kKeys + kKeys - 1 > info.first_pos + X * Tq;
@@ -419,9 +425,9 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
                 mq[k] = fmax3(mq[k], __uint_as_float(sr[c][e + 2 * k]), __uint_as_float(sr[c][e + 2 * k + 1]));
           float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
           mx *= g.scale_log2;
-          const bool rescale = mx > m[X] + kRescaleLog2;
-          const float m_use = rescale ? mx : m[X];
-          const float alpha = rescale ? fast_exp2(m[X] - m_use) : 1.f;
+          const bool rescale = mx > m + kRescaleLog2;
+          const float m_use = rescale ? mx : m;
+          const float alpha = rescale ? fast_exp2(m - m_use) : 1.f;
           // S_X(t) complete implies PV_X(t-1) complete: O_X is stable here
           if (j >= 1 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
@@ -462,23 +468,22 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
           tmem_st32(tS, pk[0]);
           tmem_st32(tS + 32, pk[1]);
           tmem_st_wait();
-          l[X] = l[X] * alpha + psum;
-          m[X] = m_use;
+          l = l * alpha + psum;
+          m = m_use;
           tc_fence_before();
           mbar_arrive(&meta->p_full[X]);
         }
       }
       if (!ok) break;
       // epilogue: O_X / l_X for the rows of real tokens
-      for (int X = 0; X < nX; ++X) {
-        if (!wait_warp(&meta->o_ready[X], items_x[X]++ & 1)) {
+      if (active) {
+        if (!wait_warp(&meta->o_ready[X], items_x++ & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t tO = tmem + lane_addr + 256 + X * 128;
         const int tok = X * Tq + row / G;
-        const float inv = 1.f / l[X];
+        const float inv = 1.f / l;
         const bool store = tok < info.ntok;
         const int64_t obase =
             (static_cast<int64_t>(info.row0 + tok) * g.num_heads + info.hk * G + row % G) * D;
