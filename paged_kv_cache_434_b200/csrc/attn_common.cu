@@ -116,12 +116,35 @@ __device__ __forceinline__ void fill_row(const AttnGeom& g, const WsView& ws, bo
   units_max = max(units_max, units);
 }
 
+// Longest run of leading block-table entries shared by every request (decode
+// batches), limited so that each request keeps at least one key of its own.
+// Cooperative over the CTA; returns 0 quickly when column 0 already differs.
+__device__ int shared_prefix_blocks(const AttnGeom& g, int max_cols, int* s_bad) {
+  if (threadIdx.x == 0) *s_bad = max_cols;
+  __syncthreads();
+  constexpr int kChunk = 32;
+  for (int c0 = 0; c0 < max_cols; c0 += kChunk) {
+    const int c1 = min(c0 + kChunk, max_cols);
+    const int pairs = (c1 - c0) * g.num_seqs;
+    for (int idx = threadIdx.x; idx < pairs; idx += blockDim.x) {
+      const int j = c0 + idx / g.num_seqs, b = idx % g.num_seqs;
+      if (g.block_tables[static_cast<int64_t>(b) * g.max_blocks + j] != g.block_tables[j])
+        atomicMin(s_bad, j);
+    }
+    __syncthreads();
+    if (*s_bad < c1) break;
+  }
+  const int r = *s_bad;
+  __syncthreads();
+  return r;
+}
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs a, WsView ws) {
   grid_launch_dependents();
   __shared__ long long s_sum[32];
   __shared__ int s_max[32];
   __shared__ int s_scan[32];
-  __shared__ int s_P, s_merge, s_npref, s_nbig, s_badpref;
+  __shared__ int s_P, s_merge, s_npref, s_nbig, s_badpref, s_minL, s_nbad, s_pbad;
   __shared__ int s_pref[kMaxPrefill];
   __shared__ int s_big[kMaxBig];
   __shared__ int s_hist[kTileBins];
@@ -139,6 +162,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     s_merge = 0;
     s_npref = 0;
     s_nbig = 0;
+    s_minL = 0x7fffffff;
+    s_nbad = 0;
   }
   for (int i = tid; i < kTileBins; i += kPlanThreads) s_hist[i] = 0;
   __syncthreads();
@@ -163,7 +188,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     if (L > max_keys) bits |= PA_ERRBIT_SEQ_TOO_LONG;
     if (bits) {
       if (g.err_word) atomicOr(g.err_word, bits);
+      atomicAdd(&s_nbad, 1);
       continue;  // its rows stay unwritten
+    }
+    if (decode_mode && a.cascade) {
+      // units are counted once the shared prefix is known
+      atomicMin(&s_minL, L);
+      ws.qrow_info[r0] = make_int4(b, L, 1, 0);
+      continue;
     }
     const bool tile = !(decode_mode || q_b == 1 || a.expand_prefill);
     if (tile) {
@@ -235,6 +267,45 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     __syncthreads();
   }
 
+  // 1d. decode cascade: a prefix of blocks shared by every request is attended
+  // once by tensor-core tiles; each row keeps only its own suffix
+  int prefix_tokens = 0, prefix_chunks = 0;
+  if (decode_mode && a.cascade) {
+    __syncthreads();
+    if (s_nbad == 0 && g.num_seqs >= kCascadeMinSeqs && s_minL > kCascadeMinPrefix) {
+      const int max_cols = min((s_minL - 1) / g.block_size, g.max_blocks);
+      const int pb = shared_prefix_blocks(g, max_cols, &s_pbad);
+      if (pb * g.block_size >= kCascadeMinPrefix) prefix_tokens = pb * g.block_size;
+    }
+    for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
+      int4 info = ws.qrow_info[r];
+      if (info.z == 0) continue;
+      info.w = prefix_tokens;
+      ws.qrow_info[r] = info;
+      const int units = (info.y - prefix_tokens + kStageTokens - 1) / kStageTokens;
+      my_units += units;
+      my_max = max(my_max, units);
+    }
+    if (prefix_tokens > 0) {
+      // tiles of (requests x heads) rows; the prefix keys are split into chunks
+      // so that there are about as many tiles as SMs
+      const int per = a.tile_tokens;  // requests per tile pair
+      const int groups = (g.num_seqs + per - 1) / per;
+      const int kv_tiles = (prefix_tokens + 127) / 128;
+      const int base = groups * g.num_kv_heads;
+      const int want = min(min(kMaxPrefixChunks, kv_tiles), max(1, (a.num_sms + base - 1) / base));
+      const int per_chunk = (kv_tiles + want - 1) / want;
+      prefix_chunks = (kv_tiles + per_chunk - 1) / per_chunk;  // no empty chunk
+      for (int idx = tid; idx < base * prefix_chunks; idx += kPlanThreads) {
+        const int c = idx / base, rest = idx % base;
+        const int grp = rest / g.num_kv_heads, hk = rest % g.num_kv_heads;
+        if (idx < ws.max_tiles)
+          ws.tiles[idx] = make_int4(grp * per, hk, min(per, g.num_seqs - grp * per), c);
+      }
+      n_tiles_total = base * prefix_chunks;
+    }
+  }
+
   // partition length
   for (int o = 16; o; o >>= 1) {
     my_units += __shfl_xor_sync(0xffffffffu, my_units, o);
@@ -253,7 +324,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
       mx = max(mx, s_max[w]);
     }
     long long by_target = (total * a.head_groups + a.target_items - 1) / max(a.target_items, 1);
-    long long by_cap = (mx + ws.max_parts - 1) / ws.max_parts;
+    const long long cap =
+        max(1LL, static_cast<long long>(ws.max_parts) - (a.cascade ? kMaxPrefixChunks : 0));
+    long long by_cap = (mx + cap - 1) / cap;
     long long P = max(static_cast<long long>(a.min_part_stages), max(by_target, by_cap));
     s_P = static_cast<int>(max(P, 1LL));
   }
@@ -265,7 +338,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
     const int4 info = ws.qrow_info[r];
     if (info.z == 0) continue;
-    const int units = (info.y + kStageTokens - 1) / kStageTokens;
+    const int units = (info.y - info.w + kStageTokens - 1) / kStageTokens;
     my_items += (units + P - 1) / P * a.head_groups;
   }
   int incl = my_items;
@@ -297,10 +370,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
     const int4 info = ws.qrow_info[r];
     if (info.z == 0) continue;
-    const int units = (info.y + kStageTokens - 1) / kStageTokens;
+    const int units = (info.y - info.w + kStageTokens - 1) / kStageTokens;
     const int np = (units + P - 1) / P;
-    ws.nparts[r] = np;
-    if (np != 1) ws.merge_rows[atomicAdd(&s_merge, 1)] = r;
+    ws.nparts[r] = np + (info.w > 0 ? prefix_chunks : 0);  // the last ones: shared-prefix chunks
+    if (ws.nparts[r] != 1) ws.merge_rows[atomicAdd(&s_merge, 1)] = r;
     for (int p = 0; p < np; ++p)
       for (int hg = 0; hg < a.head_groups; ++hg) ws.items[pos++] = make_int4(r, hg, p, 0);
   }
@@ -336,6 +409,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   if (tid == 0) {
     ws.ctrl[4] = static_cast<int>(min(static_cast<int64_t>(n_tiles_total), ws.max_tiles));
     ws.ctrl[5] = s_merge;
+    ws.ctrl[6] = prefix_tokens;
+    ws.ctrl[7] = prefix_chunks;
   }
 }
 
@@ -404,7 +479,7 @@ __global__ void __launch_bounds__(kGenWarps * 32) attn_generic_kernel(AttnGeom g
     const int r = item.x, hk = item.y, p = item.z;
     const int4 info = ws.qrow_info[r];
     const int b = info.x, key_len = info.y;
-    const int lo = p * P, hi = min(lo + P, key_len);
+    const int lo = info.w + p * P, hi = min(lo + P, key_len);
     for (int idx = tid; idx < G * D; idx += blockDim.x) {
       const int gq = idx / D, d = idx % D;
       s_q[gq][d] = to_f32(q[(static_cast<int64_t>(r) * g.num_heads + hk * G + gq) * D + d]);

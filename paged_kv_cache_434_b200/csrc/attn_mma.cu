@@ -117,8 +117,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         item = ws.items[it];
         qi = ws.qrow_info[item.x];
       }
-      const int lo = item.z * P;
-      const int hi = done ? lo + 1 : min(lo + P, qi.y);
+      const int lo = qi.w + item.z * P;  // partitions start after a shared prefix
+      // lo >= hi: empty item, skipped; never past the table
+      const int hi = done ? lo + 1 : min(min(lo + P, qi.y), g.max_blocks * g.block_size);
       const int32_t* table = g.block_tables + static_cast<int64_t>(qi.x) * g.max_blocks;
       for (int key0 = lo; key0 < hi; key0 += kStageTokens) {
         if (round > 0 && !mbar_wait_bounded(&empty[stage], phase ^ 1, kWaitLimitNs)) {

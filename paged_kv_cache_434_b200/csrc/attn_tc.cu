@@ -16,6 +16,14 @@
 // 128-key K/V tile: one K/V read serves 256 query rows, which halves the
 // bytes per FLOP that must come from L2.
 //
+// The same kernel serves the shared-prefix cascade of a decode batch: when
+// every request's block table starts with the same blocks, the rows of an
+// item are 256/G requests x G heads, all see the whole prefix (no causal
+// mask), and the result is written as a split-KV partial (m, l, unnormalised
+// o) that the log-sum-exp merge combines with the requests' own suffixes
+// ("总结": partials re-normalised with log-sum-exp; "Paged Attention": blocks
+// shared through the block table).
+//
 // CTA (persistent, one per SM, 12 warps in three warpgroups; the first gives
 // registers to the two softmax warpgroups: 128 x 104 + 256 x 200 = 384 x 168):
 //   warp 3   scheduler: takes the next item from the planner's longest-first
@@ -62,7 +70,11 @@ struct Item {
   int n_kv;               // 128-key tiles to visit (0: end of work)
   int first_pos;          // position of the first token
   int row0;               // flattened row of the first token
-  int L;                  // seq_len of the request
+  int L;                  // keys [0, L) exist: seq_len, or the shared prefix length
+  int causal;             // 0: shared-prefix item (every row sees all L keys)
+  int kv0;                // first 128-key tile (shared-prefix chunks)
+  int chunk;              // shared-prefix chunk index
+  int end;                // 1: no more work
 };
 
 template <int D>
@@ -75,7 +87,10 @@ struct Cfg {
   static constexpr int kOffK = 2 * kQTile;
   static constexpr int kOffV = kOffK + kKStages * kKVBytes;
   static constexpr int kOffMeta = kOffV + kVStages * kKVBytes;
-  static constexpr int kSmem = kOffMeta + 1024 + 1024;  // meta + alignment slack
+  // meta + alignment slack; at least 120 KB so that one CTA runs per SM (each
+  // CTA takes all 512 TMEM columns)
+  static constexpr int kSmem0 = kOffMeta + 1024 + 1024;
+  static constexpr int kSmem = kSmem0 > 120 * 1024 ? kSmem0 : 120 * 1024;
 };
 
 struct Meta {
@@ -144,6 +159,8 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
   grid_dependency_wait();
   const uint32_t tmem = meta->tmem_base;
   const int n_tiles = ws.ctrl[4];
+  const int prefix = ws.ctrl[6];  // > 0: decode cascade over a shared prefix
+  const int prefix_chunks = ws.ctrl[7];
   const uint32_t sQ = smem_u32(smem + C::kOffQ);
   const uint32_t sK = smem_u32(smem + C::kOffK);
   const uint32_t sV = smem_u32(smem + C::kOffV);
@@ -155,7 +172,23 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
       for (int n = 0;; ++n) {
         const int it = atomicAdd(&ws.ctrl[3], 1);
         Item info{};
-        if (it < n_tiles) {
+        info.end = it >= n_tiles;
+        if (it < n_tiles && prefix > 0) {
+          const int4 t = ws.tiles[it];  // {first request, kv head, requests}
+          info.b = t.x;
+          info.hk = t.y;
+          info.tok0 = 0;
+          info.ntok = t.z;
+          info.L = prefix;
+          info.first_pos = prefix - 1;
+          info.row0 = t.x;
+          const int kv_all = (prefix + kKeys - 1) / kKeys;
+          const int per_chunk = (kv_all + prefix_chunks - 1) / prefix_chunks;
+          info.kv0 = t.w * per_chunk;
+          info.n_kv = max(0, min(per_chunk, kv_all - info.kv0));
+          info.causal = 0;
+          info.chunk = t.w;
+        } else if (it < n_tiles) {
           const int4 t = ws.tiles[it];
           const int qs = g.query_start_loc[t.x];
           const int qb = g.query_start_loc[t.x + 1] - qs;
@@ -167,6 +200,19 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
           info.first_pos = info.L - qb + t.z;
           info.row0 = qs + t.z;
           info.n_kv = (info.first_pos + t.w - 1) / kKeys + 1;
+          info.causal = 1;
+          info.kv0 = 0;
+        }
+        // an entry that does not describe a valid tile is reported and skipped
+        const int64_t max_keys = static_cast<int64_t>(g.max_blocks) * g.block_size;
+        if (!info.end &&
+            (info.b < 0 || info.b >= g.num_seqs || info.hk < 0 || info.hk >= g.num_kv_heads ||
+             info.ntok < 1 || info.ntok > 2 * Tq || info.n_kv < 1 || info.L > max_keys ||
+             static_cast<int64_t>(info.kv0 + info.n_kv) * kKeys > max_keys + kKeys ||
+             info.row0 < 0 || info.row0 + info.ntok > g.num_qrows)) {
+          if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_QUERY_TOO_LONG);
+          --n;
+          continue;
         }
         const int slot = n & 1;
         if (n >= 2 && !mbar_wait_bounded(&meta->item_empty[slot], ((n >> 1) - 1) & 1,
@@ -176,7 +222,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         }
         meta->ring[slot] = info;
         mbar_arrive(&meta->item_full[slot]);
-        if (info.n_kv == 0) break;
+        if (info.end) break;
         // the 256 query rows: box [64 dims x G heads x 2Tq tokens] per half
         if (n >= 1 && !mbar_wait_bounded(&meta->q_empty, (n - 1) & 1, kWaitLimitNs)) {
           if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
@@ -210,7 +256,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
       }
       const Item info = meta->ring[slot];
       mbar_arrive(&meta->item_empty[slot]);
-      if (info.n_kv == 0) break;
+      if (info.end) break;
       const int32_t* table = g.block_tables + static_cast<int64_t>(info.b) * g.max_blocks;
       for (int j = 0; j < info.n_kv; ++j) {
         const int t = tile_base + j;
@@ -230,7 +276,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         const __nv_bfloat16* rowp[kKeysPerLane];
 #pragma unroll
         for (int q = 0; q < kKeysPerLane; ++q) {
-          const int kpos = j * kKeys + q * kKPI + ksub;
+          const int kpos = (info.kv0 + j) * kKeys + q * kKPI + ksub;
           rowp[q] = nullptr;
           if (kpos < info.L) {
             const int phys = table[kpos >> bshift];
@@ -319,7 +365,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         }
         const Item info = meta->ring[slot];
         mbar_arrive(&meta->item_empty[slot]);
-        if (info.n_kv == 0) break;
+        if (info.end) break;
         const bool hasB = info.ntok > Tq;
         if (!mbar_wait_bounded(&meta->q_full, n & 1, kWaitLimitNs) || !wait_k(tile_base) ||
             (n >= 1 && !mbar_wait_bounded(&meta->o_empty, (n - 1) & 1, kWaitLimitNs))) {
@@ -388,7 +434,7 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
       }
       const Item info = meta->ring[slot];
       mbar_arrive(&meta->item_empty[slot]);
-      if (info.n_kv == 0) break;
+      if (info.end) break;
       const bool active = X == 0 || info.ntok > Tq;  // tile B may be empty
       float m = -INFINITY, l = 0.f;
       for (int j = 0; active && j < info.n_kv && ok; ++j) {
@@ -399,9 +445,11 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
           }
           ++cnt;
           tc_fence_after();
-          const int pos = info.first_pos + X * Tq + row / G;  // this row's position
-          const bool masked = j * kKeys + kKeys - 1 > info.first_pos + X * Tq;
-          const int lim = pos - j * kKeys;  // keys c <= lim are visible
+          // last visible key of this row (causal) or of every row (shared prefix)
+          const int pos = info.causal ? info.first_pos + X * Tq + row / G : info.L - 1;
+          const int kbase = (info.kv0 + j) * kKeys;
+          const bool masked = kbase + kKeys - 1 > (info.causal ? info.first_pos + X * Tq : info.L - 1);
+          const int lim = pos - kbase;  // keys c <= lim are visible
           // the whole S row in one round trip: 4 loads of 32 columns, one wait
           uint32_t sr[4][32];
 #pragma unroll
@@ -487,29 +535,54 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         const bool store = tok < info.ntok;
         const int64_t obase =
             (static_cast<int64_t>(info.row0 + tok) * g.num_heads + info.hk * G + row % G) * D;
+        if (!info.causal) {
+          // shared prefix: one of the request's last split-KV partitions (m, l, o).
+          // Every lane takes part in the TMEM loads; only the stores depend on the row.
+          const int r = info.row0 + tok;
+          const int part = store && r < g.num_qrows ? ws.nparts[r] - prefix_chunks + info.chunk : -1;
+          const bool put = part >= 0 && part < ws.max_parts;
+          if (store && !put && g.err_word) atomicOr(g.err_word, PA_ERRBIT_BLOCK_OOB);
+          const int64_t slot =
+              (static_cast<int64_t>(r) * g.num_heads + info.hk * G + row % G) * ws.max_parts + part;
+          if (put) ws.part_ml[slot] = make_float2(m, l);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + c * 32, r);
-          tmem_ld_wait();
-          if (store) {
-            if (g.out_dtype == PA_F32) {
-              float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(g.out) + obase + c * 32);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r32[32];
+            tmem_ld32(tO + c * 32, r32);
+            tmem_ld_wait();
+            if (put) {
+              float4* po = reinterpret_cast<float4*>(ws.part_o + slot * D + c * 32);
 #pragma unroll
               for (int e = 0; e < 8; ++e)
-                o4[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
-                                    __uint_as_float(r[4 * e + 2]) * inv,
-                                    __uint_as_float(r[4 * e + 3]) * inv);
-            } else {
-              uint4* o4 =
-                  reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + obase + c * 32);
+                po[e] = make_float4(__uint_as_float(r32[4 * e]), __uint_as_float(r32[4 * e + 1]),
+                                    __uint_as_float(r32[4 * e + 2]), __uint_as_float(r32[4 * e + 3]));
+            }
+          }
+        } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                o4[e] = make_uint4(
-                    pack_bf16x2(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
-                    pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
-                    pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
-                    pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+            tmem_ld_wait();
+            if (store) {
+              if (g.out_dtype == PA_F32) {
+                float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(g.out) + obase + c * 32);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  o4[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                                      __uint_as_float(r[4 * e + 2]) * inv,
+                                      __uint_as_float(r[4 * e + 3]) * inv);
+              } else {
+                uint4* o4 =
+                    reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + obase + c * 32);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  o4[e] = make_uint4(
+                      pack_bf16x2(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
+                      pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
+                      pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
+                      pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
+              }
             }
           }
         }

@@ -18,8 +18,12 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 // One attention call's scratch, carved from the caller's workspace buffer.
 //   ctrl      int32[64]   [0] dynamic work counter, [1] number of items,
 //                         [2] partition length in tokens, [3] tile counter,
-//                         [4] number of prefill tiles, [5] rows to merge
-//   qrow_info int4[R]     {request b, key_len, valid, first_key_pos}
+//                         [4] number of tensor-core tiles, [5] rows to merge,
+//                         [6] shared-prefix tokens (decode cascade, 0: none),
+//                         [7] key chunks the shared prefix is split into
+//   qrow_info int4[R]     {request b, key_len, valid, key_start}: the row's
+//                         partitions cover keys [key_start, key_len); keys
+//                         below key_start (a shared prefix) come from tiles
 //   nparts    int32[R]    partitions of the row (0: empty -> zero row;
 //                         -1: invalid -> row left unwritten)
 //   qrow_bad  int32[R]    set when a block id outside the pool was met
@@ -28,7 +32,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 //   part_ml   float2[R*H*P]   per (row, query head, partition): (m, l),
 //                         m in log2 units (score * scale * log2 e)
 //   part_o    float[R*H*P*D]  unnormalised partial outputs
-//   tiles     int4[Tl]    prefill tiles {request b, kv head, first query row, rows}
+//   tiles     int4[Tl]    tensor-core tiles: prefill {request b, kv head, first
+//                         token, tokens}; shared prefix {first request, kv
+//                         head, requests, key chunk}
 struct WsLayout {
   size_t ctrl, qrow_info, nparts, qrow_bad, merge_rows, items, part_ml, part_o, tiles, total;
   int64_t num_qrows, max_parts, max_items, max_tiles;
@@ -83,8 +89,15 @@ struct PlanArgs {
   int32_t target_items;     // aim for about this many items in total
   int32_t min_part_stages;  // lower bound of a partition, in 16-key stages
   int32_t expand_prefill;   // 1: every query of a q_b>1 request is its own row
-  int32_t tile_tokens;      // tokens per prefill tile (when expand_prefill == 0)
+  int32_t tile_tokens;      // tokens (rows of a request) per tensor-core tile pair
+  int32_t cascade;          // decode: attend a prefix shared by all requests once
+  int32_t num_sms;
 };
+
+// Shared-prefix cascade: only worth it for long prefixes and enough requests.
+constexpr int kCascadeMinPrefix = 256;
+constexpr int kCascadeMinSeqs = 16;
+constexpr int kMaxPrefixChunks = 8;  // partitions reserved per row for the shared prefix
 
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error.

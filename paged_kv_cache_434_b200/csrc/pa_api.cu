@@ -40,7 +40,8 @@ static int elt_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
 // workspace-size query and in the call itself.
 struct AttnPlan {
   bool use_mma;
-  bool use_tc;       // prefill requests (q_b > 1) on tcgen05 tiles
+  bool use_tc;       // tcgen05 tiles: prefill requests, or a decode batch's shared prefix
+  bool cascade;      // decode: shared-prefix tiles + suffix partitions
   int tile_tokens;
   int heads_per_group;
   int head_groups;
@@ -81,11 +82,14 @@ static AttnPlan make_plan(int64_t num_qrows, int num_heads, int max_blocks,
   int64_t mp = denom > 0 ? (p.target_items + denom - 1) / denom : 1;
   if (mp > max_units) mp = max_units;
   if (mp < 1) mp = 1;
-  p.max_parts = mp;
-  p.use_tc = mixed && bf16_fast_ok && tc_path_supported(probe);
+  const bool tc_ok = p.use_mma && tc_path_supported(probe);
+  p.cascade = !mixed && tc_ok && num_qrows >= kCascadeMinSeqs;
+  p.use_tc = (mixed && tc_ok) || p.cascade;
+  p.max_parts = mp + (p.cascade ? kMaxPrefixChunks : 0);  // shared-prefix chunks
   p.tile_tokens = p.use_tc ? tc_tokens_per_tile(probe) : 0;
   p.max_tiles = p.use_tc ? ((num_qrows + p.tile_tokens - 1) / p.tile_tokens + num_seqs) *
-                               static_cast<int64_t>(c->num_kv_heads)
+                               static_cast<int64_t>(c->num_kv_heads) *
+                               (p.cascade ? kMaxPrefixChunks : 1)
                          : 0;
   return p;
 }
@@ -145,8 +149,10 @@ static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* works
   a.heads_per_group = p.heads_per_group;
   a.target_items = p.target_items;
   a.min_part_stages = 2;
-  a.expand_prefill = p.use_tc ? 0 : 1;
+  a.expand_prefill = (p.use_tc && !p.cascade) ? 0 : 1;
   a.tile_tokens = p.tile_tokens;
+  a.cascade = p.cascade ? 1 : 0;
+  a.num_sms = p.num_sms;
   if (launch_plan(g, a, ws, s) != cudaSuccess) return PA_ERR_CUDA;
   if (p.use_tc && launch_attn_tc(g, ws, p.num_sms, s) != cudaSuccess) return PA_ERR_CUDA;
   cudaError_t e = p.use_mma ? launch_attn_mma(g, ws, p.num_sms, p.heads_per_group, s)

@@ -101,6 +101,36 @@ def test_mixed_gqa_packings(cuda_device, hq, hkv, D):
     _check_all(w, cuda_device)
 
 
+def _shared_prefix_workload(name, n_seqs, prefix_blocks, suffixes, hq, hkv, d, bs, seed):
+    """Decode batch whose block tables all start with the same physical blocks."""
+    rng = np.random.default_rng(seed)
+    sblocks = [(s + bs - 1) // bs for s in suffixes]
+    nb = prefix_blocks + sum(sblocks) + 3
+    order = rng.permutation(nb).astype(np.int32)
+    width = prefix_blocks + max(sblocks)
+    tables = np.full((n_seqs, width), -1, np.int32)
+    tables[:, :prefix_blocks] = order[:prefix_blocks]
+    c = prefix_blocks
+    for b, n in enumerate(sblocks):
+        tables[b, prefix_blocks:prefix_blocks + n] = order[c:c + n]
+        c += n
+    lens = (prefix_blocks * bs + np.asarray(suffixes)).astype(np.int32)
+    w = W.custom(name, lens, np.ones(n_seqs, np.int32), hq, hkv, d, bs, "bf16", seed=seed)
+    w.block_tables, w.num_blocks = tables, nb
+    return w
+
+
+@pytest.mark.parametrize("hq,hkv,d,bs", [(32, 8, 128, 16), (64, 8, 128, 32), (16, 8, 64, 16),
+                                         (32, 2, 128, 8)])
+def test_shared_prefix_cascade(cuda_device, hq, hkv, d, bs):
+    # 40 requests share a prefix that is not a multiple of 128 keys; the prefix
+    # is attended once by tensor-core tiles and merged with each suffix
+    rng = np.random.default_rng(hq + bs)
+    suffixes = rng.integers(1, 300, size=40).tolist()
+    w = _shared_prefix_workload("prefix_cascade", 40, 600 // bs, suffixes, hq, hkv, d, bs, 17)
+    _check_all(w, cuda_device)
+
+
 def test_bf16_output_variant(cuda_device):
     w = W.custom("bf16_out", [5, 77, 300, 1], [1, 1, 1, 1], 32, 8, 128, 16, "bf16", seed=4)
     _check_all(w, cuda_device, out_dtype=torch.bfloat16)
