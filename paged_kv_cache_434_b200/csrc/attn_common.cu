@@ -293,7 +293,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
       const int groups = (g.num_seqs + per - 1) / per;
       const int kv_tiles = (prefix_tokens + 127) / 128;
       const int base = groups * g.num_kv_heads;
-      const int want = min(min(kMaxPrefixChunks, kv_tiles), max(1, (a.num_sms + base - 1) / base));
+      // one wave: at most one tile per SM
+      const int want = min(min(kMaxPrefixChunks, kv_tiles), max(1, a.num_sms / base));
       const int per_chunk = (kv_tiles + want - 1) / want;
       prefix_chunks = (kv_tiles + per_chunk - 1) / per_chunk;  // no empty chunk
       for (int idx = tid; idx < base * prefix_chunks; idx += kPlanThreads) {
@@ -595,14 +596,63 @@ cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms
 }
 
 // ======================================================================= merge
-// One CTA of 8 warps per (row, query head).  Rows with a single partition were
-// written by the attention kernel; rows with none get zeros; invalid rows are
-// skipped.  The CTA first reduces M = max_k m_k and the denominator over all
-// partitions, keeping the weights 2^(m_k - M) in shared memory, then each warp
-// accumulates every 8th partition's unnormalised output (lanes own D/32
-// columns, 4 partitions in flight) and the 8 warp sums are combined.
+// Rows with a single partition were written by the attention kernel; rows with
+// none get zeros; invalid rows are skipped.  The rows to merge come from the
+// planner's list.  Pass 1: one warp per (row, query head) whose partitions fit
+// in a warp (<= 32): lane k holds partition k's (m, l), the weights
+// 2^(m_k - M) are shuffled to all lanes and each lane accumulates D/32 output
+// columns.  Pass 2: one 8-warp CTA per remaining (row, head): max and
+// denominator reduced over the CTA, then each warp accumulates every 8th
+// partition (4 in flight) and the warp sums are combined.
 constexpr int kMergeWarps = 8;
 constexpr int kMergeCached = 2048;  // partition weights kept in shared memory
+
+template <int D>
+__device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView& ws, int64_t idx,
+                                                int np, int lane) {
+  constexpr int V = D / 32;
+  const int64_t out_base = idx * D + lane * V;
+  if (np == 0) {
+#pragma unroll
+    for (int e = 0; e < V; ++e) store_out(g.out, g.out_dtype, out_base + e, 0.f);
+    return;
+  }
+  const int64_t base = idx * ws.max_parts;
+  const float2 ml = lane < np ? ws.part_ml[base + lane] : make_float2(-INFINITY, 0.f);
+  float M = ml.x;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float c = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
+  float den = c * ml.y;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  const float* po = ws.part_o + base * D + lane * V;
+  int k = 0;
+  for (; k + 3 < np; k += 4) {
+    float x[4][V], ck[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      ck[u] = __shfl_sync(0xffffffffu, c, k + u);
+#pragma unroll
+      for (int e = 0; e < V; ++e) x[u][e] = po[static_cast<int64_t>(k + u) * D + e];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[e] = fmaf(x[u][e], ck[u], acc[e]);
+  }
+  for (; k < np; ++k) {
+    const float ck = __shfl_sync(0xffffffffu, c, k);
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = fmaf(po[static_cast<int64_t>(k) * D + e], ck, acc[e]);
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int e = 0; e < V; ++e) store_out(g.out, g.out_dtype, out_base + e, acc[e] * inv);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(AttnGeom g, WsView ws) {
@@ -613,16 +663,21 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(AttnGeom g, WsV
   grid_dependency_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pairs = static_cast<int64_t>(ws.ctrl[5]) * g.num_heads;
+  // pass 1: (row, head) pairs with at most 32 partitions, one warp each
+  for (int64_t pi = static_cast<int64_t>(blockIdx.x) * kMergeWarps + warp; pi < pairs;
+       pi += static_cast<int64_t>(gridDim.x) * kMergeWarps) {
+    const int r = ws.merge_rows[pi / g.num_heads];
+    const int np = ws.nparts[r];
+    if (np == 1 || np < 0 || np > 32 || ws.qrow_bad[r]) continue;
+    merge_pair_warp<D>(g, ws, static_cast<int64_t>(r) * g.num_heads + pi % g.num_heads, np, lane);
+  }
+  // pass 2: pairs with more partitions, one CTA each
   for (int64_t pi = blockIdx.x; pi < pairs; pi += gridDim.x) {
     const int r = ws.merge_rows[pi / g.num_heads];
     const int64_t idx = static_cast<int64_t>(r) * g.num_heads + pi % g.num_heads;
     const int np = ws.nparts[r];
-    if (np == 1 || np < 0 || ws.qrow_bad[r]) continue;
+    if (np <= 32 || ws.qrow_bad[r]) continue;
     const int64_t out_base = idx * D;
-    if (np == 0) {
-      for (int d = tid; d < D; d += blockDim.x) store_out(g.out, g.out_dtype, out_base + d, 0.f);
-      continue;
-    }
     const int64_t base = idx * ws.max_parts;
     // M
     float M = -INFINITY;
