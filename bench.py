@@ -198,6 +198,19 @@ def byte_counts(w, out_elt=4):
             "step": kv + q + o + cw}
 
 
+def decode_kernel_bytes(w, out_elt=4):
+    """Algorithmic bytes of the decode-partition launch: the K/V rows of the
+    q_b = 1 requests (valid tokens; a block prefix common to every table is
+    left to the tensor-core prefix tiles when the batch has one), their Q rows
+    read and their output rows written."""
+    row = 2 * w.num_kv_heads * w.head_dim * w.elt_bytes
+    dec = [b for b in range(w.num_seqs) if int(w.query_lens[b]) == 1]
+    shared = w.shared_prefix_blocks * w.block_size
+    toks = sum(int(w.seq_lens[b]) - min(shared, int(w.seq_lens[b])) for b in dec)
+    qo = len(dec) * w.num_heads * w.head_dim * (w.elt_bytes + out_elt)
+    return toks * row + qo
+
+
 def prefill_flops(w):
     """Causal-only FLOPs (QK^T and PV, 2 each per MAC) of the q_b > 1 requests."""
     tot = 0
@@ -280,51 +293,6 @@ def oracle_sample(w, pools, seconds: float, rng_seed: int = 0):
 
 # ---------------------------------------------------------------- our arm
 
-def time_prefill_tiles(P, w, t, idx, flush, stream, steps, peaks, flops):
-    """Time the tensor-core prefill tiles alone: a mixed step over only the
-    q_b > 1 requests of the batch (same pools and block tables).  The timed
-    call still includes the planner and two near-empty launches."""
-    qsl = w.query_start_loc
-    pre = [b for b in range(w.num_seqs) if w.query_lens[b] > 1]
-    if not pre:
-        return None
-    rows = np.concatenate([np.arange(qsl[b], qsl[b + 1]) for b in pre])
-    dev = t["q"].device
-    q_sub = t["q"][torch.from_numpy(rows).to(dev)].contiguous()
-    qlens = w.query_lens[pre]
-    qsl_sub = torch.from_numpy(np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)).to(dev)
-    lens_sub = torch.from_numpy(w.seq_lens[pre].copy()).to(dev)
-    tables_sub = torch.from_numpy(np.ascontiguousarray(w.block_tables[pre])).to(dev)
-    out = torch.empty(q_sub.shape, dtype=torch.float32, device=dev)
-    nbytes = P.mixed_step_workspace_size(len(pre), q_sub.shape[0], w.num_heads,
-                                         tables_sub.shape[1], t["k_cache"])
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-
-    def call():
-        P.mixed_step(q_sub, t["k_cache"], t["v_cache"], tables_sub, qsl_sub, lens_sub, w.scale,
-                     out=out, workspace=ws)
-    for _ in range(3):
-        call()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(min(steps, 50))]
-    torch.cuda.synchronize()
-    for a, b in evs:
-        flush.fill_(1)
-        a.record(stream)
-        call()
-        b.record(stream)
-    torch.cuda.synchronize()
-    sec = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
-    tf = flops / sec / 1e12
-    return {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": round(tf, 1),
-            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": round(tf / peaks["bf16_tflops"], 4),
-            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16_tflops, burst: timed alone)",
-            "timed_over": "pa_mixed_step on the prefill requests only (planner + tiles)",
-            "ms": round(sec * 1e3, 4), "algorithmic_flops_per_launch": flops,
-            "traffic": None}
-
-
 def run_ours(args, rank, world, local):
     import paged_kv_cache_434_b200 as P
     from paged_kv_cache_434_b200 import workloads as W
@@ -393,6 +361,21 @@ def run_ours(args, rank, world, local):
     if P.read_error(err) != 0:
         raise RuntimeError("device error bits set during the timed steps")
 
+    # ---- per-launch device times: a pass of its own (events between launches
+    # end their programmatic overlap, so these steps are not the timed ones)
+    n_k = min(args.steps, 50)
+    kt = {}
+    P.kernel_timing(True)
+    try:
+        for _ in range(n_k):
+            flush.fill_(1)
+            step()
+            for k, v in P.kernel_times().items():
+                kt.setdefault(k, []).append(v)
+    finally:
+        P.kernel_timing(False)
+    kernel_ms = {k: round(statistics.mean(v), 4) for k, v in kt.items()}
+
     bc = byte_counts(w)
     metric, unit = metric_of(args.workload)
     if args.workload in ("mixed", "mixed_prefill"):
@@ -401,22 +384,42 @@ def run_ours(args, rank, world, local):
         value = bc["step"] * args.steps * world / total_s / 1e9
     peaks = load_peaks()
     attn_s = statistics.mean(attn_ms) / 1e3
-    achieved = bc["attention"] / attn_s / 1e9
     dominant = "attn_mma_kernel" if w.dtype == "bf16" else "attn_generic_kernel"
     src = "attn_mma.cu" if w.dtype == "bf16" else "attn_common.cu"
+    dk_bytes = decode_kernel_bytes(w)
+    dk_s = kernel_ms["decode"] / 1e3
+    achieved = dk_bytes / dk_s / 1e9
     roofline = {"bound": "hbm", "kernel": dominant,
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)",
-                "timed_over": "the whole attention call (plan + attention + merge launches)",
+                "timed_over": f"the decode-partition launch alone: CUDA events on its stream, "
+                              f"mean of {n_k} launches, L2 flushed before each",
+                "ms": round(dk_s * 1e3, 4),
                 "traffic": kernel_traffic(src, f"{dominant}_{args.workload}.md"),
-                "algorithmic_bytes_per_launch": bc["attention"]}
+                "algorithmic_bytes_per_launch": dk_bytes,
+                "attention_call": {"ms": round(attn_s * 1e3, 4),
+                                   "achieved": round(bc["attention"] / attn_s / 1e9, 1),
+                                   "frac": round(bc["attention"] / attn_s / 1e9 /
+                                                 peaks["hbm_gbs"], 4),
+                                   "bytes": bc["attention"]}}
     extra = {}
     prefill_roofline = None
     if args.workload in ("mixed", "mixed_prefill"):
         fl = prefill_flops(w)
         extra["prefill_flops_per_step"] = fl
-        prefill_roofline = time_prefill_tiles(P, w, t, idx, flush, stream, args.steps, peaks, fl)
+        if "tiles" in kernel_ms:
+            tf = fl / (kernel_ms["tiles"] / 1e3) / 1e12
+            prefill_roofline = {
+                "bound": "tensor", "kernel": "attn_tc_kernel", "achieved": round(tf, 1),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(tf / peaks["bf16_tflops"], 4),
+                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json bf16_tflops, burst: "
+                               f"timed alone)",
+                "timed_over": f"the tensor-core tile launch of the step alone: CUDA events on "
+                              f"its stream, mean of {n_k} launches",
+                "ms": kernel_ms["tiles"], "algorithmic_flops_per_launch": fl,
+                "traffic": kernel_traffic("attn_tc.cu", f"attn_tc_kernel_{args.workload}.md")}
 
     # ---- end to end: host buffers in, result back to the host, each step
     e2e = None
@@ -465,6 +468,8 @@ def run_ours(args, rank, world, local):
             "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": max(args.warmup, 3),
             "ms_per_step": round(total_s * 1e3 / args.steps, 4),
+            "ms_per_step_p10_p50_p90": [round(float(x), 4) for x in
+                                        np.percentile(step_ms, [10, 50, 90])],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype,
             "data": "synthetic: seeded N(0,1) Q/K/V rounded to the dtype, seeded lengths and "
@@ -481,7 +486,8 @@ def run_ours(args, rank, world, local):
             **({"prefill_roofline": prefill_roofline} if prefill_roofline else {}),
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 5 * args.steps,
+            "kernel_ms": kernel_ms,
+            "gpu_launches": (2 + len(kernel_ms)) * args.steps,
             "clocks": clk,
             "wall_s_timed_region": round(wall, 3),
         }

@@ -189,6 +189,31 @@ pa_status pa_decode_no_alloc(const void* q, const void* key_cache, const void* v
                              const pa_cache_desc* cache, int32_t* err_word, void* stream);
 
 /*
+ * pa_kernel_timing_enable / pa_kernel_timing_read -- a measurement aid with no
+ * counterpart on the pages: device time of each launch of one attention call.
+ *   pa_kernel_timing_enable(1) creates PA_TIMED_KERNELS pairs of CUDA events on
+ *   the current device; from then on every pa_decode / pa_mixed_step call made
+ *   on that device records one pair around each of its launches, on the call's
+ *   stream.  A recorded event between two launches ends the overlap that
+ *   programmatic dependent launch otherwise gives them, so timed calls run each
+ *   launch on its own: use it in a pass of its own, not in the timed steps.
+ *   pa_kernel_timing_enable(0) destroys the events.  Not for concurrent use
+ *   from several host threads.
+ *   pa_kernel_timing_read waits for the last timed call's events and writes
+ *   ms[PA_TIMED_KERNELS] (index PA_TK_*); -1 for a launch the call did not
+ *   make.  Returns PA_ERR_INVALID_ARG when timing is off, nothing was timed
+ *   since the last read, or ms is NULL; PA_ERR_CUDA if an event call failed.
+ */
+#define PA_TIMED_KERNELS 4
+#define PA_TK_PLAN 0    /* work planner                                  */
+#define PA_TK_TILES 1   /* tensor-core tiles (prefill or shared prefix)  */
+#define PA_TK_DECODE 2  /* decode partitions                             */
+#define PA_TK_MERGE 3   /* split-KV merge                                */
+
+pa_status pa_kernel_timing_enable(int32_t enable);
+pa_status pa_kernel_timing_read(float* ms);
+
+/*
  * pa_read_error -- synchronise `stream`, copy *err_word to *host_bits and
  * reset it to 0.  Returns PA_OK when no bit was set, PA_ERR_DEVICE when some
  * were, PA_ERR_CUDA if a CUDA call failed (e.g. an earlier kernel faulted).

@@ -20,6 +20,8 @@ from .binding import (  # noqa: F401
     cache_write,
     decode,
     decode_workspace_size,
+    kernel_times,
+    kernel_timing,
     library_path,
     mixed_step,
     mixed_step_workspace_size,

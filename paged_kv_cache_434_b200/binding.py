@@ -27,7 +27,8 @@ ERRBIT_TIMEOUT = 0x10
 
 EXPORTS = ("pa_status_str", "pa_version", "pa_slot_mapping", "pa_cache_write",
            "pa_decode_workspace_size", "pa_decode", "pa_mixed_step_workspace_size",
-           "pa_mixed_step", "pa_read_error", "pa_decode_no_alloc")
+           "pa_mixed_step", "pa_read_error", "pa_decode_no_alloc", "pa_kernel_timing_enable",
+           "pa_kernel_timing_read")
 
 
 class PagedAttentionError(RuntimeError):
@@ -62,7 +63,12 @@ _SIGNATURES = {
     "pa_read_error": ([_vp, ctypes.POINTER(ctypes.c_int32), _vp], ctypes.c_int),
     "pa_decode_no_alloc": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i32, _i32, _i32, _desc_p,
                             _vp, _vp], ctypes.c_int),
+    "pa_kernel_timing_enable": ([_i32], ctypes.c_int),
+    "pa_kernel_timing_read": ([ctypes.POINTER(ctypes.c_float)], ctypes.c_int),
 }
+
+# Launch kinds timed by kernel_timing (PA_TK_* order).
+TIMED_KERNELS = ("plan", "tiles", "decode", "merge")
 
 # Size of the library's static scratch used by decode_no_alloc (PA_DECODE_NO_ALLOC_MAX_BYTES).
 DECODE_NO_ALLOC_MAX_BYTES = 32 << 20
@@ -147,6 +153,18 @@ def read_error(err: torch.Tensor) -> int:
     if st not in (PA_OK, PA_ERR_DEVICE):
         raise PagedAttentionError(st, "pa_read_error")
     return bits.value
+
+
+def kernel_timing(enable: bool) -> None:
+    """Turn per-launch event timing of attention calls on or off (current device)."""
+    _check(_lib().pa_kernel_timing_enable(1 if enable else 0), "pa_kernel_timing_enable")
+
+
+def kernel_times() -> dict:
+    """Device ms of each launch of the last timed attention call (absent: not launched)."""
+    ms = (ctypes.c_float * len(TIMED_KERNELS))()
+    _check(_lib().pa_kernel_timing_read(ms), "pa_kernel_timing_read")
+    return {k: float(v) for k, v in zip(TIMED_KERNELS, ms) if v >= 0}
 
 
 # ---------------------------------------------------------------- operations

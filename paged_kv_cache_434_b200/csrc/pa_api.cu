@@ -5,6 +5,7 @@
 // synchronisation except in pa_read_error.
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "internal.h"
 
@@ -136,6 +137,43 @@ static pa_status check_attn_args(int32_t num_seqs, int64_t num_qrows, int32_t nu
   return PA_OK;
 }
 
+// Per-launch device timing (a measurement aid): one event pair per launch kind,
+// recorded on the call's stream while timing is on for the current device.
+struct LaunchTimer {
+  std::mutex mu;
+  bool on = false;
+  bool pending = false;
+  bool failed = false;
+  int device = -1;
+  bool launched[PA_TIMED_KERNELS] = {};
+  cudaEvent_t ev[2 * PA_TIMED_KERNELS] = {};
+};
+static LaunchTimer g_timer;
+
+class TimedCall {
+ public:
+  explicit TimedCall(cudaStream_t s) : s_(s) {
+    std::lock_guard<std::mutex> lk(g_timer.mu);
+    int dev = -1;
+    if (!g_timer.on || cudaGetDevice(&dev) != cudaSuccess || dev != g_timer.device) return;
+    active_ = true;
+    g_timer.pending = true;
+    g_timer.failed = false;
+    for (bool& l : g_timer.launched) l = false;
+  }
+  void begin(int k) { record(2 * k, k); }
+  void end(int k) { record(2 * k + 1, k); }
+
+ private:
+  void record(int i, int k) {
+    if (!active_) return;
+    if (cudaEventRecord(g_timer.ev[i], s_) != cudaSuccess) g_timer.failed = true;
+    g_timer.launched[k] = true;
+  }
+  cudaStream_t s_;
+  bool active_ = false;
+};
+
 static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* workspace,
                                size_t ws_bytes, cudaStream_t s) {
   const WsLayout L = ws_layout(p.num_qrows, g.num_heads, g.head_dim, p.head_groups, p.max_parts,
@@ -153,12 +191,23 @@ static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* works
   a.tile_tokens = p.tile_tokens;
   a.cascade = p.cascade ? 1 : 0;
   a.num_sms = p.num_sms;
+  TimedCall tm(s);
+  tm.begin(PA_TK_PLAN);
   if (launch_plan(g, a, ws, s) != cudaSuccess) return PA_ERR_CUDA;
-  if (p.use_tc && launch_attn_tc(g, ws, p.num_sms, s) != cudaSuccess) return PA_ERR_CUDA;
+  tm.end(PA_TK_PLAN);
+  if (p.use_tc) {
+    tm.begin(PA_TK_TILES);
+    if (launch_attn_tc(g, ws, p.num_sms, s) != cudaSuccess) return PA_ERR_CUDA;
+    tm.end(PA_TK_TILES);
+  }
+  tm.begin(PA_TK_DECODE);
   cudaError_t e = p.use_mma ? launch_attn_mma(g, ws, p.num_sms, p.heads_per_group, s)
                             : launch_attn_generic(g, ws, p.num_sms, s);
   if (e != cudaSuccess) return PA_ERR_CUDA;
+  tm.end(PA_TK_DECODE);
+  tm.begin(PA_TK_MERGE);
   if (launch_merge(g, ws, p.num_sms, s) != cudaSuccess) return PA_ERR_CUDA;
+  tm.end(PA_TK_MERGE);
   return PA_OK;
 }
 
@@ -280,6 +329,50 @@ pa_status pa_mixed_step(const void* q, const void* key_cache, const void* value_
                                query_start_loc, scale, out, num_seqs, num_tokens, num_heads,
                                max_blocks_per_seq, out_dtype, cache, err_word);
   return run_attention(g, p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_kernel_timing_enable(int32_t enable) {
+  std::lock_guard<std::mutex> lk(g_timer.mu);
+  if (g_timer.on) {
+    int prev = -1;
+    cudaGetDevice(&prev);
+    cudaSetDevice(g_timer.device);
+    for (cudaEvent_t& e : g_timer.ev) {
+      if (e) cudaEventDestroy(e);
+      e = nullptr;
+    }
+    cudaSetDevice(prev);
+    g_timer.on = false;
+    g_timer.pending = false;
+  }
+  if (!enable) return PA_OK;
+  if (cudaGetDevice(&g_timer.device) != cudaSuccess) return PA_ERR_CUDA;
+  for (cudaEvent_t& e : g_timer.ev) {
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      for (cudaEvent_t& f : g_timer.ev) {
+        if (f) cudaEventDestroy(f);
+        f = nullptr;
+      }
+      return PA_ERR_CUDA;
+    }
+  }
+  g_timer.on = true;
+  return PA_OK;
+}
+
+pa_status pa_kernel_timing_read(float* ms) {
+  std::lock_guard<std::mutex> lk(g_timer.mu);
+  if (!ms || !g_timer.on || !g_timer.pending) return PA_ERR_INVALID_ARG;
+  g_timer.pending = false;
+  if (g_timer.failed) return PA_ERR_CUDA;
+  for (int k = 0; k < PA_TIMED_KERNELS; ++k) {
+    ms[k] = -1.f;
+    if (!g_timer.launched[k]) continue;
+    if (cudaEventSynchronize(g_timer.ev[2 * k + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms[k], g_timer.ev[2 * k], g_timer.ev[2 * k + 1]) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  return PA_OK;
 }
 
 pa_status pa_read_error(int32_t* err_word, int32_t* host_bits, void* stream) {

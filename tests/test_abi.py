@@ -142,3 +142,11 @@ def test_product_code_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_kernel_timing_off_paths(lib):
+    from paged_kv_cache_434_b200 import binding as B
+    ms = (ctypes.c_float * 4)()
+    assert lib.pa_kernel_timing_enable(0) == B.PA_OK          # off while off: no CUDA call
+    assert lib.pa_kernel_timing_read(ms) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_kernel_timing_read(None) == B.PA_ERR_INVALID_ARG
