@@ -93,6 +93,7 @@ constexpr int kMaxPrefill = 512;  // prefill requests served by tensor-core tile
 constexpr int kTileBins = 2048;   // longest-first ordering of tiles by 128-key tile count
 constexpr int kInlineRows = 8;    // requests with at most this many rows: one thread
 constexpr int kMaxBig = 1024;     // larger per-row requests: whole CTA, one at a time
+constexpr int kInlineItems = 32;  // rows with more work items: written by the whole CTA
 
 __device__ __forceinline__ int tile_bin(int n_kv) { return n_kv < kTileBins ? n_kv : kTileBins - 1; }
 
@@ -118,21 +119,38 @@ __device__ __forceinline__ void fill_row(const AttnGeom& g, const WsView& ws, bo
 
 // Longest run of leading block-table entries shared by every request (decode
 // batches), limited so that each request keeps at least one key of its own.
-// Cooperative over the CTA; returns 0 quickly when column 0 already differs.
+// Cooperative over the CTA: column 0 alone first (most batches already differ
+// there), then as many columns at once as keeps 16 loads in flight per thread.
 __device__ int shared_prefix_blocks(const AttnGeom& g, int max_cols, int* s_bad) {
+  constexpr int kPer = 16;
   if (threadIdx.x == 0) *s_bad = max_cols;
   __syncthreads();
-  constexpr int kChunk = 32;
-  for (int c0 = 0; c0 < max_cols; c0 += kChunk) {
-    const int c1 = min(c0 + kChunk, max_cols);
+  int c0 = 0, width = 1;
+  while (c0 < max_cols) {
+    const int c1 = min(c0 + width, max_cols);
     const int pairs = (c1 - c0) * g.num_seqs;
-    for (int idx = threadIdx.x; idx < pairs; idx += blockDim.x) {
-      const int j = c0 + idx / g.num_seqs, b = idx % g.num_seqs;
-      if (g.block_tables[static_cast<int64_t>(b) * g.max_blocks + j] != g.block_tables[j])
-        atomicMin(s_bad, j);
+    int v[kPer], ref[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = threadIdx.x + u * blockDim.x;
+      v[u] = ref[u] = 0;
+      if (idx < pairs) {
+        const int j = c0 + idx / g.num_seqs, b = idx % g.num_seqs;
+        v[u] = g.block_tables[static_cast<int64_t>(b) * g.max_blocks + j];
+        ref[u] = g.block_tables[j];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = threadIdx.x + u * blockDim.x;
+      if (idx < pairs && v[u] != ref[u]) atomicMin(s_bad, c0 + idx / g.num_seqs);
     }
     __syncthreads();
+    // later atomics only lower s_bad to columns >= c1, so every thread sees the
+    // same answer to this test
     if (*s_bad < c1) break;
+    c0 = c1;
+    width = max(1, kPer * static_cast<int>(blockDim.x) / max(g.num_seqs, 1));
   }
   const int r = *s_bad;
   __syncthreads();
@@ -141,12 +159,14 @@ __device__ int shared_prefix_blocks(const AttnGeom& g, int max_cols, int* s_bad)
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs a, WsView ws) {
   grid_launch_dependents();
+  grid_dependency_wait();  // seq_lens / tables / the workspace may come from the previous launch
   __shared__ long long s_sum[32];
   __shared__ int s_max[32];
   __shared__ int s_scan[32];
   __shared__ int s_P, s_merge, s_npref, s_nbig, s_badpref, s_minL, s_nbad, s_pbad;
   __shared__ int s_pref[kMaxPrefill];
   __shared__ int s_big[kMaxBig];
+  __shared__ int s_bigpos[kMaxBig];
   __shared__ int s_hist[kTileBins];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool decode_mode = g.query_start_loc == nullptr;
@@ -367,7 +387,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   __syncthreads();
   int pos = s_scan[warp] + incl - my_items;
 
-  // 3. items, partition counts, rows to merge
+  // 3. items, partition counts, rows to merge; a row with many items is listed
+  // and its items written by the whole CTA below (one thread storing hundreds
+  // of items one after another takes tens of microseconds)
+  if (tid == 0) s_nbig = 0;
+  __syncthreads();
   for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
     const int4 info = ws.qrow_info[r];
     if (info.z == 0) continue;
@@ -375,8 +399,28 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     const int np = (units + P - 1) / P;
     ws.nparts[r] = np + (info.w > 0 ? prefix_chunks : 0);  // the last ones: shared-prefix chunks
     if (ws.nparts[r] != 1) ws.merge_rows[atomicAdd(&s_merge, 1)] = r;
+    const int n_it = np * a.head_groups;
+    if (n_it > kInlineItems) {
+      const int slot = atomicAdd(&s_nbig, 1);
+      if (slot < kMaxBig) {
+        s_big[slot] = r;
+        s_bigpos[slot] = pos;
+        pos += n_it;
+        continue;
+      }
+    }
     for (int p = 0; p < np; ++p)
       for (int hg = 0; hg < a.head_groups; ++hg) ws.items[pos++] = make_int4(r, hg, p, 0);
+  }
+  __syncthreads();
+  const int nbig_rows = min(s_nbig, kMaxBig);
+  for (int k = 0; k < nbig_rows; ++k) {
+    const int r = s_big[k];
+    const int4 info = ws.qrow_info[r];
+    const int units = (info.y - info.w + kStageTokens - 1) / kStageTokens;
+    const int n_it = (units + P - 1) / P * a.head_groups;
+    for (int i = tid; i < n_it; i += kPlanThreads)
+      ws.items[s_bigpos[k] + i] = make_int4(r, i % a.head_groups, i / a.head_groups, 0);
   }
 
   // 4. tiles, longest first
@@ -416,8 +460,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
 }
 
 cudaError_t launch_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws, cudaStream_t s) {
-  plan_kernel<<<1, kPlanThreads, 0, s>>>(g, a, ws);
-  return cudaGetLastError();
+  return launch_pdl<plan_kernel>(dim3(1), dim3(kPlanThreads), 0, s, g, a, ws);
 }
 
 // ======================================================================= generic
@@ -577,22 +620,14 @@ __global__ void __launch_bounds__(kGenWarps * 32) attn_generic_kernel(AttnGeom g
 
 cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms,
                                 cudaStream_t s) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(num_sms * 8);
-  cfg.blockDim = dim3(kGenWarps * 32);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  const dim3 grid(num_sms * 8), block(kGenWarps * 32);
   if (g.dtype == PA_F32) {
-    if (g.head_dim == 64) return cudaLaunchKernelEx(&cfg, attn_generic_kernel<float, 64>, g, ws);
-    return cudaLaunchKernelEx(&cfg, attn_generic_kernel<float, 128>, g, ws);
+    if (g.head_dim == 64) return launch_pdl<attn_generic_kernel<float, 64>>(grid, block, 0, s, g, ws);
+    return launch_pdl<attn_generic_kernel<float, 128>>(grid, block, 0, s, g, ws);
   }
   if (g.head_dim == 64)
-    return cudaLaunchKernelEx(&cfg, attn_generic_kernel<__nv_bfloat16, 64>, g, ws);
-  return cudaLaunchKernelEx(&cfg, attn_generic_kernel<__nv_bfloat16, 128>, g, ws);
+    return launch_pdl<attn_generic_kernel<__nv_bfloat16, 64>>(grid, block, 0, s, g, ws);
+  return launch_pdl<attn_generic_kernel<__nv_bfloat16, 128>>(grid, block, 0, s, g, ws);
 }
 
 // ======================================================================= merge
@@ -754,17 +789,9 @@ cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, int num_sms, cudaS
   int64_t blocks = static_cast<int64_t>(g.num_qrows) * g.num_heads;
   if (blocks == 0) return cudaSuccess;
   if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
-  cfg.blockDim = dim3(kMergeWarps * 32);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (g.head_dim == 64) return cudaLaunchKernelEx(&cfg, merge_kernel<64>, g, ws);
-  return cudaLaunchKernelEx(&cfg, merge_kernel<128>, g, ws);
+  const dim3 grid(static_cast<unsigned>(blocks)), block(kMergeWarps * 32);
+  if (g.head_dim == 64) return launch_pdl<merge_kernel<64>>(grid, block, 0, s, g, ws);
+  return launch_pdl<merge_kernel<128>>(grid, block, 0, s, g, ws);
 }
 
 }  // namespace pa

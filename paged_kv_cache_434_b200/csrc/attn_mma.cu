@@ -70,7 +70,7 @@ __device__ __forceinline__ uint32_t swz(int key, int chunk) {
 template <int D, int HG>
 __global__ void __launch_bounds__((HG + 1) * 32, 1)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                    AttnGeom g, WsView ws, int box_rows, int heads_per_box) {
+                    AttnGeom g, WsView ws, int box_rows, int heads_per_box, int after_tiles) {
   using C = mmak::Cfg<D, HG>;
   constexpr int NS = C::NS;
   constexpr int NH = C::NH;
@@ -95,10 +95,17 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     prefetch_tmap(&tmV);
   }
   __syncthreads();
-  grid_dependency_wait();
+  // (no early launch_dependents: the merge has no prologue to overlap, and an
+  // early launch of it measured slower than launching it at our completion)
+  // Launched right after the tensor-core tile kernel (after_tiles), this grid
+  // starts once every tile CTA has passed its own wait on the planner, so the
+  // plan is complete; the tiles' results are not read here.  It then runs
+  // beside the tile CTAs still at work and waits for them only before it
+  // exits, so that the merge (which waits for this grid) sees both.
+  if (!after_tiles) grid_dependency_wait();
 
-  const int n_items = ws.ctrl[1];
-  const int P = ws.ctrl[2];
+  const int n_items = __ldcg(&ws.ctrl[1]);
+  const int P = __ldcg(&ws.ctrl[2]);
   const int G = g.num_heads / g.num_kv_heads;
 
   if (warp == HG) {
@@ -114,8 +121,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       const bool done = it >= n_items;
       int4 item = make_int4(0, 0, 0, 0), qi = make_int4(0, 0, 0, 0);
       if (!done) {
-        item = ws.items[it];
-        qi = ws.qrow_info[item.x];
+        item = __ldcg(&ws.items[it]);
+        qi = __ldcg(&ws.qrow_info[item.x]);
       }
       const int lo = qi.w + item.z * P;  // partitions start after a shared prefix
       // lo >= hi: empty item, skipped; never past the table
@@ -348,7 +355,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_BLOCK_OOB);
         }
       } else {
-        const int np = ws.nparts[r];
+        const int np = __ldcg(&ws.nparts[r]);
         if (np == 1) {
           const float i0 = 1.f / l0, i1 = 1.f / l1;
           const int64_t ob = (static_cast<int64_t>(r) * g.num_heads + head) * D;
@@ -401,6 +408,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       phase ^= 1;
     }
   }
+  if (after_tiles) grid_dependency_wait();
 }
 
 // ----------------------------------------------------------------- host side
@@ -460,7 +468,8 @@ bool mma_path_supported(const AttnGeom& g) {
 }
 
 template <int D, int HG>
-static cudaError_t launch_mma_t(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {
+static cudaError_t launch_mma_t(const AttnGeom& g, const WsView& ws, int num_sms, int after_tiles,
+                                cudaStream_t s) {
   using C = mmak::Cfg<D, HG>;
   const int box_rows = g.block_size < kStageTokens ? g.block_size : kStageTokens;
   CUtensorMap tk, tv;
@@ -478,34 +487,26 @@ static cudaError_t launch_mma_t(const AttnGeom& g, const WsView& ws, int num_sms
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(num_sms * per_sm);
-  cfg.blockDim = dim3(C::kThreads);
-  cfg.dynamicSmemBytes = C::kSmem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tk, tv, g, ws, box_rows, heads_per_box);
+  return launch_pdl<attn_mma_kernel<D, HG>>(dim3(num_sms * per_sm), dim3(C::kThreads), C::kSmem,
+                                            s, tk, tv, g, ws, box_rows, heads_per_box,
+                                            after_tiles);
 }
 
 cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,
-                            cudaStream_t s) {
+                            int after_tiles, cudaStream_t s) {
   if (g.head_dim == 128) {
     switch (heads_per_group) {
-      case 8: return launch_mma_t<128, 8>(g, ws, num_sms, s);
-      case 4: return launch_mma_t<128, 4>(g, ws, num_sms, s);
-      case 2: return launch_mma_t<128, 2>(g, ws, num_sms, s);
-      default: return launch_mma_t<128, 1>(g, ws, num_sms, s);
+      case 8: return launch_mma_t<128, 8>(g, ws, num_sms, after_tiles, s);
+      case 4: return launch_mma_t<128, 4>(g, ws, num_sms, after_tiles, s);
+      case 2: return launch_mma_t<128, 2>(g, ws, num_sms, after_tiles, s);
+      default: return launch_mma_t<128, 1>(g, ws, num_sms, after_tiles, s);
     }
   }
   switch (heads_per_group) {
-    case 8: return launch_mma_t<64, 8>(g, ws, num_sms, s);
-    case 4: return launch_mma_t<64, 4>(g, ws, num_sms, s);
-    case 2: return launch_mma_t<64, 2>(g, ws, num_sms, s);
-    default: return launch_mma_t<64, 1>(g, ws, num_sms, s);
+    case 8: return launch_mma_t<64, 8>(g, ws, num_sms, after_tiles, s);
+    case 4: return launch_mma_t<64, 4>(g, ws, num_sms, after_tiles, s);
+    case 2: return launch_mma_t<64, 2>(g, ws, num_sms, after_tiles, s);
+    default: return launch_mma_t<64, 1>(g, ws, num_sms, after_tiles, s);
   }
 }
 

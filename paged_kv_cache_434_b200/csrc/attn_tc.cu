@@ -157,6 +157,9 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   grid_dependency_wait();
+  // after the wait: the next launch may start while tiles run, and relies on
+  // the plan being complete by then
+  grid_launch_dependents();
   const uint32_t tmem = meta->tmem_base;
   const int n_tiles = ws.ctrl[4];
   const int prefix = ws.ctrl[6];  // > 0: decode cascade over a shared prefix
@@ -651,20 +654,8 @@ static cudaError_t launch_tc_t(const AttnGeom& g, const WsView& ws, int num_sms,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = attn_tc_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(num_sms);
-  cfg.blockDim = dim3(tck::kThreads);
-  cfg.dynamicSmemBytes = C::kSmem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tq, g, ws);
+  return launch_pdl<attn_tc_kernel<D>>(dim3(num_sms), dim3(tck::kThreads), C::kSmem, s, tq, g,
+                                       ws);
 }
 
 cudaError_t launch_attn_tc(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {

@@ -8,6 +8,7 @@
 // slot * num_kv_heads * head_dim, so the scatter is one contiguous row copy per
 // token, done with 16-byte vector loads and stores.
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace pa {
 
@@ -18,6 +19,8 @@ __global__ void __launch_bounds__(256) slot_mapping_kernel(
     const int32_t* __restrict__ qsl, const int32_t* __restrict__ seq_lens, int32_t num_seqs,
     int64_t num_tokens, int32_t block_size, int64_t num_blocks, int64_t* __restrict__ slots,
     int32_t* __restrict__ err) {
+  grid_launch_dependents();
+  grid_dependency_wait();  // tables and lengths may come from the previous launch
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (b >= num_seqs) return;
@@ -53,6 +56,8 @@ __global__ void __launch_bounds__(256) cache_write_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ kc,
     uint4* __restrict__ vc, const int64_t* __restrict__ slots, int64_t num_tokens,
     int64_t row_vec, int64_t num_slots, int32_t* __restrict__ err) {
+  grid_launch_dependents();
+  grid_dependency_wait();  // the slots usually come from the previous launch
   const int lane = threadIdx.x & 31;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t t = w >> 1;
@@ -85,10 +90,9 @@ cudaError_t launch_slot_mapping(const int32_t* block_tables, int32_t max_blocks,
   if (num_seqs == 0) return cudaSuccess;
   const int warps = 8;
   dim3 grid((num_seqs + warps - 1) / warps);
-  slot_mapping_kernel<<<grid, warps * 32, 0, s>>>(block_tables, max_blocks, qsl, seq_lens,
-                                                  num_seqs, num_tokens, block_size, num_blocks,
-                                                  slots, err);
-  return cudaGetLastError();
+  return launch_pdl<slot_mapping_kernel>(grid, dim3(warps * 32), 0, s, block_tables, max_blocks,
+                                         qsl, seq_lens, num_seqs, num_tokens, block_size,
+                                         num_blocks, slots, err);
 }
 
 cudaError_t launch_cache_write(const void* k, const void* v, void* kc, void* vc,
@@ -98,10 +102,10 @@ cudaError_t launch_cache_write(const void* k, const void* v, void* kc, void* vc,
   const int warps = 8;
   const int64_t nwarps = 2 * num_tokens;
   dim3 grid(static_cast<unsigned>((nwarps + warps - 1) / warps));
-  cache_write_kernel<<<grid, warps * 32, 0, s>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(kc),
-      static_cast<uint4*>(vc), slots, num_tokens, row_bytes / 16, num_slots, err);
-  return cudaGetLastError();
+  return launch_pdl<cache_write_kernel>(
+      grid, dim3(warps * 32), 0, s, static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+      static_cast<uint4*>(kc), static_cast<uint4*>(vc), slots, num_tokens, row_bytes / 16,
+      num_slots, err);
 }
 
 }  // namespace pa

@@ -3,6 +3,8 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <atomic>
+#include <utility>
 
 #include <cuda_runtime.h>
 
@@ -101,6 +103,43 @@ constexpr int kMaxPrefixChunks = 8;  // partitions reserved per row for the shar
 
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error.
+// Every kernel of a step is launched with programmatic dependent launch
+// allowed: it may become resident while the previous kernel on the stream
+// drains, and reads nothing that kernel wrote before griddepcontrol.wait.
+// Kernels ask for the largest shared-memory carveout, so that a kernel
+// launched early can share an SM with the one before it instead of waiting
+// for the SM to be reconfigured.
+// Each kernel's dynamic shared memory is fixed by its template arguments.
+template <auto Kern, typename... Args>
+inline cudaError_t launch_pdl(dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  static std::atomic<unsigned long long> attrs_set{0};  // one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attrs_set.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess && smem > 48 * 1024)
+      e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attrs_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, Kern, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_slot_mapping(const int32_t* block_tables, int32_t max_blocks,
                                 const int32_t* qsl, const int32_t* seq_lens, int32_t num_seqs,
                                 int64_t num_tokens, int32_t block_size, int64_t num_blocks,
@@ -112,7 +151,7 @@ cudaError_t launch_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws, 
 cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms,
                                 cudaStream_t s);
 cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,
-                            cudaStream_t s);
+                            int after_tiles, cudaStream_t s);
 cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s);
 

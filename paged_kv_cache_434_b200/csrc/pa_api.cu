@@ -201,7 +201,8 @@ static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* works
     tm.end(PA_TK_TILES);
   }
   tm.begin(PA_TK_DECODE);
-  cudaError_t e = p.use_mma ? launch_attn_mma(g, ws, p.num_sms, p.heads_per_group, s)
+  cudaError_t e = p.use_mma ? launch_attn_mma(g, ws, p.num_sms, p.heads_per_group,
+                                              p.use_tc ? 1 : 0, s)
                             : launch_attn_generic(g, ws, p.num_sms, s);
   if (e != cudaSuccess) return PA_ERR_CUDA;
   tm.end(PA_TK_DECODE);
