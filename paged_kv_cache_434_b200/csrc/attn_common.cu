@@ -163,7 +163,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   __shared__ long long s_sum[32];
   __shared__ int s_max[32];
   __shared__ int s_scan[32];
-  __shared__ int s_P, s_merge, s_npref, s_nbig, s_badpref, s_minL, s_nbad, s_pbad;
+  __shared__ int s_P, s_merge, s_npref, s_nbig, s_badpref, s_minL, s_nbad, s_pbad, s_ntc;
+  __shared__ unsigned long long s_tile_kv;
   __shared__ int s_pref[kMaxPrefill];
   __shared__ int s_big[kMaxBig];
   __shared__ int s_bigpos[kMaxBig];
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     s_nbig = 0;
     s_minL = 0x7fffffff;
     s_nbad = 0;
+    s_tile_kv = 0;
   }
   for (int i = tid; i < kTileBins; i += kPlanThreads) s_hist[i] = 0;
   __syncthreads();
@@ -280,7 +282,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
       for (int idx = tid; idx < ntb * g.num_kv_heads; idx += kPlanThreads) {
         const int tb = idx / g.num_kv_heads;
         const int last = min((tb + 1) * a.tile_tokens, q_b) - 1;
-        atomicAdd(&s_hist[tile_bin((L - q_b + last) / 128 + 1)], 1);
+        const int n_kv = (L - q_b + last) / 128 + 1;
+        atomicAdd(&s_hist[tile_bin(n_kv)], 1);
+        // (query tile, key tile) products of this item: one or two query tiles
+        const int halves = last + 1 - tb * a.tile_tokens > a.tile_tokens / 2 ? 2 : 1;
+        atomicAdd(&s_tile_kv, static_cast<unsigned long long>(n_kv * halves));
       }
       n_tiles_total += ntb * g.num_kv_heads;
     }
@@ -350,6 +356,21 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     long long by_cap = (mx + cap - 1) / cap;
     long long P = max(static_cast<long long>(a.min_part_stages), max(by_target, by_cap));
     s_P = static_cast<int>(max(P, 1LL));
+    // CTAs the tensor-core tiles run on.  With decode partitions in the same
+    // call, the tiles take only as many SMs as finish them in about half the
+    // time the (HBM-bound) partitions need, and the partitions start at once
+    // on the other SMs (rough B200 rates: a 128 x 128 query x key product of
+    // head_dim 128 takes ~1.9 us on one SM; decode streams ~6.5 TB/s).
+    int ntc = a.num_sms;
+    if (!a.cascade && total > 0 && s_tile_kv > 0) {
+      const double tile_sm_us = static_cast<double>(s_tile_kv) * 1.9 * g.head_dim / 128.0;
+      const double dec_us = static_cast<double>(total) * kStageTokens * g.num_kv_heads *
+                            g.head_dim * 4.0 / 6.5e6;
+      const double want = 2.0 * tile_sm_us / max(dec_us, 1.0);
+      ntc = static_cast<int>(min(static_cast<double>(a.num_sms), ceil(want)));
+      ntc = max(ntc, min(8, a.num_sms));
+    }
+    s_ntc = ntc;
   }
   __syncthreads();
   const int P = s_P;
@@ -456,6 +477,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     ws.ctrl[5] = s_merge;
     ws.ctrl[6] = prefix_tokens;
     ws.ctrl[7] = prefix_chunks;
+    ws.ctrl[8] = s_ntc;
   }
 }
 

@@ -167,8 +167,12 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
   const uint32_t sQ = smem_u32(smem + C::kOffQ);
   const uint32_t sK = smem_u32(smem + C::kOffK);
   const uint32_t sV = smem_u32(smem + C::kOffV);
+  // the planner may leave part of the SMs to the decode partitions that run
+  // beside the tiles: those CTAs only release their TMEM
+  const bool working = static_cast<int>(blockIdx.x) < ws.ctrl[8];
 
-  if (warp == 3) {
+  if (!working) {
+  } else if (warp == 3) {
     // ---------------------------------------------------------- scheduler
     regs_dec<104>();
     if (lane == 0) {

@@ -22,7 +22,8 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 //                         [2] partition length in tokens, [3] tile counter,
 //                         [4] number of tensor-core tiles, [5] rows to merge,
 //                         [6] shared-prefix tokens (decode cascade, 0: none),
-//                         [7] key chunks the shared prefix is split into
+//                         [7] key chunks the shared prefix is split into,
+//                         [8] CTAs of the tensor-core tile kernel that work
 //   qrow_info int4[R]     {request b, key_len, valid, key_start}: the row's
 //                         partitions cover keys [key_start, key_len); keys
 //                         below key_start (a shared prefix) come from tiles
