@@ -23,7 +23,12 @@ Sources (page title, section):
   * same article, section "总结": Flash-Decoding splits the KV axis and
     re-normalises the pieces with log-sum-exp.
   * ursb.me Field Note "llm-inference-life", blurb: running max m, running
-    denominator l and the exp(m_old - m_new) correction factor.
+    denominator l and the exp(m_old - m_new) correction factor; every pair of
+    Q/K dimensions rotated in the complex plane by m*theta (rotary position
+    embedding, oracle/rope.py).
+  * "AI Infra入门干货总结", sections "Reshape & Cache" (Q/K rotated by the
+    position's rotation, cos_sin_cache [max_position, rotary_dim], then the
+    scatter into the pools) and "附1：模型配置参数" (rope_theta 500000).
 
 Pins: every function here is checked by tests/test_oracle.py against facts
 fixed by the pages or by mathematics (the worked slot example, closed forms,
@@ -50,3 +55,11 @@ from .attention import (  # noqa: F401
     ERR_QUERY_TOO_LONG,
 )
 from .brute import brute_attention  # noqa: F401
+from .rope import (  # noqa: F401
+    ERR_POS_OOB,
+    cos_sin_table,
+    inv_freq,
+    pair_index,
+    rope_cache_write,
+    rotate,
+)
