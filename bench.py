@@ -11,6 +11,11 @@ torchrun (N > 1) every rank runs its own batch on its own GPU (sequences are
 independent: weak scaling, no collective on the data path); the time is the
 max over ranks.  Rank 0 prints one JSON line.
 
+--workload rope_write times the step just upstream instead: slot mapping and
+the rotary embedding of Q/K fused with the cache write, for the 8192 new
+tokens of the mixed chunked-prefill step (Llama-3-8B geometry, rope_theta
+500000).
+
 --impl reference times the CPU oracle (float64 NumPy, the test reference) on
 a bounded sample of the same workload, on this host's cores.
 """
@@ -40,6 +45,7 @@ WORKLOADS = {
     "mixed": ("mixed_step", 4),
     "shared_prefix": ("shared_prefix_decode", 5),
     "mixed_prefill": ("mixed_step_prefill_only", 4),
+    "rope_write": ("mixed_step", 4),   # the mixed step's 8192 new tokens, fused RoPE + cache write
 }
 FLUSH_BYTES = 512 << 20
 
@@ -538,6 +544,171 @@ def run_ours(args, rank, world, local):
 
 # ---------------------------------------------------------------- reference arm
 
+# ---------------------------------------------------------------- fused RoPE + cache write
+
+ROPE_THETA = 500000.0
+
+
+def rope_inputs(w, dev, seed):
+    """New tokens of the step: q/k/v rows, positions, a pool with just room for
+    them (randomly permuted slots, so the scatter is as irregular as a real
+    pool's) and the slot of every token."""
+    rng = np.random.default_rng([seed, 79])
+    T, hq, hkv, d = w.num_tokens, w.num_heads, w.num_kv_heads, w.head_dim
+    pos = np.concatenate([np.arange(w.seq_lens[b] - w.query_lens[b], w.seq_lens[b])
+                          for b in range(w.num_seqs)]).astype(np.int64)
+    nb = (T + w.block_size - 1) // w.block_size + 64
+    slots = rng.permutation(nb * w.block_size)[:T].astype(np.int64)
+    g = torch.Generator(device=dev).manual_seed(seed)
+    mk = lambda *sh: torch.randn(*sh, generator=g, device=dev).to(torch.bfloat16)
+    return {"q": mk(T, hq, d), "k": mk(T, hkv, d), "v": mk(T, hkv, d),
+            "k_cache": torch.zeros(nb, w.block_size, hkv, d, dtype=torch.bfloat16, device=dev),
+            "v_cache": torch.zeros(nb, w.block_size, hkv, d, dtype=torch.bfloat16, device=dev),
+            "positions": torch.from_numpy(pos).to(dev), "slots": torch.from_numpy(slots).to(dev),
+            "max_pos": int(pos.max()) + 1}
+
+
+def rope_bytes(w):
+    """Algorithmic bytes of the fused launch: Q read and written, K and V read
+    and written to the pools, one float32 table row, the position and the slot
+    per token."""
+    T, e = w.num_tokens, w.elt_bytes
+    return T * (2 * w.num_heads * w.head_dim * e + 4 * w.num_kv_heads * w.head_dim * e +
+                w.head_dim * 4 + 16)
+
+
+def run_rope(args, rank, world, local):
+    import paged_kv_cache_434_b200 as P
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = workload_for("rope_write", args.seed + rank)
+    x = rope_inputs(w, dev, args.seed + rank)
+    table = P.rope_cos_sin_cache(x["max_pos"], w.head_dim, ROPE_THETA, device=dev)
+    q_out = torch.empty_like(x["q"])
+    err = P.new_error_word(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        P.rope_cache_write(x["q"], x["k"], x["v"], x["k_cache"], x["v_cache"], x["slots"],
+                           x["positions"], table, neox=True, q_out=q_out, err=err)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    if P.read_error(err) != 0:
+        raise RuntimeError("device error bits set during warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clocks = ClockSampler(dev) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    wall0 = time.perf_counter()
+    for a, b in evs:
+        flush.fill_(1)
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop() if clocks else None
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_s = max_over_ranks(sum(step_ms) / 1e3, world, dev)
+    nbytes = rope_bytes(w)
+    value = nbytes * args.steps * world / total_s / 1e9
+    peaks = load_peaks()
+    k_s = statistics.mean(step_ms) / 1e3        # one launch per step: the kernel's own time
+    achieved = nbytes / k_s / 1e9
+    roofline = {"bound": "hbm", "kernel": "rope_cache_write_kernel", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)",
+                "timed_over": f"the fused launch (the step's only launch): CUDA events on its "
+                              f"stream, mean of {args.steps} launches, L2 flushed before each",
+                "ms": round(k_s * 1e3, 4),
+                "traffic": kernel_traffic("rope.cu", "rope_cache_write_kernel_rope_write.md"),
+                "algorithmic_bytes_per_launch": nbytes}
+    e2e = None
+    if not args.no_e2e:
+        host = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "positions", "slots")}
+        out_h = torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_h.numel() * out_h.element_size()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in ev2:
+            flush.fill_(1)
+            a.record(stream)
+            for n, t in host.items():
+                x[n].copy_(t, non_blocking=True)
+            step()
+            out_h.copy_(q_out, non_blocking=True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / 1e3, world, dev)
+        e2e = {"value": round(nbytes * args.steps * world / e2e_s / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(e2e_s * 1e3 / args.steps, 4)}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = rope_oracle_sample(w, x, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps({
+            "metric": "fused RoPE + cache write GB/s", "value": round(value, 2), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": round(total_s * 1e3 / args.steps, 4),
+            "ms_per_step_p10_p50_p90": [round(float(v), 4) for v in
+                                        np.percentile(step_ms, [10, 50, 90])],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) Q/K/V rounded to bf16, the mixed step's positions, "
+                    "randomly permuted slots",
+            "config": {"workload": "rope_cache_write_llama3_8b_8192_tokens", "num_tokens": w.num_tokens,
+                       "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+                       "head_dim": w.head_dim, "rotary_dim": w.head_dim, "rope_theta": ROPE_THETA,
+                       "pairing": "split-half (neox)", "step_bytes": nbytes,
+                       "l2": "flushed before every step (512 MiB write, outside the events)",
+                       "parallelism": f"replicas x{world} (independent batches per GPU)"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": clk, "wall_s_timed_region": round(wall, 3)}),
+            flush=True)
+
+
+def rope_oracle_sample(w, x, seconds, rng_seed=0):
+    """The oracle's fused step on whole tokens until `seconds` pass (bytes/s
+    of the same algorithmic count)."""
+    import oracle
+    rng = np.random.default_rng(rng_seed)
+    table = oracle.cos_sin_table(x["max_pos"], w.head_dim, ROPE_THETA)
+    T = w.num_tokens
+    order = rng.permutation(T)[:2048]
+    q = x["q"][torch.from_numpy(order).to(x["q"].device)].cpu().to(torch.float64).numpy()
+    k = x["k"][torch.from_numpy(order).to(x["q"].device)].cpu().to(torch.float64).numpy()
+    v = x["v"][torch.from_numpy(order).to(x["q"].device)].cpu().to(torch.float64).numpy()
+    pos = x["positions"].cpu().numpy()[order]
+    nb = 64
+    kp = np.zeros((nb, w.block_size, w.num_kv_heads, w.head_dim))
+    vp = np.zeros_like(kp)
+    slots = np.arange(len(order)) % (nb * w.block_size)
+    done, t0 = 0, time.perf_counter()
+    for i in range(0, len(order), 64):
+        sl = slice(i, i + 64)
+        oracle.rope_cache_write(q[sl], k[sl], v[sl], pos[sl], slots[sl], kp, vp, table,
+                                w.head_dim, True)
+        done += min(64, len(order) - i)
+        if time.perf_counter() - t0 > seconds:
+            break
+    el = time.perf_counter() - t0
+    per_tok = rope_bytes(w) / T
+    return {"value": round(done * per_tok / el / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{done} of the {T} tokens (64 per call), float64 NumPy, one thread"}
+
+
 def run_reference(args, rank, world, local):
     """The CPU oracle timed as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -579,11 +750,54 @@ def run_reference(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+def run_rope_reference(args, rank, world, local):
+    """The oracle's fused RoPE + cache write timed as the reference arm."""
+    if rank != 0:
+        return
+    w = workload_for("rope_write", args.seed)
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    if dev.type == "cuda":
+        x = rope_inputs(w, dev, args.seed)
+    else:
+        x = rope_inputs_cpu(w, args.seed)
+    per_step = max(0.5, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    vals = [rope_oracle_sample(w, x, per_step, rng_seed=k)["value"]
+            for k in range(max(args.warmup, 3) + args.steps)][max(args.warmup, 3):]
+    value = statistics.mean(vals)
+    print(json.dumps({
+        "impl": "reference", "metric": "fused RoPE + cache write GB/s", "value": round(value, 4),
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(rope_bytes(w) / (value * 1e9) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same generator and seed as our arm)",
+        "config": {"workload": "rope_cache_write_llama3_8b_8192_tokens"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: about {per_step:.1f} s of whole tokens"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0}), flush=True)
+
+
+def rope_inputs_cpu(w, seed):
+    rng = np.random.default_rng([seed, 80])
+    T, hq, hkv, d = w.num_tokens, w.num_heads, w.num_kv_heads, w.head_dim
+    pos = np.concatenate([np.arange(w.seq_lens[b] - w.query_lens[b], w.seq_lens[b])
+                          for b in range(w.num_seqs)]).astype(np.int64)
+    mk = lambda *sh: torch.from_numpy(rng.standard_normal(sh, dtype=np.float32)).to(torch.bfloat16)
+    return {"q": mk(T, hq, d), "k": mk(T, hkv, d), "v": mk(T, hkv, d),
+            "positions": torch.from_numpy(pos), "max_pos": int(pos.max()) + 1}
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_setup()
     try:
-        if args.impl == "reference":
+        if args.workload == "rope_write":
+            if args.impl == "reference":
+                run_rope_reference(args, rank, world, local)
+            else:
+                run_rope(args, rank, world, local)
+        elif args.impl == "reference":
             run_reference(args, rank, world, local)
         else:
             run_ours(args, rank, world, local)

@@ -62,6 +62,7 @@ typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
 #define PA_ERRBIT_SEQ_TOO_LONG 0x4    /* seq_len > max_blocks_per_seq * block_size */
 #define PA_ERRBIT_QUERY_TOO_LONG 0x8  /* query_len > seq_len (or negative)         */
 #define PA_ERRBIT_TIMEOUT 0x10        /* a bounded device wait gave up             */
+#define PA_ERRBIT_POS_OOB 0x20        /* a rotary position outside the cos/sin table */
 
 /* One layer's cache pools. */
 typedef struct pa_cache_desc {
@@ -111,6 +112,57 @@ pa_status pa_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_se
 pa_status pa_cache_write(const void* k, const void* v, void* key_cache, void* value_cache,
                          const int64_t* slot_mapping, int64_t num_tokens,
                          const pa_cache_desc* cache, int32_t* err_word, void* stream);
+
+/*
+ * pa_rope_cos_sin_cache -- the rotary table, built once at start-up
+ * ("AI Infra入门干货总结：大模型是如何高效推理的", section "Reshape & Cache":
+ * cos_sin_cache of shape [max_position_embeddings, rotary_dim], indexed by
+ * position at run time so that no sin/cos is evaluated per token).
+ *   cache  float32 [max_position, rotary_dim] (output).  Row p holds
+ *          cos(p * f_i) for i < rotary_dim / 2, then sin(p * f_i), with
+ *          f_i = theta ** (-2 i / rotary_dim); angles, cos and sin in float64,
+ *          rounded once to float32.  rope_theta is 500000 for Llama-3-8B
+ *          (same article, "附1：模型配置参数").
+ * rotary_dim must be even and > 0, max_position > 0, theta > 0.
+ */
+pa_status pa_rope_cos_sin_cache(float* cache, int32_t max_position, int32_t rotary_dim,
+                                double theta, void* stream);
+
+/*
+ * pa_rope_cache_write -- rotary position embedding fused with reshape_and_cache
+ * (same article, "Reshape & Cache": Q and K rotated by the position's rotation,
+ * V unchanged, then K and V scattered into the pools through slot_mapping).
+ * For token t with position p = positions[t] and each rotated pair (x1, x2)
+ * of a Q or K head (angle a_i = p * f_i, cos/sin read from cos_sin_cache):
+ *     (x1, x2) -> (x1 cos a_i - x2 sin a_i, x2 cos a_i + x1 sin a_i)
+ * in float32, rounded to the cache dtype.  Pairs: neox != 0 pairs dimension i
+ * with i + rotary_dim / 2, neox == 0 pairs 2i with 2i + 1; dimensions
+ * >= rotary_dim are copied unchanged.
+ *   q_in   token t's [num_heads, head_dim] row at q_in + t * q_stride
+ *   k, v   token t's [num_kv_heads, head_dim] rows at k / v + t * kv_stride
+ *          (strides in elements; the three may be column slices of one fused
+ *          QKV projection output, e.g. q_stride = kv_stride =
+ *          (num_heads + 2 * num_kv_heads) * head_dim)
+ *   q_out  [num_tokens, num_heads, head_dim] rotated queries; may be q_in
+ *          itself when q_stride == num_heads * head_dim, must not otherwise
+ *          overlap it
+ *   key_cache / value_cache, slot_mapping: as pa_cache_write (rotated K and
+ *          plain V stored at the slot; negative slot = padding, skipped;
+ *          slot past the pool: skipped, PA_ERRBIT_SLOT_OOB)
+ *   positions int64 [num_tokens]; a position outside [0, max_position) sets
+ *          PA_ERRBIT_POS_OOB, copies the token's queries unrotated to q_out
+ *          and writes nothing to the pools
+ *   cos_sin_cache float32 [max_position, rotary_dim] (pa_rope_cos_sin_cache)
+ * rotary_dim: a multiple of 16, at most head_dim.  Strides: multiples of 8
+ * elements.  dtype of q/k/v/q_out: cache->dtype.
+ */
+pa_status pa_rope_cache_write(const void* q_in, const void* k, const void* v, int64_t q_stride,
+                              int64_t kv_stride, void* q_out, void* key_cache, void* value_cache,
+                              const int64_t* positions, const int64_t* slot_mapping,
+                              const float* cos_sin_cache, int32_t max_position,
+                              int32_t rotary_dim, int32_t neox, int64_t num_tokens,
+                              int32_t num_heads, const pa_cache_desc* cache, int32_t* err_word,
+                              void* stream);
 
 /* Bytes of workspace pa_decode needs for these sizes (0 on bad arguments). */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads,

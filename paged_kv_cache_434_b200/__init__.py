@@ -5,6 +5,8 @@ its Python binding plus a seeded workload generator:
 
   slot_mapping   slot of every new token from the block tables
   cache_write    reshape_and_cache into [num_blocks, block_size, Hkv, D] pools
+  rope_cache_write  rotary embedding of Q/K fused with the cache write
+  rope_cos_sin_cache  the [max_position, rotary_dim] cos/sin table
   decode         GQA decode attention, online softmax, split-KV + LSE merge
   mixed_step     causal varlen attention of a chunked-prefill + decode step
   step           slot_mapping -> cache_write -> attention, the per-layer path
@@ -15,6 +17,7 @@ from .binding import (  # noqa: F401
     ERRBIT_QUERY_TOO_LONG,
     ERRBIT_SEQ_TOO_LONG,
     ERRBIT_SLOT_OOB,
+    ERRBIT_POS_OOB,
     ERRBIT_TIMEOUT,
     PagedAttentionError,
     cache_write,
@@ -27,6 +30,8 @@ from .binding import (  # noqa: F401
     mixed_step_workspace_size,
     new_error_word,
     read_error,
+    rope_cache_write,
+    rope_cos_sin_cache,
     slot_mapping,
     version,
 )

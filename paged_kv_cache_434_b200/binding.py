@@ -24,11 +24,12 @@ ERRBIT_BLOCK_OOB = 0x2
 ERRBIT_SEQ_TOO_LONG = 0x4
 ERRBIT_QUERY_TOO_LONG = 0x8
 ERRBIT_TIMEOUT = 0x10
+ERRBIT_POS_OOB = 0x20
 
 EXPORTS = ("pa_status_str", "pa_version", "pa_slot_mapping", "pa_cache_write",
            "pa_decode_workspace_size", "pa_decode", "pa_mixed_step_workspace_size",
            "pa_mixed_step", "pa_read_error", "pa_decode_no_alloc", "pa_kernel_timing_enable",
-           "pa_kernel_timing_read")
+           "pa_kernel_timing_read", "pa_rope_cos_sin_cache", "pa_rope_cache_write")
 
 
 class PagedAttentionError(RuntimeError):
@@ -65,6 +66,9 @@ _SIGNATURES = {
                             _vp, _vp], ctypes.c_int),
     "pa_kernel_timing_enable": ([_i32], ctypes.c_int),
     "pa_kernel_timing_read": ([ctypes.POINTER(ctypes.c_float)], ctypes.c_int),
+    "pa_rope_cos_sin_cache": ([_vp, _i32, _i32, ctypes.c_double, _vp], ctypes.c_int),
+    "pa_rope_cache_write": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+                             _i32, _i64, _i32, _desc_p, _vp, _vp], ctypes.c_int),
 }
 
 # Launch kinds timed by kernel_timing (PA_TK_* order).
@@ -199,6 +203,60 @@ def cache_write(k, v, k_cache, v_cache, slot_mapping, err=None):
         _cuda(k, "k"), _cuda(v, "v"), _cuda(k_cache, "k_cache", ndim=4),
         _cuda(v_cache, "v_cache", ndim=4), _cuda(slot_mapping, "slot_mapping", torch.int64, 1),
         T, ctypes.byref(desc), _err_ptr(err), _stream()), "pa_cache_write")
+
+
+def rope_cos_sin_cache(max_position: int, rotary_dim: int, theta: float, device=None,
+                       out=None) -> torch.Tensor:
+    """float32 [max_position, rotary_dim] rotary table (see pa_rope_cos_sin_cache)."""
+    if out is None:
+        out = torch.empty(max_position, rotary_dim, dtype=torch.float32,
+                          device=device or "cuda")
+    if tuple(out.shape) != (max_position, rotary_dim):
+        raise ValueError("out must be [max_position, rotary_dim]")
+    _check(_lib().pa_rope_cos_sin_cache(_cuda(out, "out", torch.float32, 2), max_position,
+                                        rotary_dim, float(theta), _stream()),
+           "pa_rope_cos_sin_cache")
+    return out
+
+
+def _token_rows(t: torch.Tensor, name: str, heads: int, d: int) -> int:
+    """Token stride (elements) of a [T, heads, d] view whose heads of one token
+    are contiguous (a column slice of a fused QKV output qualifies)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 3 or tuple(t.shape[1:]) != (heads, d) or t.stride(2) != 1 or t.stride(1) != d:
+        raise ValueError(f"{name} must be a [num_tokens, {heads}, {d}] view with contiguous heads")
+    return t.stride(0)
+
+
+def rope_cache_write(q, k, v, k_cache, v_cache, slot_mapping, positions, cos_sin_cache,
+                     neox: bool = True, q_out=None, err=None):
+    """Rotate q and k by their positions, store rotated k and plain v at their
+    slots, return the rotated queries (see pa_rope_cache_write)."""
+    desc = cache_desc(k_cache)
+    T, Hq, D = q.shape
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
+        raise ValueError("v_cache must match k_cache")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != k_cache.dtype or t.shape[0] != T:
+            raise ValueError(f"{name} must have num_tokens rows of the cache dtype")
+    qs = _token_rows(q, "q", Hq, D)
+    ks = _token_rows(k, "k", desc.num_kv_heads, desc.head_dim)
+    if _token_rows(v, "v", desc.num_kv_heads, desc.head_dim) != ks:
+        raise ValueError("k and v must share their token stride")
+    if q_out is None:
+        q_out = torch.empty(T, Hq, D, dtype=q.dtype, device=q.device)
+    if not q_out.is_contiguous() or tuple(q_out.shape) != (T, Hq, D) or q_out.dtype != q.dtype:
+        raise ValueError("q_out must be a contiguous [num_tokens, num_heads, head_dim] tensor")
+    max_pos, rot = cos_sin_cache.shape
+    _check(_lib().pa_rope_cache_write(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), qs, ks, q_out.data_ptr(),
+        _cuda(k_cache, "k_cache", ndim=4), _cuda(v_cache, "v_cache", ndim=4),
+        _cuda(positions, "positions", torch.int64, 1),
+        _cuda(slot_mapping, "slot_mapping", torch.int64, 1),
+        _cuda(cos_sin_cache, "cos_sin_cache", torch.float32, 2), max_pos, rot, 1 if neox else 0,
+        T, Hq, ctypes.byref(desc), _err_ptr(err), _stream()), "pa_rope_cache_write")
+    return q_out
 
 
 def decode_workspace_size(num_seqs, num_heads, max_blocks_per_seq, k_cache) -> int:

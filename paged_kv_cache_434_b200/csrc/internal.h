@@ -141,6 +141,26 @@ inline cudaError_t launch_pdl(dim3 grid, dim3 block, size_t smem, cudaStream_t s
   return cudaLaunchKernelEx(&cfg, Kern, std::forward<Args>(args)...);
 }
 
+struct RopeLaunch {
+  const void* q_in;
+  const void* k;
+  const void* v;
+  int64_t q_stride, kv_stride;
+  void* q_out;
+  void* kc;
+  void* vc;
+  const int64_t* positions;
+  const int64_t* slots;
+  const float* cs;
+  int32_t max_position, rot, neox;
+  int64_t num_tokens;
+  int32_t hq, hkv, d, dtype;
+  int64_t num_slots;
+  int32_t* err;
+};
+cudaError_t launch_rope_table(float* cache, int32_t max_position, int32_t rotary_dim, double theta,
+                              int num_sms, cudaStream_t s);
+cudaError_t launch_rope_cache_write(const RopeLaunch& l, int num_sms, cudaStream_t s);
 cudaError_t launch_slot_mapping(const int32_t* block_tables, int32_t max_blocks,
                                 const int32_t* qsl, const int32_t* seq_lens, int32_t num_seqs,
                                 int64_t num_tokens, int32_t block_size, int64_t num_blocks,

@@ -332,6 +332,74 @@ pa_status pa_mixed_step(const void* q, const void* key_cache, const void* value_
   return run_attention(g, p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
+pa_status pa_rope_cos_sin_cache(float* cache, int32_t max_position, int32_t rotary_dim,
+                                double theta, void* stream) {
+  if (!cache || max_position <= 0 || rotary_dim <= 0 || (rotary_dim & 1) || !(theta > 0.0))
+    return PA_ERR_INVALID_ARG;
+  return launch_rope_table(cache, max_position, rotary_dim, theta, device_num_sms(),
+                           static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PA_OK
+             : PA_ERR_CUDA;
+}
+
+pa_status pa_rope_cache_write(const void* q_in, const void* k, const void* v, int64_t q_stride,
+                              int64_t kv_stride, void* q_out, void* key_cache, void* value_cache,
+                              const int64_t* positions, const int64_t* slot_mapping,
+                              const float* cos_sin_cache, int32_t max_position,
+                              int32_t rotary_dim, int32_t neox, int64_t num_tokens,
+                              int32_t num_heads, const pa_cache_desc* cache, int32_t* err_word,
+                              void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0 || num_heads < 1 || max_position < 1) return PA_ERR_INVALID_ARG;
+  if (rotary_dim < 16 || rotary_dim % 16 || rotary_dim > cache->head_dim)
+    return PA_ERR_UNSUPPORTED;
+  const int64_t D = cache->head_dim;
+  if (q_stride < num_heads * D || kv_stride < cache->num_kv_heads * D || q_stride % 8 ||
+      kv_stride % 8)
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!q_in || !k || !v || !q_out || !key_cache || !value_cache || !positions || !slot_mapping ||
+      !cos_sin_cache)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q_in) || !aligned16(k) || !aligned16(v) || !aligned16(q_out) ||
+      !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(cos_sin_cache))
+    return PA_ERR_INVALID_ARG;
+  // q_out either is q_in (contiguous rows, rotated in place) or does not overlap it
+  const uintptr_t qi = reinterpret_cast<uintptr_t>(q_in), qo = reinterpret_cast<uintptr_t>(q_out);
+  const int64_t eb = elt_bytes(cache->dtype);
+  const uintptr_t q_in_end = qi + static_cast<uintptr_t>(((num_tokens - 1) * q_stride + num_heads * D) * eb);
+  const uintptr_t q_out_end = qo + static_cast<uintptr_t>(num_tokens * num_heads * D * eb);
+  if (qi == qo ? q_stride != num_heads * D : (qo < q_in_end && qi < q_out_end))
+    return PA_ERR_INVALID_ARG;
+  RopeLaunch l{};
+  l.q_in = q_in;
+  l.k = k;
+  l.v = v;
+  l.q_stride = q_stride;
+  l.kv_stride = kv_stride;
+  l.q_out = q_out;
+  l.kc = key_cache;
+  l.vc = value_cache;
+  l.positions = positions;
+  l.slots = slot_mapping;
+  l.cs = cos_sin_cache;
+  l.max_position = max_position;
+  l.rot = rotary_dim;
+  l.neox = neox ? 1 : 0;
+  l.num_tokens = num_tokens;
+  l.hq = num_heads;
+  l.hkv = cache->num_kv_heads;
+  l.d = cache->head_dim;
+  l.dtype = cache->dtype;
+  l.num_slots = cache->num_blocks * cache->block_size;
+  l.err = err_word;
+  return launch_rope_cache_write(l, device_num_sms(), static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? PA_OK
+             : PA_ERR_CUDA;
+}
+
 pa_status pa_kernel_timing_enable(int32_t enable) {
   std::lock_guard<std::mutex> lk(g_timer.mu);
   if (g_timer.on) {
