@@ -26,6 +26,8 @@ Sources (page title, section):
     denominator l and the exp(m_old - m_new) correction factor; every pair of
     Q/K dimensions rotated in the complex plane by m*theta (rotary position
     embedding, oracle/rope.py).
+  * "第三部分 · 推理系统与基础设施" (llm-learning-path part 3), chapter map,
+    3.3: block tables with copy-on-write (oracle/blocks.py).
   * "AI Infra入门干货总结", sections "Reshape & Cache" (Q/K rotated by the
     position's rotation, cos_sin_cache [max_position, rotary_dim], then the
     scatter into the pools) and "附1：模型配置参数" (rope_theta 500000).
@@ -55,6 +57,11 @@ from .attention import (  # noqa: F401
     ERR_QUERY_TOO_LONG,
 )
 from .brute import brute_attention  # noqa: F401
+from .blocks import (  # noqa: F401
+    ERR_POS_OOB_TABLE,
+    copy_blocks,
+    slot_mapping_positions,
+)
 from .rope import (  # noqa: F401
     ERR_POS_OOB,
     cos_sin_table,
