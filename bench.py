@@ -16,6 +16,14 @@ the rotary embedding of Q/K fused with the cache write, for the 8192 new
 tokens of the mixed chunked-prefill step (Llama-3-8B geometry, rope_theta
 500000).
 
+--workload cow_copy times copy-on-write block copies: 2048 (source,
+destination) pairs of 16-token blocks in Llama-3-8B layer pools (8 KV heads,
+head_dim 128, bf16; 8192 blocks per pool).
+
+--workload graph_decode times a small decode step (4 requests, Llama-3-8B
+geometry) captured once in a CUDA graph and replayed, beside the same step
+launched eagerly: launch overhead is what a graph removes.
+
 --impl reference times the CPU oracle (float64 NumPy, the test reference) on
 a bounded sample of the same workload, on this host's cores.
 """
@@ -46,6 +54,8 @@ WORKLOADS = {
     "shared_prefix": ("shared_prefix_decode", 5),
     "mixed_prefill": ("mixed_step_prefill_only", 4),
     "rope_write": ("mixed_step", 4),   # the mixed step's 8192 new tokens, fused RoPE + cache write
+    "cow_copy": ("llama8b_decode", 2),  # copy-on-write block copies in Llama-3-8B layer pools
+    "graph_decode": ("llama8b_decode", 2),  # a small decode step replayed from a CUDA graph
 }
 FLUSH_BYTES = 512 << 20
 
@@ -750,6 +760,252 @@ def run_reference(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- copy-on-write block copies
+
+COW_BLOCKS, COW_PAIRS = 8192, 2048
+
+
+def cow_inputs(dev, seed):
+    g = torch.Generator(device=dev).manual_seed(seed)
+    mk = lambda: torch.randn(COW_BLOCKS, 16, 8, 128, generator=g, device=dev).to(torch.bfloat16)
+    ids = np.random.default_rng([seed, 81]).permutation(COW_BLOCKS)
+    m = np.stack([ids[:COW_PAIRS], ids[COW_PAIRS:2 * COW_PAIRS]], axis=1).astype(np.int64)
+    return mk(), mk(), torch.from_numpy(m).to(dev)
+
+
+def cow_bytes():
+    return COW_PAIRS * 2 * 2 * (16 * 8 * 128 * 2)   # pairs x pools x (read + write) x block
+
+
+def cow_oracle_sample(kc, vc, seconds):
+    """The oracle's block copy (NumPy, one thread) on 512 pairs per call in
+    1024-block pools cut from the same data, for `seconds`."""
+    import oracle
+    kh = kc[:1024].cpu().view(torch.int16).numpy()
+    vh = vc[:1024].cpu().view(torch.int16).numpy()
+    pairs = np.stack([np.arange(0, 512), np.arange(512, 1024)], axis=1)
+    done, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        oracle.copy_blocks(kh, vh, pairs)
+        done += len(pairs)
+    el = time.perf_counter() - t0
+    return {"value": round(done * cow_bytes() / COW_PAIRS / el / 1e9, 4), "unit": "GB/s",
+            "cores": 1, "kind": "oracle",
+            "sample": f"{done} block pairs (512 per call) in 1024-block pools, NumPy, one thread"}
+
+
+def run_cow(args, rank, world, local):
+    import paged_kv_cache_434_b200 as P
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    kc, vc, m = cow_inputs(dev, args.seed + rank)
+    err = P.new_error_word(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    step = lambda: P.copy_blocks(kc, vc, m, err=err)
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    if P.read_error(err) != 0:
+        raise RuntimeError("device error bits set during warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clocks = ClockSampler(dev) if rank == 0 else None
+    barrier(world)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    wall0 = time.perf_counter()
+    for a, b in evs:
+        flush.fill_(1)
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop() if clocks else None
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_s = max_over_ranks(sum(step_ms) / 1e3, world, dev)
+    nbytes = cow_bytes()
+    value = nbytes * args.steps * world / total_s / 1e9
+    peaks = load_peaks()
+    k_s = statistics.mean(step_ms) / 1e3
+    achieved = nbytes / k_s / 1e9
+    e2e = None
+    if not args.no_e2e:
+        # end to end: the pair list comes from the host each step (the pools
+        # stay on the device: a copy-on-write never moves them)
+        m_h = m.cpu().pin_memory()
+        chk = torch.empty(COW_PAIRS, 16, 8, 128, dtype=torch.bfloat16).pin_memory()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in ev2:
+            flush.fill_(1)
+            a.record(stream)
+            m.copy_(m_h, non_blocking=True)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / 1e3, world, dev)
+        e2e = {"value": round(nbytes * args.steps * world / e2e_s / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": m_h.numel() * 8, "d2h_bytes_per_step": 0,
+               "ms_per_step": round(e2e_s * 1e3 / args.steps, 4),
+               "note": "the step's result stays in the device pools; nothing is read back"}
+        del chk
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cow_oracle_sample(kc, vc, min(args.cpu_seconds, 5.0))
+    if rank == 0:
+        print(json.dumps({
+            "metric": "copy-on-write block copy GB/s", "value": round(value, 2), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": round(total_s * 1e3 / args.steps, 4),
+            "ms_per_step_p10_p50_p90": [round(float(v), 4) for v in
+                                        np.percentile(step_ms, [10, 50, 90])],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) pools, random disjoint source/destination blocks",
+            "config": {"workload": "cow_copy_llama3_8b_2048_pairs", "pairs": COW_PAIRS,
+                       "num_blocks": COW_BLOCKS, "block_size": 16, "num_kv_heads": 8,
+                       "head_dim": 128, "step_bytes": nbytes,
+                       "l2": "flushed before every step (512 MiB write, outside the events)",
+                       "parallelism": f"replicas x{world} (independent pools per GPU)"},
+            "roofline": {"bound": "hbm", "kernel": "copy_blocks_kernel", "achieved": round(achieved, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4),
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)",
+                         "timed_over": f"the copy launch (the step's only launch): CUDA events on "
+                                       f"its stream, mean of {args.steps} launches",
+                         "ms": round(k_s * 1e3, 4),
+                         "traffic": kernel_traffic("blocks.cu", "copy_blocks_kernel_cow_copy.md"),
+                         "algorithmic_bytes_per_launch": nbytes},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clk,
+            "wall_s_timed_region": round(wall, 3)}), flush=True)
+
+
+# ---------------------------------------------------------------- CUDA graph decode step
+
+GRAPH_LENS = [512, 1024, 1536, 2048]
+
+
+def run_graph(args, rank, world, local):
+    import paged_kv_cache_434_b200 as P
+    from paged_kv_cache_434_b200 import workloads as W
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = W.custom("graph_decode_llama3_8b_b4", GRAPH_LENS, [1] * len(GRAPH_LENS), 32, 8, 128, 16,
+                 "bf16", seed=args.seed + rank)
+    t = W.make_tensors(w, dev)
+    idx = W.index_tensors(w, dev)
+    T = w.num_tokens
+    ws = torch.empty(P.decode_workspace_size(w.num_seqs, w.num_heads, w.max_blocks_per_seq,
+                                             t["k_cache"]), dtype=torch.uint8, device=dev)
+    slots = torch.empty(T, dtype=torch.int64, device=dev)
+    out = torch.empty(T, w.num_heads, w.head_dim, dtype=torch.float32, device=dev)
+    err = P.new_error_word(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        P.step(t["q"], t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], idx["block_tables"],
+               idx["query_start_loc"], idx["seq_lens"], w.scale, decode_only=True, out=out,
+               slots=slots, workspace=ws, err=err)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cs):
+        step()
+    for _ in range(max(args.warmup, 3)):
+        g.replay()
+    torch.cuda.synchronize()
+    if P.read_error(err) != 0:
+        raise RuntimeError("device error bits set during warm-up")
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, flush_l2):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in evs:
+            if flush_l2:
+                flush.fill_(1)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    clocks = ClockSampler(dev) if rank == 0 else None
+    barrier(world)
+    if clocks:
+        clocks.start()
+    wall0 = time.perf_counter()
+    g_ms = timed(g.replay, True)
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop() if clocks else None
+    e_ms = timed(step, True)
+    g_hot = timed(g.replay, False)      # back to back, L2 warm: the launch-bound regime
+    e_hot = timed(step, False)
+    total_s = max_over_ranks(sum(g_ms) / 1e3, world, dev)
+    bc = byte_counts(w)
+    us = total_s * 1e6 / args.steps
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "k_new", "v_new"]
+        host = {n: t[n].cpu().pin_memory() for n in names}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in host.values())
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in ev2:
+            flush.fill_(1)
+            a.record(stream)
+            for n in names:
+                t[n].copy_(host[n], non_blocking=True)
+            g.replay()
+            out_h.copy_(out, non_blocking=True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / 1e3, world, dev)
+        e2e = {"value": round(e2e_s * 1e6 / args.steps, 2), "unit": "us/step",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_h.numel() * 4}
+    peaks = load_peaks()
+    achieved = bc["step"] / (statistics.mean(g_ms) / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "decode step us (CUDA graph replay)", "value": round(us, 2),
+            "unit": "us/step", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": round(us / 1e3, 5),
+            "ms_per_step_p10_p50_p90": [round(float(v), 5) for v in np.percentile(g_ms, [10, 50, 90])],
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) Q/K/V rounded to bf16, permuted physical blocks",
+            "config": {"workload": w.name, "num_seqs": w.num_seqs, "seq_lens": GRAPH_LENS,
+                       "num_heads": 32, "num_kv_heads": 8, "head_dim": 128, "block_size": 16,
+                       "step_bytes": bc["step"],
+                       "l2": "flushed before every step (512 MiB write, outside the events)",
+                       "parallelism": f"replicas x{world}"},
+            "eager_us_per_step": round(statistics.mean(e_ms) * 1e3, 2),
+            "l2_warm_back_to_back_us": {"graph": round(statistics.mean(g_hot) * 1e3, 2),
+                                        "eager": round(statistics.mean(e_hot) * 1e3, 2)},
+            "roofline": {"bound": "hbm", "kernel": "the whole step (graph replay)",
+                         "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4),
+                         "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs, copy)",
+                         "timed_over": "one replay per step, CUDA events on the stream",
+                         "traffic": None, "algorithmic_bytes_per_launch": bc["step"],
+                         "note": f"{bc['step'] / 1e6:.0f} MB per step: launch- and "
+                                 f"latency-bound, not an HBM roofline"},
+            "cpu_baseline": None, "e2e": e2e, "gpu_launches": 6 * args.steps, "clocks": clk,
+            "wall_s_timed_region": round(wall, 3)}), flush=True)
+    del g
+
+
 def run_rope_reference(args, rank, world, local):
     """The oracle's fused RoPE + cache write timed as the reference arm."""
     if rank != 0:
@@ -792,7 +1048,38 @@ def main():
     args = parse_args()
     rank, world, local = dist_setup()
     try:
-        if args.workload == "rope_write":
+        if args.workload == "graph_decode":
+            if args.impl == "reference":
+                if rank == 0:
+                    print(json.dumps({"impl": "reference", "unavailable":
+                                      "a CUDA graph step has no CPU counterpart; the oracle is "
+                                      "timed on the decode workloads"}), flush=True)
+            else:
+                run_graph(args, rank, world, local)
+        elif args.workload == "cow_copy":
+            if args.impl == "reference":
+                if rank == 0:
+                    dev = torch.device("cuda", local) if torch.cuda.is_available() else "cpu"
+                    kc, vc, _ = cow_inputs(dev, args.seed)
+                    per = max(0.5, min(args.cpu_seconds, 60.0 / max(1, args.steps)))
+                    vals = [cow_oracle_sample(kc, vc, per)["value"] for _ in range(args.steps)]
+                    v = statistics.mean(vals)
+                    print(json.dumps({
+                        "impl": "reference", "metric": "copy-on-write block copy GB/s",
+                        "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+                        "steps": args.steps, "warmup": 0,
+                        "ms_per_step": round(cow_bytes() / (v * 1e9) * 1e3, 3),
+                        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                        "dtype": "bf16 bits", "data": "synthetic (same generator and seed)",
+                        "config": {"workload": "cow_copy_llama3_8b_2048_pairs"},
+                        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1,
+                                         "kind": "oracle", "sample": f"each step {per:.1f} s"},
+                        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                "d2h_bytes_per_step": 0},
+                        "gpu_launches": 0}), flush=True)
+            else:
+                run_cow(args, rank, world, local)
+        elif args.workload == "rope_write":
             if args.impl == "reference":
                 run_rope_reference(args, rank, world, local)
             else:

@@ -114,6 +114,41 @@ pa_status pa_cache_write(const void* k, const void* v, void* key_cache, void* va
                          const pa_cache_desc* cache, int32_t* err_word, void* stream);
 
 /*
+ * pa_copy_blocks -- copy-on-write block copies ("第三部分 · 推理系统与基础设施",
+ * chapter map 3.3: requests that share physical blocks keep sharing them until
+ * one writes; the writer first gets its own copy of the block).
+ * For each pair i < num_pairs with (src, dst) = block_mapping[2i], [2i+1]:
+ *     key_cache[dst] = key_cache[src] and value_cache[dst] = value_cache[src]
+ * (whole blocks: block_size x num_kv_heads x head_dim elements, bit-exact).
+ *   block_mapping int64 [num_pairs, 2], device memory
+ * A pair naming a block outside [0, num_blocks) is skipped and sets
+ * PA_ERRBIT_BLOCK_OOB.  A block that is the destination of one pair and the
+ * source or destination of another pair of the same call: undefined.
+ */
+pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_mapping,
+                         int64_t num_pairs, const pa_cache_desc* cache, int32_t* err_word,
+                         void* stream);
+
+/*
+ * pa_slot_mapping_positions -- slot of each token from an explicit request
+ * index and position ("AI Infra入门干货总结：大模型是如何高效推理的", "Paged
+ * Attention": slot = block_tables[b][p / block_size] * block_size +
+ * p % block_size), for callers whose tokens are not the last q_b positions
+ * of each request (pa_slot_mapping covers that case).
+ *   token_req   int32 [num_tokens]: request index b, < 0 = padding (slot -1)
+ *   positions   int64 [num_tokens]
+ *   slot_mapping int64 [num_tokens] (output)
+ * b >= num_seqs or p outside [0, max_blocks_per_seq * block_size): slot -1,
+ * PA_ERRBIT_POS_OOB; a table entry outside [0, num_blocks): slot -1,
+ * PA_ERRBIT_BLOCK_OOB.
+ */
+pa_status pa_slot_mapping_positions(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                    int32_t num_seqs, const int32_t* token_req,
+                                    const int64_t* positions, int64_t num_tokens,
+                                    int32_t block_size, int64_t num_blocks,
+                                    int64_t* slot_mapping, int32_t* err_word, void* stream);
+
+/*
  * pa_rope_cos_sin_cache -- the rotary table, built once at start-up
  * ("AI Infra入门干货总结：大模型是如何高效推理的", section "Reshape & Cache":
  * cos_sin_cache of shape [max_position_embeddings, rotary_dim], indexed by

@@ -7,6 +7,8 @@ its Python binding plus a seeded workload generator:
   cache_write    reshape_and_cache into [num_blocks, block_size, Hkv, D] pools
   rope_cache_write  rotary embedding of Q/K fused with the cache write
   rope_cos_sin_cache  the [max_position, rotary_dim] cos/sin table
+  copy_blocks    copy-on-write block copies in both pools
+  slot_mapping_positions  slots from explicit (request, position) pairs
   decode         GQA decode attention, online softmax, split-KV + LSE merge
   mixed_step     causal varlen attention of a chunked-prefill + decode step
   step           slot_mapping -> cache_write -> attention, the per-layer path
@@ -21,6 +23,7 @@ from .binding import (  # noqa: F401
     ERRBIT_TIMEOUT,
     PagedAttentionError,
     cache_write,
+    copy_blocks,
     decode,
     decode_workspace_size,
     kernel_times,
@@ -33,6 +36,7 @@ from .binding import (  # noqa: F401
     rope_cache_write,
     rope_cos_sin_cache,
     slot_mapping,
+    slot_mapping_positions,
     version,
 )
 from .step import step  # noqa: F401

@@ -29,7 +29,8 @@ ERRBIT_POS_OOB = 0x20
 EXPORTS = ("pa_status_str", "pa_version", "pa_slot_mapping", "pa_cache_write",
            "pa_decode_workspace_size", "pa_decode", "pa_mixed_step_workspace_size",
            "pa_mixed_step", "pa_read_error", "pa_decode_no_alloc", "pa_kernel_timing_enable",
-           "pa_kernel_timing_read", "pa_rope_cos_sin_cache", "pa_rope_cache_write")
+           "pa_kernel_timing_read", "pa_rope_cos_sin_cache", "pa_rope_cache_write",
+           "pa_copy_blocks", "pa_slot_mapping_positions")
 
 
 class PagedAttentionError(RuntimeError):
@@ -67,6 +68,9 @@ _SIGNATURES = {
     "pa_kernel_timing_enable": ([_i32], ctypes.c_int),
     "pa_kernel_timing_read": ([ctypes.POINTER(ctypes.c_float)], ctypes.c_int),
     "pa_rope_cos_sin_cache": ([_vp, _i32, _i32, ctypes.c_double, _vp], ctypes.c_int),
+    "pa_copy_blocks": ([_vp, _vp, _vp, _i64, _desc_p, _vp, _vp], ctypes.c_int),
+    "pa_slot_mapping_positions": ([_vp, _i32, _i32, _vp, _vp, _i64, _i32, _i64, _vp, _vp, _vp],
+                                  ctypes.c_int),
     "pa_rope_cache_write": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                              _i32, _i64, _i32, _desc_p, _vp, _vp], ctypes.c_int),
 }
@@ -203,6 +207,37 @@ def cache_write(k, v, k_cache, v_cache, slot_mapping, err=None):
         _cuda(k, "k"), _cuda(v, "v"), _cuda(k_cache, "k_cache", ndim=4),
         _cuda(v_cache, "v_cache", ndim=4), _cuda(slot_mapping, "slot_mapping", torch.int64, 1),
         T, ctypes.byref(desc), _err_ptr(err), _stream()), "pa_cache_write")
+
+
+def copy_blocks(k_cache, v_cache, block_mapping, err=None):
+    """Copy-on-write block copies: block dst := block src in both pools for
+    every (src, dst) row of the int64 [num_pairs, 2] block_mapping."""
+    desc = cache_desc(k_cache)
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
+        raise ValueError("v_cache must match k_cache")
+    if block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
+        raise ValueError("block_mapping must be [num_pairs, 2]")
+    _check(_lib().pa_copy_blocks(
+        _cuda(k_cache, "k_cache", ndim=4), _cuda(v_cache, "v_cache", ndim=4),
+        _cuda(block_mapping, "block_mapping", torch.int64, 2), block_mapping.shape[0],
+        ctypes.byref(desc), _err_ptr(err), _stream()), "pa_copy_blocks")
+
+
+def slot_mapping_positions(block_tables, token_req, positions, block_size: int, num_blocks: int,
+                           out=None, err=None):
+    """int64 slot of every token from its request index and position."""
+    B, W = block_tables.shape
+    T = positions.shape[0]
+    if token_req.shape[0] != T:
+        raise ValueError("token_req and positions must have one entry per token")
+    if out is None:
+        out = torch.empty(T, dtype=torch.int64, device=positions.device)
+    _check(_lib().pa_slot_mapping_positions(
+        _cuda(block_tables, "block_tables", torch.int32, 2), W, B,
+        _cuda(token_req, "token_req", torch.int32, 1), _cuda(positions, "positions", torch.int64, 1),
+        T, block_size, num_blocks, _cuda(out, "out", torch.int64, 1), _err_ptr(err), _stream()),
+        "pa_slot_mapping_positions")
+    return out
 
 
 def rope_cos_sin_cache(max_position: int, rotary_dim: int, theta: float, device=None,

@@ -161,6 +161,14 @@ struct RopeLaunch {
 cudaError_t launch_rope_table(float* cache, int32_t max_position, int32_t rotary_dim, double theta,
                               int num_sms, cudaStream_t s);
 cudaError_t launch_rope_cache_write(const RopeLaunch& l, int num_sms, cudaStream_t s);
+cudaError_t launch_copy_blocks(void* kc, void* vc, const int64_t* mapping, int64_t num_pairs,
+                               int64_t block_bytes, int64_t num_blocks, int32_t* err, int num_sms,
+                               cudaStream_t s);
+cudaError_t launch_slot_positions(const int32_t* block_tables, int32_t max_blocks,
+                                  int32_t num_seqs, const int32_t* token_req,
+                                  const int64_t* positions, int64_t num_tokens,
+                                  int32_t block_size, int64_t num_blocks, int64_t* slots,
+                                  int32_t* err, int num_sms, cudaStream_t s);
 cudaError_t launch_slot_mapping(const int32_t* block_tables, int32_t max_blocks,
                                 const int32_t* qsl, const int32_t* seq_lens, int32_t num_seqs,
                                 int64_t num_tokens, int32_t block_size, int64_t num_blocks,

@@ -332,6 +332,42 @@ pa_status pa_mixed_step(const void* q, const void* key_cache, const void* value_
   return run_attention(g, p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
+pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_mapping,
+                         int64_t num_pairs, const pa_cache_desc* cache, int32_t* err_word,
+                         void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_pairs < 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!key_cache || !value_cache || !block_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned16(key_cache) || !aligned16(value_cache)) return PA_ERR_INVALID_ARG;
+  const int64_t block_bytes = static_cast<int64_t>(cache->block_size) * cache->num_kv_heads *
+                              cache->head_dim * elt_bytes(cache->dtype);
+  return launch_copy_blocks(key_cache, value_cache, block_mapping, num_pairs, block_bytes,
+                            cache->num_blocks, err_word, device_num_sms(),
+                            static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PA_OK
+             : PA_ERR_CUDA;
+}
+
+pa_status pa_slot_mapping_positions(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                    int32_t num_seqs, const int32_t* token_req,
+                                    const int64_t* positions, int64_t num_tokens,
+                                    int32_t block_size, int64_t num_blocks,
+                                    int64_t* slot_mapping, int32_t* err_word, void* stream) {
+  if (num_seqs < 0 || num_tokens < 0 || max_blocks_per_seq < 0 || block_size < 1 ||
+      num_blocks < 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!token_req || !positions || !slot_mapping || (num_seqs > 0 && !block_tables))
+    return PA_ERR_INVALID_ARG;
+  return launch_slot_positions(block_tables, max_blocks_per_seq, num_seqs, token_req, positions,
+                               num_tokens, block_size, num_blocks, slot_mapping, err_word,
+                               device_num_sms(), static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PA_OK
+             : PA_ERR_CUDA;
+}
+
 pa_status pa_rope_cos_sin_cache(float* cache, int32_t max_position, int32_t rotary_dim,
                                 double theta, void* stream) {
   if (!cache || max_position <= 0 || rotary_dim <= 0 || (rotary_dim & 1) || !(theta > 0.0))
