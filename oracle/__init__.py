@@ -27,7 +27,10 @@ Sources (page title, section):
     Q/K dimensions rotated in the complex plane by m*theta (rotary position
     embedding, oracle/rope.py).
   * "第三部分 · 推理系统与基础设施" (llm-learning-path part 3), chapter map,
-    3.3: block tables with copy-on-write (oracle/blocks.py).
+    3.3: block tables with copy-on-write (oracle/blocks.py); 3.2 / 3.6: KV
+    quantisation, FP8 formats (oracle/fp8.py).
+  * "从零构建LLM 推理引擎" (llminference.xinbetween.com), card "量化": fewer
+    bits per KV entry, fewer bytes per decoded token (oracle/fp8.py).
   * "AI Infra入门干货总结", sections "Reshape & Cache" (Q/K rotated by the
     position's rotation, cos_sin_cache [max_position, rotary_dim], then the
     scatter into the pools) and "附1：模型配置参数" (rope_theta 500000).
@@ -61,6 +64,13 @@ from .blocks import (  # noqa: F401
     ERR_POS_OOB_TABLE,
     copy_blocks,
     slot_mapping_positions,
+)
+from .fp8 import (  # noqa: F401
+    E4M3_MAX,
+    dequantize,
+    e4m3_decode,
+    e4m3_encode,
+    quantize,
 )
 from .rope import (  # noqa: F401
     ERR_POS_OOB,
