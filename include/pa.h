@@ -54,7 +54,13 @@ typedef enum pa_status {
   PA_ERR_DEVICE = 5        /* pa_read_error found device error bits set          */
 } pa_status;
 
-typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+/* PA_FP8_E4M3: the pools hold e4m3 codes (1 sign, 4 exponent bits with bias
+ * 7, 3 mantissa bits; no infinities; 448 the largest magnitude) with one
+ * float scale per pool (pa_cache_desc.k_scale / v_scale): an entry stands for
+ * code * scale.  Queries, new K/V rows and rotated queries are bf16 then.
+ * ("从零构建LLM 推理引擎", card "量化": halving the bits of every KV entry
+ * nearly halves the bytes, and so the time, of each decoded token.) */
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 
 /* Device error bits (OR-ed into *err_word). */
 #define PA_ERRBIT_SLOT_OOB 0x1        /* slot >= num_blocks * block_size           */
@@ -70,7 +76,11 @@ typedef struct pa_cache_desc {
   int32_t block_size;    /* tokens per block: 8, 16, 32, 64, 128 or 256  */
   int32_t num_kv_heads;  /* >= 1                                        */
   int32_t head_dim;      /* 64 or 128                                   */
-  int32_t dtype;         /* pa_dtype of pools, q, k and v               */
+  int32_t dtype;         /* pa_dtype of pools, q, k and v (FP8: pools
+                            e4m3, q / k / v bf16)                       */
+  float k_scale;         /* PA_FP8_E4M3: key entry = code * k_scale;
+                            positive and finite; ignored otherwise      */
+  float v_scale;         /* PA_FP8_E4M3: value entry = code * v_scale   */
 } pa_cache_desc;
 
 /* Static description of a status code; never NULL. */
@@ -108,6 +118,9 @@ pa_status pa_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_se
  *   slot_mapping int64 [num_tokens]; a negative slot marks padding (skipped)
  * Bit-exact copy.  s >= num_blocks * block_size is skipped and sets
  * PA_ERRBIT_SLOT_OOB.  Two tokens with the same slot in one call: undefined.
+ * PA_FP8_E4M3 pools: k and v are bf16 and each entry is stored as the e4m3
+ * code of the float32 quotient x / scale, rounded to nearest (ties to even)
+ * and saturated to +-448.
  */
 pa_status pa_cache_write(const void* k, const void* v, void* key_cache, void* value_cache,
                          const int64_t* slot_mapping, int64_t num_tokens,

@@ -17,7 +17,7 @@ import torch
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libpa_b200.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_DEVICE = range(6)
-PA_F32, PA_BF16 = 0, 1
+PA_F32, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
 
 ERRBIT_SLOT_OOB = 0x1
 ERRBIT_BLOCK_OOB = 0x2
@@ -43,7 +43,8 @@ class PagedAttentionError(RuntimeError):
 class CacheDesc(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int64), ("block_size", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("k_scale", ctypes.c_float),
+                ("v_scale", ctypes.c_float)]
 
 
 _LIB = None
@@ -113,7 +114,9 @@ def _dt(t: torch.Tensor) -> int:
         return PA_F32
     if t.dtype == torch.bfloat16:
         return PA_BF16
-    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+    if t.dtype == torch.float8_e4m3fn:
+        return PA_FP8_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32, bfloat16 or float8_e4m3fn pools")
 
 
 def _cuda(t: torch.Tensor, name: str, dtype=None, ndim=None) -> int:
@@ -140,9 +143,26 @@ def _err_ptr(err):
     return _cuda(err, "err", torch.int32)
 
 
-def cache_desc(k_cache: torch.Tensor) -> CacheDesc:
+def cache_desc(k_cache: torch.Tensor, kv_scales=None) -> CacheDesc:
+    """Descriptor of a layer's pools.  float8_e4m3fn pools need kv_scales =
+    (k_scale, v_scale): an entry stands for code * scale."""
     nb, bs, hkv, d = k_cache.shape
-    return CacheDesc(nb, bs, hkv, d, _dt(k_cache))
+    dt = _dt(k_cache)
+    ks = vs = 1.0
+    if dt == PA_FP8_E4M3:
+        if kv_scales is None:
+            raise ValueError("float8_e4m3fn pools need kv_scales=(k_scale, v_scale)")
+        ks, vs = (float(x) for x in kv_scales)
+    return CacheDesc(nb, bs, hkv, d, dt, ks, vs)
+
+
+def io_dtype(k_cache: torch.Tensor):
+    """dtype of the queries and new K/V rows that go with these pools."""
+    return torch.bfloat16 if k_cache.dtype == torch.float8_e4m3fn else k_cache.dtype
+
+
+def _any_scales(k_cache):
+    return (1.0, 1.0) if k_cache.dtype == torch.float8_e4m3fn else None
 
 
 def _check(status: int, where: str):
@@ -191,14 +211,16 @@ def slot_mapping(block_tables, query_start_loc, seq_lens, block_size: int, num_b
     return out
 
 
-def cache_write(k, v, k_cache, v_cache, slot_mapping, err=None):
-    """reshape_and_cache: k_cache[slot // bs, slot % bs] = k[t] (and v)."""
-    desc = cache_desc(k_cache)
+def cache_write(k, v, k_cache, v_cache, slot_mapping, err=None, kv_scales=None):
+    """reshape_and_cache: k_cache[slot // bs, slot % bs] = k[t] (and v); FP8
+    pools store the e4m3 code of k / k_scale (and v / v_scale)."""
+    desc = cache_desc(k_cache, kv_scales)
     T = k.shape[0]
     for name, t in (("k", k), ("v", v)):
         if t.dim() != 3 or tuple(t.shape[1:]) != (desc.num_kv_heads, desc.head_dim) or \
-                t.shape[0] != T or t.dtype != k_cache.dtype:
-            raise ValueError(f"{name} must be [num_tokens, num_kv_heads, head_dim] of the cache dtype")
+                t.shape[0] != T or t.dtype != io_dtype(k_cache):
+            raise ValueError(f"{name} must be [num_tokens, num_kv_heads, head_dim] of the cache's "
+                             f"input dtype")
     if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
         raise ValueError("v_cache must match k_cache")
     if slot_mapping.shape[0] != T:
@@ -212,7 +234,7 @@ def cache_write(k, v, k_cache, v_cache, slot_mapping, err=None):
 def copy_blocks(k_cache, v_cache, block_mapping, err=None):
     """Copy-on-write block copies: block dst := block src in both pools for
     every (src, dst) row of the int64 [num_pairs, 2] block_mapping."""
-    desc = cache_desc(k_cache)
+    desc = cache_desc(k_cache, _any_scales(k_cache))
     if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
         raise ValueError("v_cache must match k_cache")
     if block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
@@ -268,7 +290,7 @@ def rope_cache_write(q, k, v, k_cache, v_cache, slot_mapping, positions, cos_sin
                      neox: bool = True, q_out=None, err=None):
     """Rotate q and k by their positions, store rotated k and plain v at their
     slots, return the rotated queries (see pa_rope_cache_write)."""
-    desc = cache_desc(k_cache)
+    desc = cache_desc(k_cache, _any_scales(k_cache))
     T, Hq, D = q.shape
     if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
         raise ValueError("v_cache must match k_cache")
@@ -295,13 +317,13 @@ def rope_cache_write(q, k, v, k_cache, v_cache, slot_mapping, positions, cos_sin
 
 
 def decode_workspace_size(num_seqs, num_heads, max_blocks_per_seq, k_cache) -> int:
-    desc = cache_desc(k_cache)
+    desc = cache_desc(k_cache, _any_scales(k_cache))
     return int(_lib().pa_decode_workspace_size(num_seqs, num_heads, max_blocks_per_seq,
                                                ctypes.byref(desc)))
 
 
 def mixed_step_workspace_size(num_seqs, num_tokens, num_heads, max_blocks_per_seq, k_cache) -> int:
-    desc = cache_desc(k_cache)
+    desc = cache_desc(k_cache, _any_scales(k_cache))
     return int(_lib().pa_mixed_step_workspace_size(num_seqs, num_tokens, num_heads,
                                                    max_blocks_per_seq, ctypes.byref(desc)))
 
@@ -314,10 +336,10 @@ def _workspace(nbytes, device, workspace):
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
-def _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype):
-    desc = cache_desc(k_cache)
-    if q.dtype != k_cache.dtype or q.dim() != 3 or q.shape[2] != desc.head_dim:
-        raise ValueError("q must be [rows, num_heads, head_dim] of the cache dtype")
+def _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales=None):
+    desc = cache_desc(k_cache, kv_scales)
+    if q.dtype != io_dtype(k_cache) or q.dim() != 3 or q.shape[2] != desc.head_dim:
+        raise ValueError("q must be [rows, num_heads, head_dim] of the cache's input dtype")
     if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
         raise ValueError("v_cache must match k_cache")
     if out_dtype not in (torch.float32, torch.bfloat16):
@@ -326,9 +348,9 @@ def _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype):
 
 
 def decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=None,
-           out_dtype=torch.float32, workspace=None, err=None):
+           out_dtype=torch.float32, workspace=None, err=None, kv_scales=None):
     """Decode attention: out[b, h] over the first seq_lens[b] keys of request b."""
-    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype)
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales)
     B, H, D = q.shape
     W = block_tables.shape[1]
     if out is None:
@@ -345,9 +367,9 @@ def decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=None,
 
 
 def mixed_step(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, scale: float,
-               out=None, out_dtype=torch.float32, workspace=None, err=None):
+               out=None, out_dtype=torch.float32, workspace=None, err=None, kv_scales=None):
     """Causal varlen attention of a flattened step (chunked prefill + decode)."""
-    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype)
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales)
     T, H, D = q.shape
     B, W = block_tables.shape
     if out is None:
@@ -365,7 +387,7 @@ def mixed_step(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, sca
 
 
 def decode_no_alloc(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out,
-                    err=None):
+                    err=None, kv_scales=None):
     """pa_decode_no_alloc: decode attention for callers that can't allocate
     device memory (e.g. a plug-in inside an engine that owns all allocations).
 
@@ -375,7 +397,7 @@ def decode_no_alloc(q, k_cache, v_cache, block_tables, seq_lens, scale: float, o
     `out` must be given, so that this call allocates nothing either.  Calls
     whose kernels overlap on the GPU share the scratch and race.
     """
-    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out.dtype)
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out.dtype, kv_scales)
     B, H, D = q.shape
     W = block_tables.shape[1]
     _check(_lib().pa_decode_no_alloc(

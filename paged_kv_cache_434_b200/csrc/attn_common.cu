@@ -19,6 +19,7 @@
 #include <cuda_bf16.h>
 
 #include <cmath>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -505,6 +506,31 @@ __device__ __forceinline__ void load_row(const T* p, float (&x)[V]) {
 #pragma unroll
   for (int e = 0; e < V; ++e) x[e] = to_f32(p[e]);
 }
+// FP8 pool entries: e4m3 codes, decoded exactly (the scales are applied to the
+// scores and to the output instead)
+struct e4m3_t {
+  uint8_t code;
+};
+template <int V>
+__device__ __forceinline__ void load_row_e4m3(const e4m3_t* p, float (&x)[V]) {
+  static_assert(V % 2 == 0, "pairs of codes");
+  const uint8_t* b = reinterpret_cast<const uint8_t*>(p);
+#pragma unroll
+  for (int e = 0; e < V; e += 2) {
+    const uint16_t c = static_cast<uint16_t>(b[e]) | (static_cast<uint16_t>(b[e + 1]) << 8);
+    const float2 f = f16x2_to_f32x2(e4m3x2_to_f16x2(c));
+    x[e] = f.x;
+    x[e + 1] = f.y;
+  }
+}
+template <typename T>
+struct QueryType {
+  using type = T;
+};
+template <>
+struct QueryType<e4m3_t> {
+  using type = __nv_bfloat16;  // queries of an FP8 cache are bf16
+};
 
 __device__ __forceinline__ void store_out(void* out, int out_dtype, int64_t idx, float v) {
   if (out_dtype == PA_F32)
@@ -529,7 +555,8 @@ __global__ void __launch_bounds__(kGenWarps * 32) attn_generic_kernel(AttnGeom g
   const int G = g.num_heads / g.num_kv_heads;
   const int n_items = ws.ctrl[1];
   const int P = ws.ctrl[2];
-  const T* q = static_cast<const T*>(g.q);
+  using QT = typename QueryType<T>::type;
+  const QT* q = static_cast<const QT*>(g.q);
   const T* kc = static_cast<const T*>(g.k_cache);
   const T* vc = static_cast<const T*>(g.v_cache);
 
@@ -571,8 +598,13 @@ __global__ void __launch_bounds__(kGenWarps * 32) attn_generic_kernel(AttnGeom g
       const int64_t row = static_cast<int64_t>(phys) * g.block_size + j % g.block_size;
       const int64_t off = (row * g.num_kv_heads + hk) * D + lane * V;
       float kx[V], vx[V];
-      load_row<T, V>(kc + off, kx);
-      load_row<T, V>(vc + off, vx);
+      if constexpr (std::is_same<T, e4m3_t>::value) {
+        load_row_e4m3<V>(kc + off, kx);
+        load_row_e4m3<V>(vc + off, vx);
+      } else {
+        load_row<T, V>(kc + off, kx);
+        load_row<T, V>(vc + off, vx);
+      }
 #pragma unroll
       for (int gq = 0; gq < kMaxGroup; ++gq) {
         if (gq < G) {
@@ -629,11 +661,11 @@ __global__ void __launch_bounds__(kGenWarps * 32) attn_generic_kernel(AttnGeom g
       if (np == 1) {
         if (!row_bad)
           store_out(g.out, g.out_dtype, (static_cast<int64_t>(r) * g.num_heads + h) * D + d,
-                    O / Ls);
+                    O * g.v_scale / Ls);
       } else {
         const int64_t slot = (static_cast<int64_t>(r) * g.num_heads + h) * ws.max_parts + p;
         if (d == 0) ws.part_ml[slot] = make_float2(M, Ls);
-        ws.part_o[slot * D + d] = O;
+        ws.part_o[slot * D + d] = O * g.v_scale;
       }
     }
     __syncthreads();
@@ -646,6 +678,11 @@ cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms
   if (g.dtype == PA_F32) {
     if (g.head_dim == 64) return launch_pdl<attn_generic_kernel<float, 64>>(grid, block, 0, s, g, ws);
     return launch_pdl<attn_generic_kernel<float, 128>>(grid, block, 0, s, g, ws);
+  }
+  if (g.dtype == PA_FP8_E4M3) {
+    if (g.head_dim == 64)
+      return launch_pdl<attn_generic_kernel<e4m3_t, 64>>(grid, block, 0, s, g, ws);
+    return launch_pdl<attn_generic_kernel<e4m3_t, 128>>(grid, block, 0, s, g, ws);
   }
   if (g.head_dim == 64)
     return launch_pdl<attn_generic_kernel<__nv_bfloat16, 64>>(grid, block, 0, s, g, ws);

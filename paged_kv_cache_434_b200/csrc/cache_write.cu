@@ -7,6 +7,8 @@
 // [num_kv_heads, head_dim] row of a token is contiguous at element offset
 // slot * num_kv_heads * head_dim, so the scatter is one contiguous row copy per
 // token, done with 16-byte vector loads and stores.
+#include <cuda_bf16.h>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -81,6 +83,61 @@ __global__ void __launch_bounds__(256) cache_write_kernel(
     dst[i + 96] = d;
   }
   for (; i < row_vec; i += 32) dst[i] = __ldg(src + i);
+}
+
+// FP8 pools: one warp per (token, K|V); a lane turns 16 bf16 entries into 16
+// e4m3 codes of the float32 quotients x / scale (IEEE division, the rounding
+// the oracle reproduces) per step.
+__global__ void __launch_bounds__(256) cache_write_fp8_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ kc,
+    uint4* __restrict__ vc, const int64_t* __restrict__ slots, int64_t num_tokens,
+    int64_t row_chunks /* 16-entry chunks per row */, int64_t num_slots, float k_scale,
+    float v_scale, int32_t* __restrict__ err) {
+  grid_launch_dependents();
+  grid_dependency_wait();  // the slots usually come from the previous launch
+  const int lane = threadIdx.x & 31;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t t = w >> 1;
+  if (t >= num_tokens) return;
+  const int64_t slot = slots[t];
+  if (slot < 0) return;  // padding token
+  if (slot >= num_slots) {
+    if (lane == 0 && (w & 1) == 0 && err) atomicOr(err, PA_ERRBIT_SLOT_OOB);
+    return;
+  }
+  const bool is_v = (w & 1) != 0;
+  const float sc = is_v ? v_scale : k_scale;
+  const uint4* src = (is_v ? v : k) + t * row_chunks * 2;  // 2 uint4 of bf16 per chunk
+  uint4* dst = (is_v ? vc : kc) + slot * row_chunks;       // 1 uint4 of codes per chunk
+  for (int64_t c = lane; c < row_chunks; c += 32) {
+    const uint4 a = __ldg(src + 2 * c), b = __ldg(src + 2 * c + 1);
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 p0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[2 * j]));
+      const float2 p1 =
+          __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[2 * j + 1]));
+      const uint16_t lo = f32x2_to_e4m3x2(__fdiv_rn(p0.x, sc), __fdiv_rn(p0.y, sc));
+      const uint16_t hi = f32x2_to_e4m3x2(__fdiv_rn(p1.x, sc), __fdiv_rn(p1.y, sc));
+      out[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+    dst[c] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+cudaError_t launch_cache_write_fp8(const void* k, const void* v, void* kc, void* vc,
+                                   const int64_t* slots, int64_t num_tokens, int64_t row_elems,
+                                   int64_t num_slots, float k_scale, float v_scale, int32_t* err,
+                                   cudaStream_t s) {
+  if (num_tokens == 0) return cudaSuccess;
+  const int warps = 8;
+  const int64_t nwarps = 2 * num_tokens;
+  dim3 grid(static_cast<unsigned>((nwarps + warps - 1) / warps));
+  return launch_pdl<cache_write_fp8_kernel>(
+      grid, dim3(warps * 32), 0, s, static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+      static_cast<uint4*>(kc), static_cast<uint4*>(vc), slots, num_tokens, row_elems / 16,
+      num_slots, k_scale, v_scale, err);
 }
 
 cudaError_t launch_slot_mapping(const int32_t* block_tables, int32_t max_blocks,

@@ -81,7 +81,8 @@ struct AttnGeom {
   int32_t max_blocks;
   int32_t dtype;          // pa_dtype of q / caches
   int32_t out_dtype;
-  float scale_log2;       // scale * log2(e)
+  float scale_log2;       // scale * log2(e) (* k_scale for an FP8 cache)
+  float v_scale;          // FP8 cache: value entry = code * v_scale; 1 otherwise
   int32_t* err_word;
 };
 
@@ -169,6 +170,10 @@ cudaError_t launch_slot_positions(const int32_t* block_tables, int32_t max_block
                                   const int64_t* positions, int64_t num_tokens,
                                   int32_t block_size, int64_t num_blocks, int64_t* slots,
                                   int32_t* err, int num_sms, cudaStream_t s);
+cudaError_t launch_cache_write_fp8(const void* k, const void* v, void* kc, void* vc,
+                                   const int64_t* slots, int64_t num_tokens, int64_t row_elems,
+                                   int64_t num_slots, float k_scale, float v_scale, int32_t* err,
+                                   cudaStream_t s);
 cudaError_t launch_slot_mapping(const int32_t* block_tables, int32_t max_blocks,
                                 const int32_t* qsl, const int32_t* seq_lens, int32_t num_seqs,
                                 int64_t num_tokens, int32_t block_size, int64_t num_blocks,

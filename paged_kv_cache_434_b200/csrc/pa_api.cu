@@ -31,11 +31,18 @@ static pa_status check_cache(const pa_cache_desc* c) {
   if (!(bs == 8 || bs == 16 || bs == 32 || bs == 64 || bs == 128 || bs == 256))
     return PA_ERR_UNSUPPORTED;
   if (c->head_dim != 64 && c->head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (c->dtype != PA_F32 && c->dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (c->dtype != PA_F32 && c->dtype != PA_BF16 && c->dtype != PA_FP8_E4M3)
+    return PA_ERR_UNSUPPORTED;
+  if (c->dtype == PA_FP8_E4M3 &&
+      !(c->k_scale > 0.f && c->k_scale < INFINITY && c->v_scale > 0.f && c->v_scale < INFINITY))
+    return PA_ERR_INVALID_ARG;
   return PA_OK;
 }
 
+// bytes of one element of q / new k, v rows (bf16 for an FP8 cache)
 static int elt_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+// bytes of one pool entry
+static int pool_elt_bytes(int dtype) { return dtype == PA_F32 ? 4 : dtype == PA_BF16 ? 2 : 1; }
 
 // Launch plan of one attention call (decode or mixed step); identical in the
 // workspace-size query and in the call itself.
@@ -119,6 +126,11 @@ static AttnGeom make_geom(const void* q, const void* kc, const void* vc, const i
   g.dtype = c->dtype;
   g.out_dtype = out_dtype;
   g.scale_log2 = scale * 1.4426950408889634f;
+  g.v_scale = 1.f;
+  if (c->dtype == PA_FP8_E4M3) {  // scores see code * k_scale, outputs code * v_scale
+    g.scale_log2 *= c->k_scale;
+    g.v_scale = c->v_scale;
+  }
   g.err_word = err;
   return g;
 }
@@ -230,7 +242,7 @@ const char* pa_status_str(int status) {
   }
 }
 
-int pa_version(void) { return 100; }
+int pa_version(void) { return 101; }
 
 pa_status pa_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_seq,
                           const int32_t* query_start_loc, const int32_t* seq_lens,
@@ -260,11 +272,17 @@ pa_status pa_cache_write(const void* k, const void* v, void* key_cache, void* va
   if (!k || !v || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(key_cache) || !aligned16(value_cache))
     return PA_ERR_INVALID_ARG;
-  const int64_t row_bytes =
-      static_cast<int64_t>(cache->num_kv_heads) * cache->head_dim * elt_bytes(cache->dtype);
-  cudaError_t e = launch_cache_write(k, v, key_cache, value_cache, slot_mapping, num_tokens,
-                                     row_bytes, cache->num_blocks * cache->block_size, err_word,
-                                     static_cast<cudaStream_t>(stream));
+  const int64_t row_elems = static_cast<int64_t>(cache->num_kv_heads) * cache->head_dim;
+  cudaError_t e;
+  if (cache->dtype == PA_FP8_E4M3)
+    e = launch_cache_write_fp8(k, v, key_cache, value_cache, slot_mapping, num_tokens, row_elems,
+                               cache->num_blocks * cache->block_size, cache->k_scale,
+                               cache->v_scale, err_word, static_cast<cudaStream_t>(stream));
+  else
+    e = launch_cache_write(k, v, key_cache, value_cache, slot_mapping, num_tokens,
+                           row_elems * elt_bytes(cache->dtype),
+                           cache->num_blocks * cache->block_size, err_word,
+                           static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -342,7 +360,7 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
   if (!key_cache || !value_cache || !block_mapping) return PA_ERR_INVALID_ARG;
   if (!aligned16(key_cache) || !aligned16(value_cache)) return PA_ERR_INVALID_ARG;
   const int64_t block_bytes = static_cast<int64_t>(cache->block_size) * cache->num_kv_heads *
-                              cache->head_dim * elt_bytes(cache->dtype);
+                              cache->head_dim * pool_elt_bytes(cache->dtype);
   return launch_copy_blocks(key_cache, value_cache, block_mapping, num_pairs, block_bytes,
                             cache->num_blocks, err_word, device_num_sms(),
                             static_cast<cudaStream_t>(stream)) == cudaSuccess
@@ -387,6 +405,7 @@ pa_status pa_rope_cache_write(const void* q_in, const void* k, const void* v, in
                               void* stream) {
   pa_status st = check_cache(cache);
   if (st != PA_OK) return st;
+  if (cache->dtype == PA_FP8_E4M3) return PA_ERR_UNSUPPORTED;
   if (num_tokens < 0 || num_heads < 1 || max_position < 1) return PA_ERR_INVALID_ARG;
   if (rotary_dim < 16 || rotary_dim % 16 || rotary_dim > cache->head_dim)
     return PA_ERR_UNSUPPORTED;

@@ -7,6 +7,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace pa {
 
@@ -174,6 +175,24 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// e4m3 (FP8) conversions.  Two floats to two e4m3 codes (nearest, ties to
+// even, saturating to +-448): `lo` goes to the low byte.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two e4m3 codes (low byte first) to two halves of an f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(codes));
+  return r;
+}
+__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t h) {
+  const __half2 v = *reinterpret_cast<const __half2*>(&h);
+  return __half22float2(v);
 }
 
 // 2^x via the hardware approximation (ex2.approx, flush-to-zero).

@@ -13,11 +13,12 @@ from . import binding
 
 def step(q, k_new, v_new, k_cache, v_cache, block_tables, query_start_loc, seq_lens,
          scale: float, *, decode_only: bool = False, out=None, out_dtype=torch.float32,
-         slots=None, workspace=None, err=None):
+         slots=None, workspace=None, err=None, kv_scales=None):
     """Run slot_mapping -> cache_write -> decode / mixed_step on the current stream.
 
     q: [T, Hq, D]; k_new, v_new: [T, Hkv, D]; query_start_loc: [B+1] int32;
-    seq_lens: [B] int32 (lengths after this step).  With decode_only=True every
+    seq_lens: [B] int32 (lengths after this step).  float8_e4m3fn pools take
+    kv_scales=(k_scale, v_scale) and bf16 q / k_new / v_new.  With decode_only=True every
     request has exactly one new token (T == B) and pa_decode is used.
     Returns out [T, Hq, D].
     """
@@ -25,9 +26,11 @@ def step(q, k_new, v_new, k_cache, v_cache, block_tables, query_start_loc, seq_l
     nb, bs = k_cache.shape[0], k_cache.shape[1]
     slots = binding.slot_mapping(block_tables, query_start_loc, seq_lens, bs, nb, T, out=slots,
                                  err=err)
-    binding.cache_write(k_new, v_new, k_cache, v_cache, slots, err=err)
+    binding.cache_write(k_new, v_new, k_cache, v_cache, slots, err=err, kv_scales=kv_scales)
     if decode_only:
         return binding.decode(q, k_cache, v_cache, block_tables, seq_lens, scale, out=out,
-                              out_dtype=out_dtype, workspace=workspace, err=err)
+                              out_dtype=out_dtype, workspace=workspace, err=err,
+                              kv_scales=kv_scales)
     return binding.mixed_step(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, scale,
-                              out=out, out_dtype=out_dtype, workspace=workspace, err=err)
+                              out=out, out_dtype=out_dtype, workspace=workspace, err=err,
+                              kv_scales=kv_scales)

@@ -48,6 +48,8 @@ class Workload:
     scale: float
     seed: int
     shared_prefix_blocks: int = 0  # leading table entries common to all rows
+    kv_dtype: str = ""             # "fp8": e4m3 pools (q / new K/V stay bf16)
+    kv_scale: float = 1.0          # fp8 pools: an entry stands for code * kv_scale
 
     @property
     def num_seqs(self) -> int:
@@ -68,6 +70,14 @@ class Workload:
     @property
     def elt_bytes(self) -> int:
         return 4 if self.dtype == "f32" else 2
+
+    @property
+    def pool_elt_bytes(self) -> int:
+        return 1 if self.kv_dtype == "fp8" else self.elt_bytes
+
+    @property
+    def kv_scales(self):
+        return (self.kv_scale, self.kv_scale) if self.kv_dtype == "fp8" else None
 
     @property
     def is_decode(self) -> bool:
@@ -244,7 +254,20 @@ def make_tensors(w: Workload, device="cpu", where: str = "auto"):
         else:
             t = torch.empty(shape, dtype=_torch_dtype(w.dtype), device=device)
             out[name] = _device_normal_(t, w.seed, VALUE_TAGS[name])
+        if w.kv_dtype == "fp8" and name in ("k_cache", "v_cache"):
+            # the same draws, stored as e4m3 codes by torch's own conversion
+            # (inputs for both sides; the oracle decodes the codes itself)
+            x = torch.clamp(out[name].float() / w.kv_scale, -448.0, 448.0)
+            out[name] = x.to(torch.float8_e4m3fn)
     return out
+
+
+def with_fp8_cache(w: Workload, scale: float = 1.0 / 56.0) -> Workload:
+    """The same workload over e4m3 pools (N(0,1) entries over 1/56: |x| <= 8
+    stays below the format's 448)."""
+    import dataclasses
+    return dataclasses.replace(w, name=w.name + "_fp8kv", dtype="bf16", kv_dtype="fp8",
+                               kv_scale=scale)
 
 
 def index_tensors(w: Workload, device="cpu"):
@@ -260,7 +283,7 @@ def index_tensors(w: Workload, device="cpu"):
 def kv_bytes_touched(w: Workload, unique: bool = True) -> int:
     """Algorithmic K+V bytes one pass of attention must read: valid tokens only;
     with unique=True a physical block shared by several tables counts once."""
-    row = 2 * w.num_kv_heads * w.head_dim * w.elt_bytes
+    row = 2 * w.num_kv_heads * w.head_dim * w.pool_elt_bytes
     if not unique:
         return int(w.seq_lens.astype(np.int64).sum()) * row
     seen = {}

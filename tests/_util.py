@@ -90,3 +90,25 @@ def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
         assert err.max() <= TOL_BF16_MAX, f"{what}: max-abs {err.max():.3g} > {TOL_BF16_MAX}"
         assert err.mean() <= TOL_BF16_MEAN, f"{what}: mean-abs {err.mean():.3g} > {TOL_BF16_MEAN}"
     return float(err.max()), float(err.mean())
+
+
+def fp8_codes(t: torch.Tensor) -> np.ndarray:
+    """Raw bytes of a float8_e4m3fn tensor."""
+    return t.detach().cpu().contiguous().view(torch.uint8).numpy()
+
+
+def oracle_full_fp8(w, host):
+    """oracle_full for e4m3 pools: the expected pool codes after the cache
+    write (oracle quantisation of the new rows) and the attention over the
+    dequantised pools.  Returns (slots, k_codes, v_codes, out, errors, valid)."""
+    qsl = w.query_start_loc
+    slots = oracle.slot_mapping(w.block_tables, qsl, w.seq_lens, w.block_size)
+    kc0, vc0 = fp8_codes(host["k_cache"]), fp8_codes(host["v_cache"])
+    kq = oracle.quantize(f64(host["k_new"]).astype(np.float32), w.kv_scale)
+    vq = oracle.quantize(f64(host["v_new"]).astype(np.float32), w.kv_scale)
+    kc, vc, err_w = oracle.cache_write(kc0, vc0, kq, vq, slots)
+    k64 = oracle.dequantize(kc, w.kv_scale)
+    v64 = oracle.dequantize(vc, w.kv_scale)
+    out, err_a, valid = oracle.paged_mixed_step(f64(host["q"]), k64, v64, w.block_tables, qsl,
+                                                w.seq_lens, w.scale)
+    return slots, kc, vc, out, err_w | err_a, valid
