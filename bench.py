@@ -53,6 +53,8 @@ WORKLOADS = {
     "mixed": ("mixed_step", 4),
     "shared_prefix": ("shared_prefix_decode", 5),
     "mixed_prefill": ("mixed_step_prefill_only", 4),
+    "llama8b_decode_fp8": ("llama8b_decode_fp8", 2),   # the same batch over e4m3 pools
+    "long_context_fp8": ("long_context_decode_fp8", 3),
     "rope_write": ("mixed_step", 4),   # the mixed step's 8192 new tokens, fused RoPE + cache write
     "cow_copy": ("llama8b_decode", 2),  # copy-on-write block copies in Llama-3-8B layer pools
     "graph_decode": ("llama8b_decode", 2),  # a small decode step replayed from a CUDA graph
@@ -209,7 +211,7 @@ def byte_counts(w, out_elt=4):
     kv = W.kv_bytes_touched(w, unique=True)
     q = w.num_tokens * w.num_heads * w.head_dim * w.elt_bytes
     o = w.num_tokens * w.num_heads * w.head_dim * out_elt
-    cw = 2 * 2 * w.num_tokens * w.num_kv_heads * w.head_dim * w.elt_bytes
+    cw = 2 * w.num_tokens * w.num_kv_heads * w.head_dim * (w.elt_bytes + w.pool_elt_bytes)
     return {"kv": kv, "q": q, "o": o, "cache_write": cw, "attention": kv + q + o,
             "step": kv + q + o + cw}
 
@@ -219,7 +221,7 @@ def decode_kernel_bytes(w, out_elt=4):
     q_b = 1 requests (valid tokens; a block prefix common to every table is
     left to the tensor-core prefix tiles when the batch has one), their Q rows
     read and their output rows written."""
-    row = 2 * w.num_kv_heads * w.head_dim * w.elt_bytes
+    row = 2 * w.num_kv_heads * w.head_dim * w.pool_elt_bytes
     dec = [b for b in range(w.num_seqs) if int(w.query_lens[b]) == 1]
     shared = w.shared_prefix_blocks * w.block_size
     toks = sum(int(w.seq_lens[b]) - min(shared, int(w.seq_lens[b])) for b in dec)
@@ -271,7 +273,7 @@ def oracle_sample(w, pools, seconds: float, rng_seed: int = 0):
         for a, b in zip(pi, dec):
             rows.append(pre[a])
             rows.append((b, 0))
-    row_kv = 2 * w.num_kv_heads * w.head_dim * w.elt_bytes
+    row_kv = 2 * w.num_kv_heads * w.head_dim * w.pool_elt_bytes
     # fetch the blocks for up to a generous number of rows first (not timed)
     prepared = []
     cache = {}
@@ -295,8 +297,13 @@ def oracle_sample(w, pools, seconds: float, rng_seed: int = 0):
             L, qb = int(w.seq_lens[b]), int(w.query_lens[b])
             pos = L - qb + i
             table = np.arange(kb.shape[0])
-            K = oracle.gather(kb.to(torch.float64).numpy(), table, pos + 1)
-            V = oracle.gather(vb.to(torch.float64).numpy(), table, pos + 1)
+            if w.kv_dtype == "fp8":
+                kd = oracle.dequantize(kb.view(torch.uint8).numpy(), w.kv_scale)
+                vd = oracle.dequantize(vb.view(torch.uint8).numpy(), w.kv_scale)
+            else:
+                kd, vd = kb.to(torch.float64).numpy(), vb.to(torch.float64).numpy()
+            K = oracle.gather(kd, table, pos + 1)
+            V = oracle.gather(vd, table, pos + 1)
             oracle.attend_two_pass(q.to(torch.float64).numpy(), K, V, w.scale, pos)
             done_units += (pos + 1) * row_kv if w.is_decode else 1
             if time.perf_counter() - t0 > seconds:
@@ -373,15 +380,16 @@ def run_ours(args, rank, world, local):
     def step():
         P.slot_mapping(idx["block_tables"], idx["query_start_loc"], idx["seq_lens"],
                        w.block_size, w.num_blocks, T, out=slots, err=err)
-        P.cache_write(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], slots, err=err)
+        P.cache_write(t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], slots, err=err,
+                      kv_scales=w.kv_scales)
         mid.record(stream)
         if decode_only:
             P.decode(t["q"], t["k_cache"], t["v_cache"], idx["block_tables"], idx["seq_lens"],
-                     w.scale, out=out, workspace=ws, err=err)
+                     w.scale, out=out, workspace=ws, err=err, kv_scales=w.kv_scales)
         else:
             P.mixed_step(t["q"], t["k_cache"], t["v_cache"], idx["block_tables"],
                          idx["query_start_loc"], idx["seq_lens"], w.scale, out=out,
-                         workspace=ws, err=err)
+                         workspace=ws, err=err, kv_scales=w.kv_scales)
 
     mid = torch.cuda.Event(enable_timing=True)
     for _ in range(max(args.warmup, 3)):
@@ -441,6 +449,10 @@ def run_ours(args, rank, world, local):
     attn_s = statistics.mean(attn_ms) / 1e3
     dominant = "attn_mma_kernel" if w.dtype == "bf16" else "attn_generic_kernel"
     src = "attn_mma.cu" if w.dtype == "bf16" else "attn_common.cu"
+    if w.kv_dtype == "fp8":
+        extra_kv = {"kv_cache": "e4m3, per-pool scale", "kv_scale": w.kv_scale}
+    else:
+        extra_kv = {}
     dk_bytes = decode_kernel_bytes(w)
     dk_s = kernel_ms["decode"] / 1e3
     achieved = dk_bytes / dk_s / 1e9
@@ -458,7 +470,7 @@ def run_ours(args, rank, world, local):
                                    "frac": round(bc["attention"] / attn_s / 1e9 /
                                                  peaks["hbm_gbs"], 4),
                                    "bytes": bc["attention"]}}
-    extra = {}
+    extra = dict(extra_kv)
     prefill_roofline = None
     if args.workload in ("mixed", "mixed_prefill"):
         fl = prefill_flops(w)

@@ -69,6 +69,8 @@ typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 #define PA_ERRBIT_QUERY_TOO_LONG 0x8  /* query_len > seq_len (or negative)         */
 #define PA_ERRBIT_TIMEOUT 0x10        /* a bounded device wait gave up             */
 #define PA_ERRBIT_POS_OOB 0x20        /* a rotary position outside the cos/sin table */
+#define PA_ERRBIT_Q_RANGE 0x40        /* FP8 cache: a query entry beyond +-65504 (the
+                                         tensor-core path takes queries as f16)  */
 
 /* One layer's cache pools. */
 typedef struct pa_cache_desc {

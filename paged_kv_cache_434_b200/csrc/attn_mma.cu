@@ -47,17 +47,23 @@ struct StageInfo {
   int pad0, pad1;
 };
 
-template <int D, int HG>
+// F8: e4m3 pools (head_dim 128).  A stage then holds [16 keys x 128 codes]
+// per head and tensor (one 128-byte swizzled row per key, the same 2 KiB tile
+// size); each consumer warp widens its head's codes to f16 in a scratch of its
+// own, laid out as the bf16 path's two [16 x 64] halves, and runs the same
+// fragment code with f16 products.
+template <int D, int HG, bool F8 = false>
 struct Cfg {
-  static constexpr int NH = D / 64;                     // 64-column halves
-  static constexpr int kTile = 2048;                    // [16 keys x 64 dims] bf16
+  static constexpr int NH = F8 ? 1 : D / 64;            // tiles per head and tensor in a stage
+  static constexpr int kTile = 2048;                    // [16 keys x 128 bytes]
   static constexpr int kTensorBytes = HG * NH * kTile;  // K (or V) part of a stage
   static constexpr int kStageBytes = 2 * kTensorBytes;
-  static constexpr int kBudget = 200 * 1024;
+  static constexpr int kScratch = F8 ? HG * 2 * (D / 64) * kTile : 0;  // f16 K and V per warp
+  static constexpr int kBudget = 200 * 1024 - kScratch;
   static constexpr int NS0 = kBudget / kStageBytes;
   static constexpr int NS = NS0 > 6 ? 6 : (NS0 < 2 ? 2 : NS0);
   static constexpr int kThreads = (HG + 1) * 32;
-  static constexpr int kSmem = NS * kStageBytes + 1024 /*align*/ + 1024 /*info+bars*/;
+  static constexpr int kSmem = NS * kStageBytes + kScratch + 1024 /*align*/ + 1024 /*info+bars*/;
 };
 
 // byte offset of (key, 16-byte chunk) inside one 128B-swizzled [16 x 64] tile
@@ -67,18 +73,21 @@ __device__ __forceinline__ uint32_t swz(int key, int chunk) {
 
 }  // namespace mmak
 
-template <int D, int HG>
+template <int D, int HG, bool F8>
 __global__ void __launch_bounds__((HG + 1) * 32, 1)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     AttnGeom g, WsView ws, int box_rows, int heads_per_box, int after_tiles) {
-  using C = mmak::Cfg<D, HG>;
+  static_assert(!F8 || D == 128, "e4m3 pools: head_dim 128");
+  using C = mmak::Cfg<D, HG, F8>;
   constexpr int NS = C::NS;
   constexpr int NH = C::NH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* stages = smem;
-  mmak::StageInfo* info = reinterpret_cast<mmak::StageInfo*>(smem + NS * C::kStageBytes);
+  uint8_t* scratch = smem + NS * C::kStageBytes;  // F8: f16 K / V tiles, 8 KiB per warp
+  mmak::StageInfo* info =
+      reinterpret_cast<mmak::StageInfo*>(smem + NS * C::kStageBytes + C::kScratch);
   uint64_t* full = reinterpret_cast<uint64_t*>(info + NS);
   uint64_t* empty = full + NS;
   __shared__ int s_abort;
@@ -218,6 +227,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   int stage = 0;
   uint32_t phase = 0;
   const __nv_bfloat16* qbase = static_cast<const __nv_bfloat16*>(g.q);
+  // score and output scales (the pools' k_scale / v_scale are already in g)
+  const float sl2 = g.scale_log2;
+  const float vsc = g.v_scale;
 
   for (;;) {
     if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
@@ -238,18 +250,68 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         qa[kk][3] =
             qr + 8 < G ? *reinterpret_cast<const uint32_t*>(qrow + (qr + 8) * D + c + 8) : 0u;
       }
+      if constexpr (F8) {
+        // f16 operands: bf16 queries are exact in f16 within +-65504
+        bool out_of_range = false;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f =
+                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[kk][i]));
+            out_of_range |= fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+            qa[kk][i] = pack_f16x2(f.x, f.y);
+          }
+        if (out_of_range && g.err_word) atomicOr(g.err_word, PA_ERRBIT_Q_RANGE);
+      }
 #pragma unroll
       for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
       m0 = m1 = -INFINITY;
       l0 = l1 = 0.f;
       bad = false;
     }
+    bool released = false;
     if (si.flags & mmak::kBad) {
       bad = true;
     } else {
-      const uint32_t kt = smem_u32(stages + stage * C::kStageBytes) + hh * C::kTile;
-      const uint32_t vt = kt + C::kTensorBytes;
-      constexpr uint32_t kHalf = HG * C::kTile;  // distance between the two halves
+      uint32_t kt = smem_u32(stages + stage * C::kStageBytes) + hh * C::kTile;
+      uint32_t vt = kt + C::kTensorBytes;
+      constexpr uint32_t kHalf = F8 ? C::kTile : HG * C::kTile;  // between the two halves
+      if constexpr (F8) {
+        // widen this head's codes to f16 in the warp's scratch (keys past the
+        // end of the request become zeros: the pool may hold NaN codes there)
+        uint8_t* k8 = stages + stage * C::kStageBytes + hh * C::kTile;
+        uint8_t* ks = scratch + hh * (4 * C::kTile);
+        __syncwarp();  // the previous stage's fragments have been read
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = lane + 32 * u;           // 128 chunks of K, then 128 of V
+          const int tsr = i >> 7, key = (i >> 3) & 15, c = i & 7;
+          const uint4 w8 = *reinterpret_cast<const uint4*>(k8 + tsr * C::kTensorBytes +
+                                                           mmak::swz(key, c));
+          uint32_t h[8];
+          const uint32_t w[4] = {w8.x, w8.y, w8.z, w8.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            h[2 * j] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] & 0xffffu));
+            h[2 * j + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] >> 16));
+          }
+          if (key >= si.nvalid) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = 0u;
+          }
+          uint8_t* dst = ks + tsr * (2 * C::kTile) + (c >> 2) * C::kTile;
+          *reinterpret_cast<uint4*>(dst + mmak::swz(key, 2 * (c & 3))) =
+              make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(dst + mmak::swz(key, 2 * (c & 3) + 1)) =
+              make_uint4(h[4], h[5], h[6], h[7]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);  // the codes are no longer needed
+        released = true;
+        kt = smem_u32(ks);
+        vt = kt + 2 * C::kTile;
+      }
       // ---- S = Q K^T over 16 keys
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
       {
@@ -261,8 +323,13 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           const int chunk = 2 * c16 + (mi & 1);
           uint32_t b0, b1, b2, b3;
           ldmatrix_x4(kt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
-          mma_bf16_16816(s0, qa[kk], b0, b1);
-          mma_bf16_16816(s1, qa[kk], b2, b3);
+          if constexpr (F8) {
+            mma_f16_16816(s0, qa[kk], b0, b1);
+            mma_f16_16816(s1, qa[kk], b2, b3);
+          } else {
+            mma_bf16_16816(s0, qa[kk], b0, b1);
+            mma_bf16_16816(s1, qa[kk], b2, b3);
+          }
         }
       }
       // ---- mask, scale, online softmax
@@ -271,8 +338,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int key = qc + (e & 1);
-        p[e] = key < nv ? s0[e] * g.scale_log2 : -INFINITY;
-        p[4 + e] = key + 8 < nv ? s1[e] * g.scale_log2 : -INFINITY;
+        p[e] = key < nv ? s0[e] * sl2 : -INFINITY;
+        p[4 + e] = key + 8 < nv ? s1[e] * sl2 : -INFINITY;
       }
       float mx0 = fmaxf(fmaxf(p[0], p[1]), fmaxf(p[4], p[5]));
       float mx1 = fmaxf(fmaxf(p[2], p[3]), fmaxf(p[6], p[7]));
@@ -291,14 +358,24 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         const float e2 = fast_exp2(p[2] - mn1), e3 = fast_exp2(p[3] - mn1);
         const float e4 = fast_exp2(p[4] - mn0), e5 = fast_exp2(p[5] - mn0);
         const float e6 = fast_exp2(p[6] - mn1), e7 = fast_exp2(p[7] - mn1);
-        pa[0] = pack_bf16x2(e0, e1);
-        pa[1] = pack_bf16x2(e2, e3);
-        pa[2] = pack_bf16x2(e4, e5);
-        pa[3] = pack_bf16x2(e6, e7);
-        // the row sums use the same bf16-rounded weights the PV product sees
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(pa);
-        const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
-        const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+        float2 f0, f1, f2, f3;
+        if constexpr (F8) {
+          pa[0] = pack_f16x2(e0, e1);
+          pa[1] = pack_f16x2(e2, e3);
+          pa[2] = pack_f16x2(e4, e5);
+          pa[3] = pack_f16x2(e6, e7);
+          f0 = f16x2_to_f32x2(pa[0]), f1 = f16x2_to_f32x2(pa[1]);
+          f2 = f16x2_to_f32x2(pa[2]), f3 = f16x2_to_f32x2(pa[3]);
+        } else {
+          pa[0] = pack_bf16x2(e0, e1);
+          pa[1] = pack_bf16x2(e2, e3);
+          pa[2] = pack_bf16x2(e4, e5);
+          pa[3] = pack_bf16x2(e6, e7);
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(pa);
+          f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+          f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+        }
+        // the row sums use the same rounded weights the PV product sees
         ps0 = f0.x + f0.y + f2.x + f2.y;
         ps1 = f1.x + f1.y + f3.x + f3.y;
       }
@@ -313,7 +390,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       }
       // ---- keys past the end of the request: zero their V rows (P is 0 there,
       // but the pool may hold non-finite garbage and 0 * inf is NaN)
-      if (nv < kStageTokens) {
+      if (!F8 && nv < kStageTokens) {
         uint8_t* vrow = stages + stage * C::kStageBytes + C::kTensorBytes + hh * C::kTile;
         for (int idx = lane; idx < (kStageTokens - nv) * 8 * NH; idx += 32) {
           const int dh = idx / ((kStageTokens - nv) * 8);
@@ -334,14 +411,19 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           const int chunk = 2 * c16 + (mi >> 1);
           uint32_t b0, b1, b2, b3;
           ldmatrix_x4_trans(vt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
-          mma_bf16_16816(o[2 * n2], pa, b0, b1);
-          mma_bf16_16816(o[2 * n2 + 1], pa, b2, b3);
+          if constexpr (F8) {
+            mma_f16_16816(o[2 * n2], pa, b0, b1);
+            mma_f16_16816(o[2 * n2 + 1], pa, b2, b3);
+          } else {
+            mma_bf16_16816(o[2 * n2], pa, b0, b1);
+            mma_bf16_16816(o[2 * n2 + 1], pa, b2, b3);
+          }
         }
       }
-      if (nv < kStageTokens) fence_proxy_async_smem();
+      if (!F8 && nv < kStageTokens) fence_proxy_async_smem();
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
+    if (lane == 0 && !released) mbar_arrive(&empty[stage]);
 
     if (si.flags & mmak::kLast) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -357,7 +439,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       } else {
         const int np = __ldcg(&ws.nparts[r]);
         if (np == 1) {
-          const float i0 = 1.f / l0, i1 = 1.f / l1;
+          const float i0 = vsc / l0, i1 = vsc / l1;
           const int64_t ob = (static_cast<int64_t>(r) * g.num_heads + head) * D;
           if (g.out_dtype == PA_F32) {
             float* out = static_cast<float*>(g.out) + ob;
@@ -390,7 +472,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
             float* po = ws.part_o + sl * D;
 #pragma unroll
             for (int j = 0; j < D / 8; ++j)
-              *reinterpret_cast<float2*>(po + j * 8 + qc) = make_float2(o[j][0], o[j][1]);
+              *reinterpret_cast<float2*>(po + j * 8 + qc) =
+                  make_float2(o[j][0] * vsc, o[j][1] * vsc);
           }
           if (qr + 8 < G) {
             const int64_t sl = slot0 + static_cast<int64_t>(qr + 8) * ws.max_parts;
@@ -398,7 +481,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
             float* po = ws.part_o + sl * D;
 #pragma unroll
             for (int j = 0; j < D / 8; ++j)
-              *reinterpret_cast<float2*>(po + j * 8 + qc) = make_float2(o[j][2], o[j][3]);
+              *reinterpret_cast<float2*>(po + j * 8 + qc) =
+                  make_float2(o[j][2] * vsc, o[j][3] * vsc);
           }
         }
       }
@@ -440,7 +524,9 @@ static bool make_pool_map(CUtensorMap* m, const void* base, const AttnGeom& g, i
                           int heads_per_box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t head_stride = static_cast<cuuint64_t>(g.head_dim) * 2;
+  // e4m3 pools: bytes; a box row is the head's 128 codes (one 128-byte row)
+  const bool f8 = g.dtype == PA_FP8_E4M3;
+  const cuuint64_t head_stride = static_cast<cuuint64_t>(g.head_dim) * (f8 ? 1 : 2);
   const cuuint64_t token_stride = head_stride * g.num_kv_heads;
   const cuuint64_t tokens = static_cast<cuuint64_t>(g.num_blocks) * g.block_size;
   const bool by_token = heads_per_box > 1;
@@ -449,11 +535,12 @@ static bool make_pool_map(CUtensorMap* m, const void* base, const AttnGeom& g, i
                         by_token ? static_cast<cuuint64_t>(g.num_kv_heads) : tokens};
   cuuint64_t strides[2] = {by_token ? token_stride : head_stride,
                            by_token ? head_stride : token_stride};
-  cuuint32_t box[3] = {64, by_token ? static_cast<cuuint32_t>(box_rows) : 1u,
+  cuuint32_t box[3] = {f8 ? 128u : 64u, by_token ? static_cast<cuuint32_t>(box_rows) : 1u,
                        by_token ? static_cast<cuuint32_t>(heads_per_box)
                                 : static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+  CUresult r = fn(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -462,15 +549,17 @@ static bool make_pool_map(CUtensorMap* m, const void* base, const AttnGeom& g, i
 bool mma_path_supported(const AttnGeom& g) {
   const int G = g.num_kv_heads > 0 ? g.num_heads / g.num_kv_heads : 0;
   const bool bs_ok = g.block_size == 8 || (g.block_size % 16 == 0 && g.block_size <= 256);
-  return g.dtype == PA_BF16 && (g.head_dim == 64 || g.head_dim == 128) && G >= 1 &&
-         G <= kMaxGroup && bs_ok && encode_fn() != nullptr &&
+  const bool type_ok = g.dtype == PA_BF16 ||
+                       (g.dtype == PA_FP8_E4M3 && g.head_dim == 128 && g.block_size % 16 == 0);
+  return type_ok && (g.head_dim == 64 || g.head_dim == 128) && G >= 1 && G <= kMaxGroup &&
+         bs_ok && encode_fn() != nullptr &&
          static_cast<int64_t>(g.num_blocks) * g.block_size < (1LL << 31);
 }
 
-template <int D, int HG>
+template <int D, int HG, bool F8 = false>
 static cudaError_t launch_mma_t(const AttnGeom& g, const WsView& ws, int num_sms, int after_tiles,
                                 cudaStream_t s) {
-  using C = mmak::Cfg<D, HG>;
+  using C = mmak::Cfg<D, HG, F8>;
   const int box_rows = g.block_size < kStageTokens ? g.block_size : kStageTokens;
   CUtensorMap tk, tv;
   int heads_per_box = (box_rows == kStageTokens && HG > 1) ? HG : 1;
@@ -480,20 +569,29 @@ static cudaError_t launch_mma_t(const AttnGeom& g, const WsView& ws, int num_sms
   if (heads_per_box == 1 && !(make_pool_map(&tk, g.k_cache, g, box_rows, 1) &&
                               make_pool_map(&tv, g.v_cache, g, box_rows, 1)))
     return cudaErrorInvalidValue;
-  auto kern = attn_mma_kernel<D, HG>;
+  auto kern = attn_mma_kernel<D, HG, F8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  return launch_pdl<attn_mma_kernel<D, HG>>(dim3(num_sms * per_sm), dim3(C::kThreads), C::kSmem,
+  return launch_pdl<attn_mma_kernel<D, HG, F8>>(dim3(num_sms * per_sm), dim3(C::kThreads),
+                                                C::kSmem,
                                             s, tk, tv, g, ws, box_rows, heads_per_box,
                                             after_tiles);
 }
 
 cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,
                             int after_tiles, cudaStream_t s) {
+  if (g.dtype == PA_FP8_E4M3) {  // head_dim 128 (mma_path_supported)
+    switch (heads_per_group) {
+      case 8: return launch_mma_t<128, 8, true>(g, ws, num_sms, after_tiles, s);
+      case 4: return launch_mma_t<128, 4, true>(g, ws, num_sms, after_tiles, s);
+      case 2: return launch_mma_t<128, 2, true>(g, ws, num_sms, after_tiles, s);
+      default: return launch_mma_t<128, 1, true>(g, ws, num_sms, after_tiles, s);
+    }
+  }
   if (g.head_dim == 128) {
     switch (heads_per_group) {
       case 8: return launch_mma_t<128, 8>(g, ws, num_sms, after_tiles, s);

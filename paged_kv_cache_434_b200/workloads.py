@@ -262,6 +262,16 @@ def make_tensors(w: Workload, device="cpu", where: str = "auto"):
     return out
 
 
+def llama8b_decode_fp8(seed: int = 0) -> Workload:
+    """llama8b_decode over e4m3 pools (per-pool scale 1/56)."""
+    return with_fp8_cache(llama8b_decode(seed))
+
+
+def long_context_decode_fp8(seed: int = 0) -> Workload:
+    """long_context_decode over e4m3 pools (per-pool scale 1/56)."""
+    return with_fp8_cache(long_context_decode(seed))
+
+
 def with_fp8_cache(w: Workload, scale: float = 1.0 / 56.0) -> Workload:
     """The same workload over e4m3 pools (N(0,1) entries over 1/56: |x| <= 8
     stays below the format's 448)."""
