@@ -135,17 +135,21 @@ __device__ int shared_prefix_blocks(const AttnGeom& g, int max_cols, int* s_bad)
     for (int u = 0; u < kPer; ++u) {
       const int idx = threadIdx.x + u * blockDim.x;
       v[u] = ref[u] = 0;
-      if (idx < pairs) {
-        const int j = c0 + idx / g.num_seqs, b = idx % g.num_seqs;
+      if (idx < pairs) {  // consecutive threads: consecutive columns of one table row
+        const int w = c1 - c0;
+        const int j = c0 + idx % w, b = idx / w;
         v[u] = g.block_tables[static_cast<int64_t>(b) * g.max_blocks + j];
         ref[u] = g.block_tables[j];
       }
     }
+    int first = 0x7fffffff;  // first differing column this thread saw
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int idx = threadIdx.x + u * blockDim.x;
-      if (idx < pairs && v[u] != ref[u]) atomicMin(s_bad, c0 + idx / g.num_seqs);
+      if (idx < pairs && v[u] != ref[u]) first = min(first, c0 + idx % (c1 - c0));
     }
+    first = __reduce_min_sync(0xffffffffu, first);  // one shared atomic per warp
+    if ((threadIdx.x & 31) == 0 && first != 0x7fffffff) atomicMin(s_bad, first);
     __syncthreads();
     // later atomics only lower s_bad to columns >= c1, so every thread sees the
     // same answer to this test
@@ -257,6 +261,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   // cooperatively, rows marked, tiles counted per bin
   const int npref = min(s_npref, kMaxPrefill);
   int n_tiles_total = 0;
+  unsigned long long my_tile_kv = 0;  // summed per warp below (one shared atomic per warp)
   for (int pi = 0; pi < npref; ++pi) {
     const int b = s_pref[pi];
     const int L = g.seq_lens[b];
@@ -287,11 +292,17 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
         atomicAdd(&s_hist[tile_bin(n_kv)], 1);
         // (query tile, key tile) products of this item: one or two query tiles
         const int halves = last + 1 - tb * a.tile_tokens > a.tile_tokens / 2 ? 2 : 1;
-        atomicAdd(&s_tile_kv, static_cast<unsigned long long>(n_kv * halves));
+        my_tile_kv += static_cast<unsigned long long>(n_kv * halves);
       }
       n_tiles_total += ntb * g.num_kv_heads;
     }
     __syncthreads();
+  }
+
+  if (npref > 0) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) my_tile_kv += __shfl_xor_sync(0xffffffffu, my_tile_kv, o);
+    if (lane == 0 && my_tile_kv) atomicAdd(&s_tile_kv, my_tile_kv);
   }
 
   // 1d. decode cascade: a prefix of blocks shared by every request is attended
@@ -447,14 +458,32 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
 
   // 4. tiles, longest first
   if (npref > 0) {
-    if (tid == 0) {
-      int acc = 0;
-      for (int bin = kTileBins - 1; bin >= 0; --bin) {
-        const int c = s_hist[bin];
-        s_hist[bin] = acc;
-        acc += c;
-      }
+    // exclusive scan of the bins from the longest down: two bins per thread
+    static_assert(kTileBins == 2 * kPlanThreads, "two bins per thread");
+    const int b0 = kTileBins - 1 - 2 * tid, b1 = b0 - 1;
+    const int c0 = s_hist[b0], c1 = s_hist[b1];
+    int incl = c0 + c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
     }
+    if (lane == 31) s_scan[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int v = s_scan[lane];
+      int vi = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, vi, o);
+        if (lane >= o) vi += n;
+      }
+      s_scan[lane] = vi - v;  // warps before this one
+    }
+    __syncthreads();
+    const int before = s_scan[warp] + incl - (c0 + c1);
+    s_hist[b0] = before;
+    s_hist[b1] = before + c0;
     __syncthreads();
     for (int pi = 0; pi < npref; ++pi) {
       const int b = s_pref[pi];
