@@ -746,7 +746,7 @@ def run_reference(args, rank, world, local):
     else:
         t = W.make_tensors(w, "cpu", where="host")
         pools = (t["k_cache"], t["v_cache"])
-    per_step = max(0.5, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.1, min(args.cpu_seconds, 60.0 / max(1, args.steps + args.warmup)))
     vals = []
     desc = threads = None
     for k in range(max(args.warmup, 3) + args.steps):
@@ -1028,7 +1028,7 @@ def run_rope_reference(args, rank, world, local):
         x = rope_inputs(w, dev, args.seed)
     else:
         x = rope_inputs_cpu(w, args.seed)
-    per_step = max(0.5, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.1, min(args.cpu_seconds, 60.0 / max(1, args.steps + args.warmup)))
     vals = [rope_oracle_sample(w, x, per_step, rng_seed=k)["value"]
             for k in range(max(args.warmup, 3) + args.steps)][max(args.warmup, 3):]
     value = statistics.mean(vals)
