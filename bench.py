@@ -34,6 +34,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -126,9 +127,11 @@ def kernel_traffic(kernel_src: str, profile_md: str):
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     vals = {}
     for line in open(path, encoding="utf-8"):
-        if ":" in line and line.strip().startswith(("kernel_source_sha256", "traffic_bytes_per_launch")):
+        if ":" in line and line.strip().lstrip("- ").startswith(("kernel_source_sha256",
+                                                                  "traffic_bytes_per_launch")):
             k, v = line.split(":", 1)
-            vals[k.strip().lstrip("- ").strip()] = v.strip().strip("`")
+            m = re.search(r"`([^`]+)`", v)  # the value is the first `quoted` token
+            vals[k.strip().lstrip("- ").strip()] = m.group(1) if m else v.strip()
     if vals.get("kernel_source_sha256") != sha:
         return None
     try:
