@@ -243,23 +243,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x on the FMA pipe (no XU/MUFU use), for softmax weights that are rounded to
-// bf16 afterwards.  Cody-Waite style range reduction: x = j + f with
-// j = round(x) (obtained by adding 1.5 * 2^23) and f in [-0.5, 0.5]; 2^f from a
-// cubic fitted by least squares to the relative error on [-0.5, 0.5] (max
-// relative error 7.7e-5, far below bf16's 2^-9); j is added to the exponent
-// field.  x is clamped to >= -126, so -inf gives 2^-126 (about 1e-38).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const int j = __float_as_int(t) - 0x4B400000;
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(f, 0.05508868f, 0.24260405f);
-  p = fmaf(p, f, 0.69327623f);
-  p = fmaf(p, f, 0.99992895f);
-  return __int_as_float(__float_as_int(p) + (j << 23));
-}
-
 // ------------------------------------------------------------------ tcgen05 (sm_100a)
 // Tensor memory: 128 lanes x 512 columns of 32-bit cells per SM.  A warp may
 // only touch lanes [32 * (warp % 4), +32).  Address = (lane << 16) | column.
