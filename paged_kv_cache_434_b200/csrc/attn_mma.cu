@@ -36,6 +36,7 @@ namespace pa {
 namespace mmak {
 
 enum : int { kFirst = 1, kLast = 2, kBad = 4, kEnd = 8 };
+constexpr float kRescaleLog2 = 8.f;  // lazy O rescale threshold (log2 units)
 
 struct StageInfo {
   int qrow;
@@ -347,8 +348,14 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float a0 = fast_exp2(m0 - mn0), a1 = fast_exp2(m1 - mn1);
+      // lazy rescale: the reference max moves only when a row's max grows by
+      // more than 2^8 (the weights then stay <= 256, exact enough in bf16 / f16
+      // and fp32), so in steady state O is not touched; (m, l, o) stay
+      // consistent for any reference, and the merge re-normalises partials
+      const bool up0 = mx0 > m0 + mmak::kRescaleLog2, up1 = mx1 > m1 + mmak::kRescaleLog2;
+      const float mn0 = up0 ? mx0 : m0, mn1 = up1 ? mx1 : m1;
+      const float a0 = up0 ? fast_exp2(m0 - mn0) : 1.f, a1 = up1 ? fast_exp2(m1 - mn1) : 1.f;
+      const bool rescale = __any_sync(0xffffffffu, up0 || up1);
       m0 = mn0;
       m1 = mn1;
       uint32_t pa[4];
@@ -381,12 +388,14 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       }
       l0 = l0 * a0 + ps0;
       l1 = l1 * a1 + ps1;
+      if (rescale) {
 #pragma unroll
-      for (int j = 0; j < D / 8; ++j) {
-        o[j][0] *= a0;
-        o[j][1] *= a0;
-        o[j][2] *= a1;
-        o[j][3] *= a1;
+        for (int j = 0; j < D / 8; ++j) {
+          o[j][0] *= a0;
+          o[j][1] *= a0;
+          o[j][2] *= a1;
+          o[j][3] *= a1;
+        }
       }
       // ---- keys past the end of the request: zero their V rows (P is 0 there,
       // but the pool may hold non-finite garbage and 0 * inf is NaN)
