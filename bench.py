@@ -79,16 +79,29 @@ def parse_args(argv=None):
 
 
 def dist_setup():
+    """Rank, world size and local rank from the torchrun environment; with more
+    than one rank, a process group (NCCL on GPUs; gloo where no GPU is present,
+    which only the host-side tests use) with a short timeout."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout,
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     return rank, world, local
+
+
+def job_throughput(units_per_step: float, steps: int, world: int, max_total_s: float) -> float:
+    """Whole-job rate: every rank processed `units_per_step` each step (weak
+    scaling), divided by the slowest rank's timed seconds."""
+    return units_per_step * steps * world / max_total_s
 
 
 def barrier(world):
@@ -445,9 +458,9 @@ def run_ours(args, rank, world, local):
     bc = byte_counts(w)
     metric, unit = metric_of(args.workload)
     if args.workload in ("mixed", "mixed_prefill"):
-        value = T * args.steps * world / total_s
+        value = job_throughput(T, args.steps, world, total_s)
     else:
-        value = bc["step"] * args.steps * world / total_s / 1e9
+        value = job_throughput(bc["step"], args.steps, world, total_s) / 1e9
     peaks = load_peaks()
     attn_s = statistics.mean(attn_ms) / 1e3
     dominant = "attn_mma_kernel" if w.dtype == "bf16" else "attn_generic_kernel"
