@@ -150,3 +150,52 @@ def test_kernel_timing_off_paths(lib):
     assert lib.pa_kernel_timing_enable(0) == B.PA_OK          # off while off: no CUDA call
     assert lib.pa_kernel_timing_read(ms) == B.PA_ERR_INVALID_ARG
     assert lib.pa_kernel_timing_read(None) == B.PA_ERR_INVALID_ARG
+
+
+def test_fp8_descriptor_validation(lib):
+    from paged_kv_cache_434_b200 import binding as B
+    ok = _desc(dtype=2, k_scale=0.5, v_scale=0.25)
+    # zero tokens: nothing to do once the descriptor is valid
+    assert lib.pa_cache_write(None, None, None, None, None, 0, ctypes.byref(ok), None, None) == B.PA_OK
+    for bad in (dict(k_scale=0.0, v_scale=1.0), dict(k_scale=1.0, v_scale=-2.0),
+                dict(k_scale=float("inf"), v_scale=1.0), dict(k_scale=float("nan"), v_scale=1.0)):
+        d = _desc(dtype=2, **bad)
+        assert lib.pa_cache_write(None, None, None, None, None, 0, ctypes.byref(d), None,
+                                  None) == B.PA_ERR_INVALID_ARG
+    # rotary embedding does not take an e4m3 cache
+    assert lib.pa_rope_cache_write(16, 16, 16, 512, 128, 32, 16, 16, 16, 16, 16, 64, 64, 1, 1, 4,
+                                   ctypes.byref(ok), None, None) == B.PA_ERR_UNSUPPORTED
+
+
+def test_rope_validation(lib):
+    from paged_kv_cache_434_b200 import binding as B
+    d = _desc(head_dim=64)
+    call = lambda **kw: lib.pa_rope_cache_write(  # noqa: E731
+        kw.get("q", 16), 16, 16, kw.get("qs", 4 * 64), kw.get("ks", 2 * 64), kw.get("qo", 1 << 20),
+        16, 16, 16, 16, 16, 64, kw.get("rot", 64), 1, kw.get("T", 3), 4, ctypes.byref(d), None,
+        None)
+    assert call(rot=24) == B.PA_ERR_UNSUPPORTED               # not a multiple of 16
+    assert call(rot=128) == B.PA_ERR_UNSUPPORTED              # larger than head_dim
+    assert call(qs=64) == B.PA_ERR_INVALID_ARG                # q rows shorter than 4 heads
+    assert call(ks=36) == B.PA_ERR_INVALID_ARG                # not a multiple of 8 elements
+    assert call(qo=16 + 64) == B.PA_ERR_INVALID_ARG           # q_out overlaps q_in, not equal
+    assert call(q=None) == B.PA_ERR_INVALID_ARG
+    assert call(T=0, q=None) == B.PA_OK                       # nothing to do
+    assert lib.pa_rope_cos_sin_cache(None, 16, 16, 1e4, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_rope_cos_sin_cache(16, 16, 15, 1e4, None) == B.PA_ERR_INVALID_ARG   # odd
+    assert lib.pa_rope_cos_sin_cache(16, 16, 16, 0.0, None) == B.PA_ERR_INVALID_ARG
+
+
+def test_block_management_validation(lib):
+    from paged_kv_cache_434_b200 import binding as B
+    d = _desc()
+    assert lib.pa_copy_blocks(16, 16, 16, -1, ctypes.byref(d), None, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_copy_blocks(None, None, None, 0, ctypes.byref(d), None, None) == B.PA_OK
+    assert lib.pa_copy_blocks(None, 16, 16, 3, ctypes.byref(d), None, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_copy_blocks(8, 16, 16, 3, ctypes.byref(d), None, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_slot_mapping_positions(None, 4, 2, None, None, 5, 16, 16, None, None, None) == \
+        B.PA_ERR_INVALID_ARG
+    assert lib.pa_slot_mapping_positions(None, 4, 2, None, None, 0, 16, 16, None, None, None) == \
+        B.PA_OK
+    assert lib.pa_slot_mapping_positions(16, 4, 2, 16, 16, 5, 0, 16, 16, None, None) == \
+        B.PA_ERR_INVALID_ARG                                 # block size 0
