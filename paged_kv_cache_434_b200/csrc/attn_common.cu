@@ -219,9 +219,12 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
       continue;  // its rows stay unwritten
     }
     if (decode_mode && a.cascade) {
-      // units are counted once the shared prefix is known
+      // units as if no prefix is shared; recounted below if one is
       atomicMin(&s_minL, L);
       ws.qrow_info[r0] = make_int4(b, L, 1, 0);
+      const int units = (L + kStageTokens - 1) / kStageTokens;
+      my_units += units;
+      my_max = max(my_max, units);
       continue;
     }
     const bool tile = !(decode_mode || q_b == 1 || a.expand_prefill);
@@ -315,16 +318,19 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
       const int pb = shared_prefix_blocks(g, max_cols, &s_pbad);
       if (pb * g.block_size >= kCascadeMinPrefix) prefix_tokens = pb * g.block_size;
     }
-    for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
-      int4 info = ws.qrow_info[r];
-      if (info.z == 0) continue;
-      info.w = prefix_tokens;
-      ws.qrow_info[r] = info;
-      const int units = (info.y - prefix_tokens + kStageTokens - 1) / kStageTokens;
-      my_units += units;
-      my_max = max(my_max, units);
-    }
     if (prefix_tokens > 0) {
+      // rows keep only their suffix (thread tid filled rows tid, tid + 1024, ...)
+      my_units = 0;
+      my_max = 0;
+      for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
+        int4 info = ws.qrow_info[r];
+        if (info.z == 0) continue;
+        info.w = prefix_tokens;
+        ws.qrow_info[r] = info;
+        const int units = (info.y - prefix_tokens + kStageTokens - 1) / kStageTokens;
+        my_units += units;
+        my_max = max(my_max, units);
+      }
       // tiles of (requests x heads) rows; the prefix keys are split into chunks
       // so that there are about as many tiles as SMs
       const int per = a.tile_tokens;  // requests per tile pair
