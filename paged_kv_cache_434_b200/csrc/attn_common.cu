@@ -332,13 +332,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
         my_max = max(my_max, units);
       }
       // tiles of (requests x heads) rows; the prefix keys are split into chunks
-      // so that there are about as many tiles as SMs
       const int per = a.tile_tokens;  // requests per tile pair
       const int groups = (g.num_seqs + per - 1) / per;
       const int kv_tiles = (prefix_tokens + 127) / 128;
       const int base = groups * g.num_kv_heads;
-      // one wave: at most one tile per SM
-      const int want = min(min(kMaxPrefixChunks, kv_tiles), max(1, a.num_sms / base));
+      // at most one tile per two SMs: the suffix partitions start at once on
+      // the SMs the tiles leave free (longer tiles on half the SMs measured
+      // 11 % faster than one wave of shorter tiles, a quarter 13 % slower)
+      const int want = min(min(kMaxPrefixChunks, kv_tiles), max(1, a.num_sms / (2 * base)));
       const int per_chunk = (kv_tiles + want - 1) / want;
       prefix_chunks = (kv_tiles + per_chunk - 1) / per_chunk;  // no empty chunk
       for (int idx = tid; idx < base * prefix_chunks; idx += kPlanThreads) {
