@@ -168,7 +168,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   __shared__ long long s_sum[32];
   __shared__ int s_max[32];
   __shared__ int s_scan[32];
-  __shared__ int s_P, s_merge, s_npref, s_nbig, s_badpref, s_minL, s_nbad, s_pbad, s_ntc;
+  __shared__ int s_P, s_merge, s_merge_big, s_npref, s_nbig, s_badpref, s_minL, s_nbad, s_pbad,
+      s_ntc;
   __shared__ unsigned long long s_tile_kv;
   __shared__ int s_pref[kMaxPrefill];
   __shared__ int s_big[kMaxBig];
@@ -186,6 +187,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   }
   if (tid == 0) {
     s_merge = 0;
+    s_merge_big = 0;
     s_npref = 0;
     s_nbig = 0;
     s_minL = 0x7fffffff;
@@ -438,7 +440,12 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     const int units = (info.y - info.w + kStageTokens - 1) / kStageTokens;
     const int np = (units + P - 1) / P;
     ws.nparts[r] = np + (info.w > 0 ? prefix_chunks : 0);  // the last ones: shared-prefix chunks
-    if (ws.nparts[r] != 1) ws.merge_rows[atomicAdd(&s_merge, 1)] = r;
+    // rows to merge: those a warp merges from the front of the list, those
+    // with more than 32 partitions (a CTA each) from the back
+    if (ws.nparts[r] > 32)
+      ws.merge_rows[g.num_qrows - 1 - atomicAdd(&s_merge_big, 1)] = r;
+    else if (ws.nparts[r] != 1)
+      ws.merge_rows[atomicAdd(&s_merge, 1)] = r;
     const int n_it = np * a.head_groups;
     if (n_it > kInlineItems) {
       const int slot = atomicAdd(&s_nbig, 1);
@@ -512,6 +519,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   if (tid == 0) {
     ws.ctrl[4] = static_cast<int>(min(static_cast<int64_t>(n_tiles_total), ws.max_tiles));
     ws.ctrl[5] = s_merge;
+    ws.ctrl[9] = s_merge_big;
     ws.ctrl[6] = prefix_tokens;
     ws.ctrl[7] = prefix_chunks;
     ws.ctrl[8] = s_ntc;
@@ -799,6 +807,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(AttnGeom g, WsV
   grid_dependency_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pairs = static_cast<int64_t>(ws.ctrl[5]) * g.num_heads;
+  const int64_t big_pairs = static_cast<int64_t>(ws.ctrl[9]) * g.num_heads;
   // pass 1: (row, head) pairs with at most 32 partitions, one warp each
   for (int64_t pi = static_cast<int64_t>(blockIdx.x) * kMergeWarps + warp; pi < pairs;
        pi += static_cast<int64_t>(gridDim.x) * kMergeWarps) {
@@ -807,9 +816,9 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(AttnGeom g, WsV
     if (np == 1 || np < 0 || np > 32 || ws.qrow_bad[r]) continue;
     merge_pair_warp<D>(g, ws, static_cast<int64_t>(r) * g.num_heads + pi % g.num_heads, np, lane);
   }
-  // pass 2: pairs with more partitions, one CTA each
-  for (int64_t pi = blockIdx.x; pi < pairs; pi += gridDim.x) {
-    const int r = ws.merge_rows[pi / g.num_heads];
+  // pass 2: pairs with more partitions (listed from the back), one CTA each
+  for (int64_t pi = blockIdx.x; pi < big_pairs; pi += gridDim.x) {
+    const int r = ws.merge_rows[g.num_qrows - 1 - pi / g.num_heads];
     const int64_t idx = static_cast<int64_t>(r) * g.num_heads + pi % g.num_heads;
     const int np = ws.nparts[r];
     if (np <= 32 || ws.qrow_bad[r]) continue;
