@@ -1,8 +1,8 @@
 // ptx.cuh -- thin inline-PTX wrappers used by the sm_100a kernels.
 //
-// Written from the public PTX ISA: mbarrier, cp.async.bulk.tensor (TMA, no
-// multicast), cp.async, ldmatrix, mma.sync, tcgen05 (TMEM, UMMA), ex2.approx,
-// griddepcontrol, %globaltimer.
+// Written from the public PTX ISA: mbarrier, cp.async.bulk.tensor (TMA into
+// the issuing CTA's own shared memory only), cp.async, ldmatrix, mma.sync,
+// tcgen05 (TMEM, UMMA), ex2.approx, griddepcontrol, %globaltimer.
 #pragma once
 
 #include <cstdint>
