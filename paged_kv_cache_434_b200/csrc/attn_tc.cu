@@ -168,8 +168,8 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
   const uint32_t sK = smem_u32(smem + C::kOffK);
   const uint32_t sV = smem_u32(smem + C::kOffV);
   // the planner may leave part of the SMs to the decode partitions that run
-  // beside the tiles: those CTAs only release their TMEM
-  const bool working = static_cast<int>(blockIdx.x) < ws.ctrl[8];
+  // beside the tiles, or find no tile at all: such CTAs only release their TMEM
+  const bool working = static_cast<int>(blockIdx.x) < ws.ctrl[8] && n_tiles > 0;
 
   if (!working) {
   } else if (warp == 3) {
