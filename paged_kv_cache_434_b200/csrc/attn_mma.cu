@@ -50,16 +50,18 @@ struct StageInfo {
 
 // F8: e4m3 pools (head_dim 128).  A stage then holds [16 keys x 128 codes]
 // per head and tensor (one 128-byte swizzled row per key, the same 2 KiB tile
-// size); each consumer warp widens its head's codes to f16 in a scratch of its
-// own, laid out as the bf16 path's two [16 x 64] halves, and runs the same
-// fragment code with f16 products.
+// size).  K fragments are widened in registers straight from an ldmatrix of
+// the codes (the dimension order inside each 16-dim step is permuted, and the
+// query fragments follow the same order); V codes are widened to f16 in a
+// scratch of the warp's own, laid out as the bf16 path's two [16 x 64]
+// halves, for the transposed loads of the P V product.
 template <int D, int HG, bool F8 = false>
 struct Cfg {
   static constexpr int NH = F8 ? 1 : D / 64;            // tiles per head and tensor in a stage
   static constexpr int kTile = 2048;                    // [16 keys x 128 bytes]
   static constexpr int kTensorBytes = HG * NH * kTile;  // K (or V) part of a stage
   static constexpr int kStageBytes = 2 * kTensorBytes;
-  static constexpr int kScratch = F8 ? HG * 2 * (D / 64) * kTile : 0;  // f16 K and V per warp
+  static constexpr int kScratch = F8 ? HG * (D / 64) * kTile : 0;  // f16 V per warp
   static constexpr int kBudget = 200 * 1024 - kScratch;
   static constexpr int NS0 = kBudget / kStageBytes;
   static constexpr int NS = NS0 > 6 ? 6 : (NS0 < 2 ? 2 : NS0);
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* stages = smem;
-  uint8_t* scratch = smem + NS * C::kStageBytes;  // F8: f16 K / V tiles, 8 KiB per warp
+  uint8_t* scratch = smem + NS * C::kStageBytes;  // F8: f16 V tiles, 4 KiB per warp
   mmak::StageInfo* info =
       reinterpret_cast<mmak::StageInfo*>(smem + NS * C::kStageBytes + C::kScratch);
   uint64_t* full = reinterpret_cast<uint64_t*>(info + NS);
@@ -242,14 +244,17 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     const int head = (si.hg * HG + hh) * G;  // first query head of this warp's group
     if (si.flags & mmak::kFirst) {
       const __nv_bfloat16* qrow = qbase + (static_cast<int64_t>(si.qrow) * g.num_heads + head) * D;
+      // F8: k slots (2j, 2j+1 | 2j+8, 2j+9) of a 16-dim step hold dims
+      // (4j, 4j+1 | 4j+2, 4j+3), the order the widened K fragments come in
+      const int c_lo = F8 ? 4 * (lane & 3) : qc, c_hi = F8 ? c_lo + 2 : qc + 8;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const int c = kk * 16 + qc;
+        const int c = kk * 16 + c_lo, ch = kk * 16 + c_hi;
         qa[kk][0] = qr < G ? *reinterpret_cast<const uint32_t*>(qrow + qr * D + c) : 0u;
         qa[kk][1] = qr + 8 < G ? *reinterpret_cast<const uint32_t*>(qrow + (qr + 8) * D + c) : 0u;
-        qa[kk][2] = qr < G ? *reinterpret_cast<const uint32_t*>(qrow + qr * D + c + 8) : 0u;
+        qa[kk][2] = qr < G ? *reinterpret_cast<const uint32_t*>(qrow + qr * D + ch) : 0u;
         qa[kk][3] =
-            qr + 8 < G ? *reinterpret_cast<const uint32_t*>(qrow + (qr + 8) * D + c + 8) : 0u;
+            qr + 8 < G ? *reinterpret_cast<const uint32_t*>(qrow + (qr + 8) * D + ch) : 0u;
       }
       if constexpr (F8) {
         // f16 operands: bf16 queries are exact in f16 within +-65504
@@ -279,17 +284,16 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       uint32_t vt = kt + C::kTensorBytes;
       constexpr uint32_t kHalf = F8 ? C::kTile : HG * C::kTile;  // between the two halves
       if constexpr (F8) {
-        // widen this head's codes to f16 in the warp's scratch (keys past the
-        // end of the request become zeros: the pool may hold NaN codes there)
-        uint8_t* k8 = stages + stage * C::kStageBytes + hh * C::kTile;
-        uint8_t* ks = scratch + hh * (4 * C::kTile);
+        // widen this head's V codes to f16 in the warp's scratch (keys past
+        // the end of the request become zeros: the pool may hold NaN codes)
+        const uint8_t* v8 = stages + stage * C::kStageBytes + C::kTensorBytes + hh * C::kTile;
+        uint8_t* vs = scratch + hh * (2 * C::kTile);
         __syncwarp();  // the previous stage's fragments have been read
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int i = lane + 32 * u;           // 128 chunks of K, then 128 of V
-          const int tsr = i >> 7, key = (i >> 3) & 15, c = i & 7;
-          const uint4 w8 = *reinterpret_cast<const uint4*>(k8 + tsr * C::kTensorBytes +
-                                                           mmak::swz(key, c));
+        for (int u = 0; u < 4; ++u) {
+          const int i = lane + 32 * u;  // 128 chunks of 16 codes
+          const int key = i >> 3, c = i & 7;
+          const uint4 w8 = *reinterpret_cast<const uint4*>(v8 + mmak::swz(key, c));
           uint32_t h[8];
           const uint32_t w[4] = {w8.x, w8.y, w8.z, w8.w};
 #pragma unroll
@@ -301,21 +305,36 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 #pragma unroll
             for (int j = 0; j < 8; ++j) h[j] = 0u;
           }
-          uint8_t* dst = ks + tsr * (2 * C::kTile) + (c >> 2) * C::kTile;
+          uint8_t* dst = vs + (c >> 2) * C::kTile;
           *reinterpret_cast<uint4*>(dst + mmak::swz(key, 2 * (c & 3))) =
               make_uint4(h[0], h[1], h[2], h[3]);
           *reinterpret_cast<uint4*>(dst + mmak::swz(key, 2 * (c & 3) + 1)) =
               make_uint4(h[4], h[5], h[6], h[7]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);  // the codes are no longer needed
-        released = true;
-        kt = smem_u32(ks);
-        vt = kt + 2 * C::kTile;
+        vt = smem_u32(vs);
       }
       // ---- S = Q K^T over 16 keys
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-      {
+      if constexpr (F8) {
+        // one ldmatrix of the code tile gives two 16-dim steps x 16 keys: a
+        // lane holds 4 codes (dims 4j..4j+3) of one key per matrix
+        const int mi = lane >> 3;
+        const int key = (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; kk += 2) {
+          uint32_t r[4];
+          ldmatrix_x4(kt + mmak::swz(key, kk + (mi >> 1)), r[0], r[1], r[2], r[3]);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t lo = e4m3x2_to_f16x2(static_cast<uint16_t>(r[m] & 0xffffu));
+            const uint32_t hi = e4m3x2_to_f16x2(static_cast<uint16_t>(r[m] >> 16));
+            mma_f16_16816((m & 1) ? s1 : s0, qa[kk + (m >> 1)], lo, hi);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);  // codes of K and V consumed
+        released = true;
+      } else {
         const int mi = lane >> 3;
         const int key = (lane & 7) + ((mi >> 1) << 3);
 #pragma unroll
@@ -324,13 +343,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           const int chunk = 2 * c16 + (mi & 1);
           uint32_t b0, b1, b2, b3;
           ldmatrix_x4(kt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
-          if constexpr (F8) {
-            mma_f16_16816(s0, qa[kk], b0, b1);
-            mma_f16_16816(s1, qa[kk], b2, b3);
-          } else {
-            mma_bf16_16816(s0, qa[kk], b0, b1);
-            mma_bf16_16816(s1, qa[kk], b2, b3);
-          }
+          mma_bf16_16816(s0, qa[kk], b0, b1);
+          mma_bf16_16816(s1, qa[kk], b2, b3);
         }
       }
       // ---- mask, scale, online softmax
