@@ -16,19 +16,33 @@
  *                     step mixing chunked-prefill tokens and decode tokens, every
  *                     K/V read through the block table (same section: the v1
  *                     unified varlen call over the paged cache)
+ *   pa_rope_cos_sin_cache, pa_rope_cache_write
+ *                     rotary position embedding of Q/K fused with the cache
+ *                     write ("Reshape & Cache")
+ *   pa_copy_blocks    copy-on-write block copies ("第三部分 · 推理系统与基础设施",
+ *                     chapter map 3.3)
+ *   pa_slot_mapping_positions
+ *                     slots from explicit (request, position) pairs
+ *   PA_FP8_E4M3       e4m3 cache pools with one scale per pool ("从零构建LLM
+ *                     推理引擎", card "量化")
+ *   pa_decode_no_alloc, pa_kernel_timing_enable / _read
+ *                     entry points with no counterpart on the pages (a decode
+ *                     for callers that cannot allocate; per-launch timing)
  *
  * Conventions shared by every call
  *   - All tensor arguments are DEVICE pointers of the current CUDA device,
  *     row-major and densely packed, owned by the caller.  The library never
  *     allocates, frees or retains them, and keeps no state between calls
- *     other than a per-device cache of launch attributes.
+ *     other than a per-device cache of launch attributes (and, where those
+ *     entry points are used, the no-alloc scratch and the timing events).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *     is asynchronous: it validates on the host, enqueues kernels on `stream`
  *     and returns.  Host-detectable errors return a non-zero pa_status and
  *     enqueue nothing.
  *   - Cache pools: key_cache and value_cache are each
  *     [num_blocks, block_size, num_kv_heads, head_dim] (one layer), dtype
- *     cache->dtype.
+ *     cache->dtype (e4m3 codes for PA_FP8_E4M3, whose queries and new K/V
+ *     rows are bf16).
  *   - Index arrays are int32 (block_tables, seq_lens, query_start_loc) except
  *     slot_mapping (int64, as in the page's reshape_and_cache code).
  *   - Device-detected errors never trap: the offending item is skipped and a
