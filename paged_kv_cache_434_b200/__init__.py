@@ -10,6 +10,7 @@ its Python binding plus a seeded workload generator:
   copy_blocks    copy-on-write block copies in both pools
   slot_mapping_positions  slots from explicit (request, position) pairs
   decode         GQA decode attention, online softmax, split-KV + LSE merge
+  decode_no_alloc  decode through the library's own static scratch
   mixed_step     causal varlen attention of a chunked-prefill + decode step
   step           slot_mapping -> cache_write -> attention, the per-layer path
 """
@@ -25,6 +26,7 @@ from .binding import (  # noqa: F401
     cache_write,
     copy_blocks,
     decode,
+    decode_no_alloc,
     decode_workspace_size,
     kernel_times,
     kernel_timing,
