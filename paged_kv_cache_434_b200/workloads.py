@@ -193,15 +193,6 @@ def mixed_step_prefill_only(seed: int = 0, chunk: int = 2048, prefix: int = 4096
     return custom("mixed_prefill_chunks_bf16", lens, qlens, 32, 8, 128, 16, "bf16", seed)
 
 
-CONFIGS = {
-    1: tiny_decode,
-    2: llama8b_decode,
-    3: long_context_decode,
-    4: mixed_step,
-    5: shared_prefix_decode,
-}
-
-
 # --------------------------------------------------------------------------
 # Tensor values
 # --------------------------------------------------------------------------

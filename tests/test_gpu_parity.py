@@ -258,7 +258,7 @@ def test_error_bits_bad_inputs(cuda_device):
     assert changed == [5]
 
 
-# ---------------------------------------------------------------- full-size configs
+# ---------------------------------------------------------------- full-size workloads
 
 def _full_size(w, dev, sample_rows, out_dtype=torch.float32):
     """Run a full-size workload through the step; check slots/writes by
