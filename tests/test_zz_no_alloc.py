@@ -4,8 +4,8 @@ pa_decode_no_alloc serves callers that can't allocate device memory (a
 plug-in inside an engine that owns every allocation, a runtime that forbids
 cudaMalloc after start-up): it runs the same decode kernels on a static
 device scratch array inside the library instead of a caller workspace.  This
-file is collected last so that a run stopping at its first failure has
-already run every other test; it also passes alone in a fresh process.
+file is collected after the parity suites, so that a run stopping at its
+first failure has already run them; it also passes alone in a fresh process.
 """
 
 import numpy as np

@@ -1,0 +1,91 @@
+"""Full-size parity of the decode workloads over e4m3 pools (scale 1/56):
+the Llama-3-8B batch (64 requests of 512-8192 tokens) and the long-context
+split-KV batch (32K, 64K, 96K and 128K tokens), drawn and launched as the
+benchmark draws and launches them.
+
+Checked against the oracle, through the same step the benchmark times:
+  * the slot of every new token, bit for bit;
+  * the codes of every written row, bit for bit against the oracle's
+    quantisation of the new K/V rows;
+  * a sample of unwritten rows, unchanged;
+  * attention on sampled requests, against the fp64 oracle over the pools'
+    dequantised values, within the bf16-input tolerance.
+
+This file is collected after every other GPU test.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_434_b200 as P
+from paged_kv_cache_434_b200 import workloads as W
+from _util import assert_close, f64, oracle_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def _dequantised_blocks(w, pool_u8, seqs, table):
+    """The blocks each request of `seqs` uses, as the float64 values their
+    codes stand for (`table` holds the oracle's value of each of the 256 codes)."""
+    out = {}
+    for b in seqs:
+        n = (int(w.seq_lens[b]) + w.block_size - 1) // w.block_size
+        ids = torch.from_numpy(w.block_tables[b, :n].astype(np.int64)).to(pool_u8[0].device)
+        out[int(b)] = tuple(table[p.index_select(0, ids).cpu().numpy()] for p in pool_u8)
+    return out
+
+
+def _full_size_fp8(w, dev, sample_rows):
+    assert w.kv_dtype == "fp8"
+    t = W.make_tensors(w, dev, where="device")
+    idx = W.index_tensors(w, dev)
+    Hkv, D = w.num_kv_heads, w.head_dim
+    kc = t["k_cache"].view(torch.uint8)
+    vc = t["v_cache"].view(torch.uint8)
+    table = oracle.dequantize(np.arange(256, dtype=np.uint8), w.kv_scale)
+    owners = sorted(set(np.searchsorted(w.query_start_loc, sample_rows, side="right") - 1))
+    blocks = _dequantised_blocks(w, (kc, vc), owners, table)
+    # untouched-row sample, taken before the step
+    gen = np.random.default_rng(99)
+    probe = torch.from_numpy(gen.integers(0, w.num_blocks * w.block_size, 4096)).to(dev)
+    kc_rows = kc.view(-1, Hkv, D)
+    vc_rows = vc.view(-1, Hkv, D)
+    before = kc_rows.index_select(0, probe).clone()
+
+    err = P.new_error_word(dev)
+    slots = torch.empty(w.num_tokens, dtype=torch.int64, device=dev)
+    out = P.step(t["q"], t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], idx["block_tables"],
+                 idx["query_start_loc"], idx["seq_lens"], w.scale, decode_only=w.is_decode,
+                 out_dtype=torch.float32, slots=slots, err=err, kv_scales=w.kv_scales)
+    torch.cuda.synchronize()
+    assert P.read_error(err) == 0
+
+    ref_slots = oracle.slot_mapping(w.block_tables, w.query_start_loc, w.seq_lens, w.block_size)
+    assert np.array_equal(slots.cpu().numpy(), ref_slots)
+    k_codes = oracle.quantize(f64(t["k_new"]).astype(np.float32), w.kv_scale)
+    v_codes = oracle.quantize(f64(t["v_new"]).astype(np.float32), w.kv_scale)
+    assert np.array_equal(kc_rows.index_select(0, slots).cpu().numpy(), k_codes)
+    assert np.array_equal(vc_rows.index_select(0, slots).cpu().numpy(), v_codes)
+    written = set(ref_slots.tolist())
+    keep = torch.tensor([i for i, s in enumerate(probe.tolist()) if s not in written], device=dev)
+    assert torch.equal(kc_rows.index_select(0, probe)[keep], before[keep])
+
+    # the new rows enter attention as the values of their codes
+    k_new = torch.from_numpy(table[k_codes])
+    v_new = torch.from_numpy(table[v_codes])
+    ref = oracle_rows(w, blocks, k_new, v_new, t["q"].cpu(), sample_rows)
+    got = f64(out[torch.tensor(sample_rows, device=dev)])
+    return assert_close(got, np.stack([ref[r] for r in sample_rows]), "bf16", w.name)
+
+
+def test_full_llama8b_decode_fp8(cuda_device):
+    w = W.llama8b_decode_fp8(0)
+    rows = sorted({0, 1, int(np.argmax(w.seq_lens)), int(np.argmin(w.seq_lens)), 63})
+    _full_size_fp8(w, cuda_device, rows)
+
+
+def test_full_long_context_fp8(cuda_device):
+    # the shortest (32K) and the longest (128K) request
+    _full_size_fp8(W.long_context_decode_fp8(0), cuda_device, [0, 3])
