@@ -228,7 +228,9 @@ pa_status pa_rope_cache_write(const void* q_in, const void* k, const void* v, in
                               int32_t num_heads, const pa_cache_desc* cache, int32_t* err_word,
                               void* stream);
 
-/* Bytes of workspace pa_decode needs for these sizes (0 on bad arguments). */
+/* Bytes of workspace pa_decode needs for these sizes; 0 on bad arguments and
+ * for sizes whose workspace would exceed 2^46 bytes (pa_decode then returns
+ * PA_ERR_UNSUPPORTED). */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads,
                                 int32_t max_blocks_per_seq, const pa_cache_desc* cache);
 
@@ -254,7 +256,8 @@ pa_status pa_decode(const void* q, const void* key_cache, const void* value_cach
                     int32_t out_dtype, const pa_cache_desc* cache, void* workspace,
                     size_t workspace_bytes, int32_t* err_word, void* stream);
 
-/* Bytes of workspace pa_mixed_step needs (0 on bad arguments). */
+/* Bytes of workspace pa_mixed_step needs; 0 on bad arguments and beyond
+ * 2^46 bytes, as for pa_decode_workspace_size. */
 size_t pa_mixed_step_workspace_size(int32_t num_seqs, int64_t num_tokens, int32_t num_heads,
                                     int32_t max_blocks_per_seq, const pa_cache_desc* cache);
 

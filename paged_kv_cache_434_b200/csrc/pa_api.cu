@@ -3,6 +3,7 @@
 // Host side only: validates arguments, sizes and carves the workspace, picks the
 // kernel path and enqueues the launches.  No allocation, no host<->device
 // synchronisation except in pa_read_error.
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -44,9 +45,14 @@ static int elt_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
 // bytes of one pool entry
 static int pool_elt_bytes(int dtype) { return dtype == PA_F32 ? 4 : dtype == PA_BF16 ? 2 : 1; }
 
+// Largest workspace the library plans for: far beyond any device's memory,
+// and small enough that none of the size terms of ws_layout can wrap.
+constexpr double kMaxWorkspaceBytes = 70368744177664.0;  // 2^46
+
 // Launch plan of one attention call (decode or mixed step); identical in the
 // workspace-size query and in the call itself.
 struct AttnPlan {
+  bool size_ok;      // the workspace stays within kMaxWorkspaceBytes
   bool use_mma;
   bool use_tc;       // tcgen05 tiles: prefill requests, or a decode batch's shared prefix
   bool cascade;      // decode: shared-prefix tiles + suffix partitions
@@ -95,10 +101,22 @@ static AttnPlan make_plan(int64_t num_qrows, int num_heads, int max_blocks,
   p.use_tc = (mixed && tc_ok) || p.cascade;
   p.max_parts = mp + (p.cascade ? kMaxPrefixChunks : 0);  // shared-prefix chunks
   p.tile_tokens = p.use_tc ? tc_tokens_per_tile(probe) : 0;
-  p.max_tiles = p.use_tc ? ((num_qrows + p.tile_tokens - 1) / p.tile_tokens + num_seqs) *
-                               static_cast<int64_t>(c->num_kv_heads) *
-                               (p.cascade ? kMaxPrefixChunks : 1)
-                         : 0;
+  // ws_layout's terms in double first: arguments whose exact workspace would
+  // not fit a size_t are refused instead of getting a wrapped, too small size
+  const double rows = static_cast<double>(num_qrows), parts = static_cast<double>(p.max_parts);
+  const double tiles =
+      p.use_tc ? (std::ceil(rows / p.tile_tokens) + num_seqs) * c->num_kv_heads *
+                     (p.cascade ? kMaxPrefixChunks : 1)
+               : 0.0;
+  const double bytes = 64.0 * 4 + rows * (16 + 3 * 4) + rows * p.head_groups * parts * 16 +
+                       rows * num_heads * parts * (8 + 4.0 * c->head_dim) + tiles * 16 +
+                       9 * 256;
+  p.size_ok = bytes <= kMaxWorkspaceBytes;
+  p.max_tiles = (p.use_tc && p.size_ok)
+                    ? ((num_qrows + p.tile_tokens - 1) / p.tile_tokens + num_seqs) *
+                          static_cast<int64_t>(c->num_kv_heads) *
+                          (p.cascade ? kMaxPrefixChunks : 1)
+                    : 0;
   return p;
 }
 
@@ -291,6 +309,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t max
   if (check_attn_args(num_seqs, num_seqs, num_heads, max_blocks_per_seq, PA_F32, cache) != PA_OK)
     return 0;
   const AttnPlan p = make_plan(num_seqs, num_heads, max_blocks_per_seq, cache, true);
+  if (!p.size_ok) return 0;
   return ws_layout(p.num_qrows, num_heads, cache->head_dim, p.head_groups, p.max_parts,
                    p.max_tiles)
       .total;
@@ -310,6 +329,7 @@ pa_status pa_decode(const void* q, const void* key_cache, const void* value_cach
   if (!aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
     return PA_ERR_INVALID_ARG;
   const AttnPlan p = make_plan(num_seqs, num_heads, max_blocks_per_seq, cache, true);
+  if (!p.size_ok) return PA_ERR_UNSUPPORTED;
   const AttnGeom g = make_geom(q, key_cache, value_cache, block_tables, seq_lens, nullptr, scale,
                                out, num_seqs, num_seqs, num_heads, max_blocks_per_seq, out_dtype,
                                cache, err_word);
@@ -323,6 +343,7 @@ size_t pa_mixed_step_workspace_size(int32_t num_seqs, int64_t num_tokens, int32_
     return 0;
   const AttnPlan p =
       make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true, num_seqs, true);
+  if (!p.size_ok) return 0;
   return ws_layout(p.num_qrows, num_heads, cache->head_dim, p.head_groups, p.max_parts,
                    p.max_tiles)
       .total;
@@ -344,6 +365,7 @@ pa_status pa_mixed_step(const void* q, const void* key_cache, const void* value_
     return PA_ERR_INVALID_ARG;
   const AttnPlan p =
       make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true, num_seqs, true);
+  if (!p.size_ok) return PA_ERR_UNSUPPORTED;
   const AttnGeom g = make_geom(q, key_cache, value_cache, block_tables, seq_lens,
                                query_start_loc, scale, out, num_seqs, num_tokens, num_heads,
                                max_blocks_per_seq, out_dtype, cache, err_word);

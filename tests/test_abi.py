@@ -117,6 +117,21 @@ def test_workspace_sizes_are_positive_and_monotone(lib):
     assert m > 0
 
 
+def test_workspace_beyond_any_device_is_refused(lib):
+    """Arguments whose exact workspace would not fit a size_t (2^26 KV heads,
+    2^30 requests) get size 0 and PA_ERR_UNSUPPORTED, never a wrapped size."""
+    from paged_kv_cache_434_b200 import binding as B
+    for hkv, seqs in ((1 << 26, 1 << 30), (1 << 29, 1 << 30), (1 << 30, 1 << 20)):
+        d = _desc(num_blocks=1 << 20, num_kv_heads=hkv, head_dim=128, dtype=1)
+        assert lib.pa_decode_workspace_size(seqs, hkv, 4, ctypes.byref(d)) == 0
+        assert lib.pa_mixed_step_workspace_size(seqs, seqs, hkv, 4, ctypes.byref(d)) == 0
+        assert lib.pa_decode(16, 16, 16, 16, 16, 0.1, 16, seqs, hkv, 4, 0, ctypes.byref(d), 256,
+                             1 << 62, None, None) == B.PA_ERR_UNSUPPORTED
+        assert lib.pa_mixed_step(16, 16, 16, 16, 16, 16, 0.1, 16, seqs, seqs, hkv, 4, 0,
+                                 ctypes.byref(d), 256, 1 << 62, None, None) == \
+            B.PA_ERR_UNSUPPORTED
+
+
 def test_slot_mapping_validation(lib):
     from paged_kv_cache_434_b200 import binding as B
     assert lib.pa_slot_mapping(None, 3, None, None, 2, 5, 16, 16, None, None, None) == \
