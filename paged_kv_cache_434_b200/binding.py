@@ -133,6 +133,21 @@ def _cuda(t: torch.Tensor, name: str, dtype=None, ndim=None) -> int:
     return t.data_ptr()
 
 
+def _entries(t, name: str, count: int, ndim: int = 1):
+    """The library reads `count` rows of `t` through a raw pointer: refuse a
+    tensor with fewer, which would be read past its end on the device."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dim() != ndim or t.shape[0] < count:
+        raise ValueError(f"{name} must be a {ndim}-D tensor with at least {count} rows, "
+                         f"got shape {tuple(t.shape)}")
+
+
+def _out_shape(out, shape):
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"out must have shape {tuple(shape)}, got {tuple(out.shape)}")
+
+
 def _stream() -> int:
     return torch.cuda.current_stream().cuda_stream
 
@@ -201,8 +216,11 @@ def slot_mapping(block_tables, query_start_loc, seq_lens, block_size: int, num_b
                  num_tokens: int, out=None, err=None):
     """int64 slot of every new token (see pa_slot_mapping)."""
     B, W = block_tables.shape
+    _entries(query_start_loc, "query_start_loc", B + 1)
+    _entries(seq_lens, "seq_lens", B)
     if out is None:
         out = torch.empty(num_tokens, dtype=torch.int64, device=block_tables.device)
+    _entries(out, "slot_mapping", num_tokens)
     _check(_lib().pa_slot_mapping(
         _cuda(block_tables, "block_tables", torch.int32, 2), W,
         _cuda(query_start_loc, "query_start_loc", torch.int32, 1),
@@ -254,6 +272,7 @@ def slot_mapping_positions(block_tables, token_req, positions, block_size: int, 
         raise ValueError("token_req and positions must have one entry per token")
     if out is None:
         out = torch.empty(T, dtype=torch.int64, device=positions.device)
+    _entries(out, "out", T)
     _check(_lib().pa_slot_mapping_positions(
         _cuda(block_tables, "block_tables", torch.int32, 2), W, B,
         _cuda(token_req, "token_req", torch.int32, 1), _cuda(positions, "positions", torch.int64, 1),
@@ -297,6 +316,8 @@ def rope_cache_write(q, k, v, k_cache, v_cache, slot_mapping, positions, cos_sin
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != k_cache.dtype or t.shape[0] != T:
             raise ValueError(f"{name} must have num_tokens rows of the cache dtype")
+    _entries(slot_mapping, "slot_mapping", T)
+    _entries(positions, "positions", T)
     qs = _token_rows(q, "q", Hq, D)
     ks = _token_rows(k, "k", desc.num_kv_heads, desc.head_dim)
     if _token_rows(v, "v", desc.num_kv_heads, desc.head_dim) != ks:
@@ -336,8 +357,12 @@ def _workspace(nbytes, device, workspace):
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
-def _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales=None):
+def _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales=None,
+                num_seqs=None):
     desc = cache_desc(k_cache, kv_scales)
+    if num_seqs is not None:
+        _entries(block_tables, "block_tables", num_seqs, ndim=2)
+        _entries(seq_lens, "seq_lens", num_seqs)
     if q.dtype != io_dtype(k_cache) or q.dim() != 3 or q.shape[2] != desc.head_dim:
         raise ValueError("q must be [rows, num_heads, head_dim] of the cache's input dtype")
     if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
@@ -350,11 +375,13 @@ def _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scale
 def decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=None,
            out_dtype=torch.float32, workspace=None, err=None, kv_scales=None):
     """Decode attention: out[b, h] over the first seq_lens[b] keys of request b."""
-    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales)
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales,
+                       num_seqs=q.shape[0] if q.dim() == 3 else None)
     B, H, D = q.shape
     W = block_tables.shape[1]
     if out is None:
         out = torch.empty(B, H, D, dtype=out_dtype, device=q.device)
+    _out_shape(out, (B, H, D))
     nbytes = decode_workspace_size(B, H, W, k_cache)
     ws = _workspace(nbytes, q.device, workspace)
     _check(_lib().pa_decode(
@@ -369,11 +396,14 @@ def decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=None,
 def mixed_step(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, scale: float,
                out=None, out_dtype=torch.float32, workspace=None, err=None, kv_scales=None):
     """Causal varlen attention of a flattened step (chunked prefill + decode)."""
-    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales)
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales,
+                       num_seqs=block_tables.shape[0] if block_tables.dim() == 2 else None)
     T, H, D = q.shape
     B, W = block_tables.shape
+    _entries(query_start_loc, "query_start_loc", B + 1)
     if out is None:
         out = torch.empty(T, H, D, dtype=out_dtype, device=q.device)
+    _out_shape(out, (T, H, D))
     nbytes = mixed_step_workspace_size(B, T, H, W, k_cache)
     ws = _workspace(nbytes, q.device, workspace)
     _check(_lib().pa_mixed_step(
@@ -397,9 +427,11 @@ def decode_no_alloc(q, k_cache, v_cache, block_tables, seq_lens, scale: float, o
     `out` must be given, so that this call allocates nothing either.  Calls
     whose kernels overlap on the GPU share the scratch and race.
     """
-    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out.dtype, kv_scales)
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out.dtype, kv_scales,
+                       num_seqs=q.shape[0] if q.dim() == 3 else None)
     B, H, D = q.shape
     W = block_tables.shape[1]
+    _out_shape(out, (B, H, D))
     _check(_lib().pa_decode_no_alloc(
         _cuda(q, "q"), _cuda(k_cache, "k_cache"), _cuda(v_cache, "v_cache"),
         _cuda(block_tables, "block_tables", torch.int32, 2),

@@ -214,3 +214,45 @@ def test_block_management_validation(lib):
         B.PA_OK
     assert lib.pa_slot_mapping_positions(16, 4, 2, 16, 16, 5, 0, 16, 16, None, None) == \
         B.PA_ERR_INVALID_ARG                                 # block size 0
+
+
+def test_binding_refuses_arrays_the_library_would_overrun():
+    """The library reads num_seqs rows of block_tables / seq_lens (num_seqs + 1
+    of query_start_loc) and writes exactly [rows, Hq, D] through raw pointers:
+    the binding refuses shorter arrays and mis-shaped outputs before any call
+    (CPU tensors here, so nothing reaches a device)."""
+    import torch
+    import paged_kv_cache_434_b200 as P
+    from paged_kv_cache_434_b200 import binding as B
+    kc = torch.zeros(4, 16, 2, 64)
+    q = torch.zeros(2, 8, 64)
+    i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)  # noqa: E731
+    cases = [
+        (lambda: P.decode(q, kc, kc, i32(1, 3), i32(2), 0.1), "block_tables"),
+        (lambda: P.decode(q, kc, kc, i32(2, 3), i32(1), 0.1), "seq_lens"),
+        (lambda: P.decode(q, kc, kc, i32(2, 3), i32(2), 0.1, out=torch.zeros(2, 8, 32)), "out"),
+        (lambda: P.mixed_step(q, kc, kc, i32(2, 3), i32(2), i32(2), 0.1), "query_start_loc"),
+        (lambda: P.mixed_step(q, kc, kc, i32(2, 3), i32(3), i32(1), 0.1), "seq_lens"),
+        (lambda: P.mixed_step(q, kc, kc, i32(2, 3), i32(3), i32(2), 0.1,
+                              out=torch.zeros(1, 8, 64)), "out"),
+        (lambda: B.decode_no_alloc(q, kc, kc, i32(2, 3), i32(2), 0.1, torch.zeros(3, 8, 64)),
+         "out"),
+        (lambda: P.slot_mapping(i32(2, 3), i32(2), i32(2), 16, 4, 5), "query_start_loc"),
+        (lambda: P.slot_mapping(i32(2, 3), i32(3), i32(1), 16, 4, 5), "seq_lens"),
+        (lambda: P.slot_mapping(i32(2, 3), i32(3), i32(2), 16, 4, 5,
+                                out=torch.zeros(4, dtype=torch.int64)), "slot_mapping"),
+        (lambda: P.slot_mapping_positions(i32(2, 3), i32(5), torch.zeros(5, dtype=torch.int64),
+                                          16, 4, out=torch.zeros(4, dtype=torch.int64)), "out"),
+        (lambda: P.rope_cache_write(q, torch.zeros(2, 2, 64), torch.zeros(2, 2, 64), kc, kc,
+                                    torch.zeros(1, dtype=torch.int64),
+                                    torch.zeros(2, dtype=torch.int64), torch.zeros(8, 64)),
+         "slot_mapping"),
+        (lambda: P.rope_cache_write(q, torch.zeros(2, 2, 64), torch.zeros(2, 2, 64), kc, kc,
+                                    torch.zeros(2, dtype=torch.int64),
+                                    torch.zeros(1, dtype=torch.int64), torch.zeros(8, 64)),
+         "positions"),
+    ]
+    for call, name in cases:
+        with pytest.raises(ValueError, match=rf"^{name} must (be a \d-D tensor with at least|"
+                                             rf"have shape)"):
+            call()
