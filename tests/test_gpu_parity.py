@@ -3,8 +3,6 @@ same seeded inputs.  Cache writes and slots are compared bit for bit;
 attention within max-abs 1e-5 (fp32) or max-abs 1e-2 / mean-abs 1e-3 (bf16
 inputs, fp32 accumulation)."""
 
-import math
-
 import numpy as np
 import pytest
 import torch
