@@ -774,7 +774,6 @@ __device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView&
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       ck[u] = __shfl_sync(0xffffffffu, c, k + u);
-#pragma unroll
       if constexpr (V == 4) {  // one 16-byte load per partition
         const float4 t4 = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(k + u) * D);
         x[u][0] = t4.x, x[u][1] = t4.y, x[u][2] = t4.z, x[u][3] = t4.w;
