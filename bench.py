@@ -557,7 +557,7 @@ def run_ours(args, rank, world, local):
             "ms_per_step_p10_p50_p90": [round(float(x), 4) for x in
                                         np.percentile(step_ms, [10, 50, 90])],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.dtype,
+            "dtype": ("e4m3 pools, f16 tensor-core products" if w.kv_dtype == "fp8" else w.dtype),
             "data": "synthetic: seeded N(0,1) Q/K/V rounded to the dtype, seeded lengths and "
                     "randomly permuted physical blocks",
             "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_tokens": T,
