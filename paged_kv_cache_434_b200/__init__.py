@@ -21,6 +21,7 @@ from .binding import (  # noqa: F401
     ERRBIT_SEQ_TOO_LONG,
     ERRBIT_SLOT_OOB,
     ERRBIT_POS_OOB,
+    ERRBIT_Q_RANGE,
     ERRBIT_TIMEOUT,
     PagedAttentionError,
     cache_write,

@@ -25,6 +25,7 @@ ERRBIT_SEQ_TOO_LONG = 0x4
 ERRBIT_QUERY_TOO_LONG = 0x8
 ERRBIT_TIMEOUT = 0x10
 ERRBIT_POS_OOB = 0x20
+ERRBIT_Q_RANGE = 0x40
 
 EXPORTS = ("pa_status_str", "pa_version", "pa_slot_mapping", "pa_cache_write",
            "pa_decode_workspace_size", "pa_decode", "pa_mixed_step_workspace_size",

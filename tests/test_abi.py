@@ -256,3 +256,66 @@ def test_binding_refuses_arrays_the_library_would_overrun():
         with pytest.raises(ValueError, match=rf"^{name} must (be a \d-D tensor with at least|"
                                              rf"have shape)"):
             call()
+
+
+def _header_text():
+    return re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+
+
+def test_binding_constants_match_the_header():
+    from paged_kv_cache_434_b200 import binding as B
+    text = _header_text()
+    enums = dict((k, int(v)) for k, v in re.findall(r"\b(PA_[A-Z0-9_]+)\s*=\s*(\d+)", text))
+    for name in ("PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
+                 "PA_ERR_CUDA", "PA_ERR_DEVICE", "PA_F32", "PA_BF16", "PA_FP8_E4M3"):
+        assert getattr(B, name) == enums[name], name
+    defines = dict(re.findall(r"#define\s+(PA_[A-Z0-9_]+)\s+\(?([0-9a-fx]+)", text))
+    bits = {k: int(v, 0) for k, v in defines.items() if k.startswith("PA_ERRBIT_")}
+    assert bits and all(getattr(B, k[3:]) == v for k, v in bits.items()), bits
+    assert B.DECODE_NO_ALLOC_MAX_BYTES == 32 << 20
+    assert "(32u << 20)" in text.split("PA_DECODE_NO_ALLOC_MAX_BYTES", 1)[1].splitlines()[0]
+    assert len(B.TIMED_KERNELS) == int(defines["PA_TIMED_KERNELS"])
+    for i, name in enumerate(B.TIMED_KERNELS):
+        assert int(defines[f"PA_TK_{name.upper()}"]) == i
+
+
+_CTYPES_OF = {"int32_t": "c_int", "int64_t": "c_long", "float": "c_float", "double": "c_double",
+              "size_t": "c_ulong", "int": "c_int"}
+
+
+def _kind(ctype):
+    """Comparable name of a ctypes argument type."""
+    import ctypes
+    if ctype is ctypes.c_void_p:
+        return "ptr"
+    if isinstance(ctype, type) and issubclass(ctype, ctypes._Pointer):
+        from paged_kv_cache_434_b200.binding import CacheDesc
+        return "desc_ptr" if ctype._type_ is CacheDesc else "ptr"
+    if ctype is ctypes.c_char_p:
+        return "str"
+    return ctype.__name__
+
+
+def test_binding_signatures_match_the_header():
+    """Argument count and kind of every ctypes prototype against the C
+    prototype in include/pa.h (pointers, 32/64-bit integers, floats)."""
+    import ctypes
+    from paged_kv_cache_434_b200 import binding as B
+    text = _header_text()
+    protos = dict(re.findall(r"\b(?:pa_status|size_t|int|const char\*)\s+(pa_[a-z_]+)\(([^)]*)\)",
+                             text, flags=re.S))
+    assert set(protos) == set(B.EXPORTS)
+    for name, params in protos.items():
+        want = []
+        for p in filter(None, (x.strip() for x in params.split(","))):
+            if p == "void":
+                continue
+            if "pa_cache_desc" in p and "*" in p:
+                want.append("desc_ptr")
+            elif "*" in p:
+                want.append("ptr")
+            else:
+                base = p.rsplit(None, 1)[0].replace("const ", "").strip()
+                want.append(getattr(ctypes, _CTYPES_OF[base]).__name__)
+        got = [_kind(t) for t in B._SIGNATURES[name][0]]
+        assert got == want, (name, got, want)
