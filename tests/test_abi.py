@@ -319,3 +319,27 @@ def test_binding_signatures_match_the_header():
                 want.append(getattr(ctypes, _CTYPES_OF[base]).__name__)
         got = [_kind(t) for t in B._SIGNATURES[name][0]]
         assert got == want, (name, got, want)
+
+
+def test_cache_desc_layout_matches_the_c_struct(tmp_path):
+    """Size and field offsets of pa_cache_desc as gcc lays it out, against the
+    ctypes structure the binding passes by pointer."""
+    import ctypes
+    import shutil
+    import subprocess
+    from paged_kv_cache_434_b200.binding import CacheDesc
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    names = [n for n, _ in CacheDesc._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"pa.h\"\nint main(void) {\n"
+                   "  printf(\"%zu\\n\", sizeof(pa_cache_desc));\n" +
+                   "".join(f"  printf(\"%zu\\n\", offsetof(pa_cache_desc, {n}));\n" for n in names) +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(CacheDesc)
+    assert got[1:] == [getattr(CacheDesc, n).offset for n in names]
