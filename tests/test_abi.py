@@ -343,3 +343,40 @@ def test_cache_desc_layout_matches_the_c_struct(tmp_path):
                                           check=True).stdout.split()]
     assert got[0] == ctypes.sizeof(CacheDesc)
     assert got[1:] == [getattr(CacheDesc, n).offset for n in names]
+
+
+def test_plain_c_program_links_and_calls_the_library(tmp_path, lib):
+    """The boundary is usable from C alone: a C99 program including only
+    include/pa.h links libpa_b200.so and gets the documented statuses from
+    calls that are refused on the host (nothing reaches a device)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    libdir = os.path.join(ROOT, "paged_kv_cache_434_b200", "lib")
+    src = tmp_path / "client.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "pa.h"
+int main(void) {
+  pa_cache_desc d = {16, 16, 2, 64, PA_BF16, 1.0f, 1.0f};
+  pa_cache_desc bad = d;
+  bad.head_dim = 96;
+  printf("%d\n", pa_version() >= 100);
+  printf("%s\n", pa_status_str(PA_ERR_WORKSPACE));
+  printf("%d\n", pa_decode_workspace_size(4, 8, 3, &d) > 0);
+  printf("%d\n", (int)pa_cache_write(NULL, NULL, NULL, NULL, NULL, 4, &d, NULL, NULL));
+  printf("%d\n", (int)pa_cache_write(NULL, NULL, NULL, NULL, NULL, 1, &bad, NULL, NULL));
+  printf("%d\n", (int)pa_decode(NULL, NULL, NULL, NULL, NULL, 0.1f, NULL, 0, 8, 3, PA_F32, &d,
+                                NULL, 0, NULL, NULL));
+  return 0;
+}
+''')
+    exe = tmp_path / "client"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir,
+                    "-lpa_b200", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    assert out[0] == "1"
+    assert out[1] == "workspace missing, misaligned or too small"
+    assert out[2] == "1"
+    assert out[3:6] == ["1", "2", "0"]   # INVALID_ARG, UNSUPPORTED, OK (nothing to do)
