@@ -1,0 +1,87 @@
+"""Block sizes 64, 128 and 256, which the library accepts beside 8, 16 and 32:
+decode and mixed steps on every kernel path (fp32 generic kernel, bf16
+mma.sync partitions and tensor-core prefill tiles, e4m3 pools, the
+shared-prefix cascade) against the fp64 oracle.  A 16-key stage then covers
+part of one block, and a request's last block is mostly empty.
+
+This file is collected after every other GPU test.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_434_b200 as P
+from paged_kv_cache_434_b200 import workloads as W
+from _util import assert_close, bits, f64, fp8_codes, oracle_full, oracle_full_fp8
+
+pytestmark = pytest.mark.gpu
+
+BLOCK_SIZES = [64, 128, 256]
+
+
+def _run_and_check(w, dev):
+    host = W.make_tensors(w, "cpu", where="host")
+    t = {k: v.to(dev) for k, v in host.items()}
+    idx = W.index_tensors(w, dev)
+    err = P.new_error_word(dev)
+    slots = torch.empty(w.num_tokens, dtype=torch.int64, device=dev)
+    out = P.step(t["q"], t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], idx["block_tables"],
+                 idx["query_start_loc"], idx["seq_lens"], w.scale, decode_only=w.is_decode,
+                 slots=slots, err=err, kv_scales=w.kv_scales)
+    torch.cuda.synchronize()
+    assert P.read_error(err) == 0
+    if w.kv_dtype == "fp8":
+        ref_slots, kb, vb, ref, ref_err, valid = oracle_full_fp8(w, host)
+        assert np.array_equal(fp8_codes(t["k_cache"]), kb)
+        assert np.array_equal(fp8_codes(t["v_cache"]), vb)
+    else:
+        ref_slots, kb, vb, ref, ref_err, valid = oracle_full(w, host)
+        assert np.array_equal(bits(t["k_cache"]), kb) and np.array_equal(bits(t["v_cache"]), vb)
+    assert ref_err == set()
+    assert np.array_equal(slots.cpu().numpy(), ref_slots)
+    assert_close(f64(out)[valid], ref[valid], "f32" if w.dtype == "f32" else "bf16", w.name)
+
+
+def _lens(bs, rng):
+    # 1 key, a partial first block, exactly one block, one key more, several blocks
+    return [1, bs // 2 + 3, bs, bs + 1, 3 * bs + 17] + rng.integers(1, 1500, 3).tolist()
+
+
+@pytest.mark.parametrize("bs", BLOCK_SIZES)
+@pytest.mark.parametrize("dtype,hq,hkv,d", [("f32", 8, 2, 64), ("bf16", 32, 8, 128),
+                                            ("bf16", 8, 2, 64)])
+def test_decode_large_blocks(cuda_device, bs, dtype, hq, hkv, d):
+    rng = np.random.default_rng([bs, hq, d])
+    lens = _lens(bs, rng)
+    w = W.custom(f"decode_bs{bs}_{dtype}_{d}", lens, [1] * len(lens), hq, hkv, d, bs, dtype,
+                 seed=bs + d, extra_blocks=2)
+    _run_and_check(w, cuda_device)
+
+
+@pytest.mark.parametrize("bs", BLOCK_SIZES)
+@pytest.mark.parametrize("dtype,hq,hkv,d", [("f32", 8, 2, 64), ("bf16", 32, 8, 128),
+                                            ("bf16", 16, 2, 64)])
+def test_mixed_step_large_blocks(cuda_device, bs, dtype, hq, hkv, d):
+    # a chunk after a cached prefix, a fresh prompt, decodes
+    lens = [bs + 200, 130, 1, 2 * bs + 5, 700]
+    qlens = [150, 130, 1, 1, 1]
+    w = W.custom(f"mixed_bs{bs}_{dtype}_{d}", lens, qlens, hq, hkv, d, bs, dtype,
+                 seed=bs + d + 1)
+    _run_and_check(w, cuda_device)
+
+
+@pytest.mark.parametrize("bs", BLOCK_SIZES)
+def test_fp8_decode_large_blocks(cuda_device, bs):
+    rng = np.random.default_rng([bs, 8])
+    lens = _lens(bs, rng)
+    w = W.with_fp8_cache(W.custom(f"fp8_bs{bs}", lens, [1] * len(lens), 32, 8, 128, bs, "bf16",
+                                  seed=bs + 3))
+    _run_and_check(w, cuda_device)
+
+
+@pytest.mark.parametrize("bs", BLOCK_SIZES)
+def test_shared_prefix_large_blocks(cuda_device, bs):
+    # 24 requests whose tables start with the same 1024 tokens of blocks
+    w = W.shared_prefix_decode(bs, num_seqs=24, prefix_tokens=1024, block_size=bs)
+    _run_and_check(w, cuda_device)
