@@ -11,7 +11,7 @@ Checked against the oracle, through the same step the benchmark times:
   * attention on sampled requests, against the fp64 oracle over the pools'
     dequantised values, within the bf16-input tolerance.
 
-This file is collected after every other GPU test.
+This file is collected after the parity suites.
 """
 
 import numpy as np
