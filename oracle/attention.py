@@ -107,7 +107,11 @@ def cache_write(k_cache, v_cache, k, v, slots):
 # --------------------------------------------------------------------------
 
 def gather(cache, block_table_row, length: int):
-    """Logical K (or V) of one request: row p is cache[table[p // bs], p % bs]."""
+    """Logical K (or V) of one request: row p is cache[table[p // bs], p % bs].
+
+    Source: "AI Infra入门干货总结：大模型是如何高效推理的", "Paged Attention" (the block table maps a logical block to
+    its physical block; the offset inside the block is p % block_size).
+    """
     block_size = cache.shape[1]
     rows = [cache[int(block_table_row[p // block_size]), p % block_size]
             for p in range(length)]
@@ -144,6 +148,9 @@ def attend_two_pass(q, K, V, scale: float, first_pos: int):
     q: [n_q, num_heads, D]; K, V: [L, num_kv_heads, D]; returns [n_q, num_heads, D].
     Pass 1 takes m = max_j s_ij; pass 2 forms w_ij = exp(s_ij - m_i),
     l_i = sum_j w_ij and o_i = sum_j w_ij v_j / l_i.
+
+    Source: "AI Infra入门干货总结：大模型是如何高效推理的", "Attention (FlashAttention, Scaled Dot-Product Attention)"
+    (its table of steps: GQA head map, Q K^T, scale, mask, softmax, P V).
     """
     q = np.asarray(q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
@@ -205,6 +212,9 @@ def attend_partial(q, K, V, scale: float, first_pos: int, key_lo: int, key_hi: i
 
     m[i, h] = max of the allowed scores in the range (-inf if none),
     l[i, h] = sum exp(s - m), o[i, h] = sum exp(s - m) v.
+
+    Source: "AI Infra入门干货总结：大模型是如何高效推理的", "总结" (Flash-Decoding splits the key axis across SMs);
+    "第三部分 · 推理系统与基础设施", chapter map 3.4.
     """
     q = np.asarray(q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
@@ -234,6 +244,9 @@ def merge_partials(parts):
     With M = max_k m_k and weights c_k = exp(m_k - M):
     O = sum_k c_k o_k / sum_k c_k l_k.  Partials whose m_k is -inf (no
     allowed key) have c_k = 0.
+
+    Source: "AI Infra入门干货总结：大模型是如何高效推理的", "总结" (the partial results are re-normalised with
+    log-sum-exp).
     """
     ms = np.stack([p[0] for p in parts])            # [P, n_q, H]
     ls = np.stack([p[1] for p in parts])
@@ -311,6 +324,9 @@ def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float):
 
     q: [num_seqs, num_heads, D] -> (out [num_seqs, num_heads, D], errors, valid).
     A request with L_b == 0 attends to nothing; its output row is zero.
+
+    Source: "AI Infra入门干货总结：大模型是如何高效推理的", "附2：推理运行时变量" (seq_lens counts the computed tokens
+    plus the new one, so the decode query is the last position).
     """
     lens = np.asarray(seq_lens, dtype=np.int64)
     num_seqs = len(lens)
@@ -331,5 +347,9 @@ def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float):
 
 def kv_cache_bytes(num_layers: int, num_kv_heads: int, head_dim: int,
                    bytes_per_elt: int, context_len: int) -> int:
-    """Bytes of K and V cache for one sequence: layers x 2 x heads x dim x elt x tokens."""
+    """Bytes of K and V cache for one sequence: layers x 2 x heads x dim x elt x tokens.
+
+    Source: ursb.me Field Note "llm-inference-life", blurb (Llama-3-8B holds
+    about 1 GB of KV cache at 8K context); "AI Infra入门干货总结：大模型是如何高效推理的", "附1：模型配置参数".
+    """
     return num_layers * 2 * num_kv_heads * head_dim * bytes_per_elt * context_len

@@ -35,7 +35,11 @@ ERR_POS_OOB_TABLE = "position_outside_block_table"
 def copy_blocks(k_pool, v_pool, mapping):
     """Return copies of the pools with block dst := block src for each
     (src, dst) row of mapping; pairs naming a block outside the pool are
-    reported and skipped.  Works on any dtype (bit-exact)."""
+    reported and skipped.  Works on any dtype (bit-exact).
+
+    Source: "第三部分 · 推理系统与基础设施", chapter map 3.3 (copy-on-write:
+    a request about to write into a shared block first gets its own copy).
+    """
     kp = np.array(k_pool, copy=True)
     vp = np.array(v_pool, copy=True)
     nb = kp.shape[0]

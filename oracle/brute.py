@@ -18,6 +18,9 @@ def brute_attention(q, K, V, scale, first_pos):
 
     Query i is at position first_pos + i and sees keys 0 .. first_pos + i.
     Returns nested lists [n_q][num_heads][D] of Python floats.
+
+    Source: "AI Infra入门干货总结：大模型是如何高效推理的", "Attention (FlashAttention, Scaled Dot-Product Attention)",
+    written out with loops and math.exp only.
     """
     n_q = len(q)
     num_heads = len(q[0])

@@ -28,7 +28,11 @@ E4M3_MAX = 448.0
 
 
 def e4m3_decode(codes) -> np.ndarray:
-    """float64 value of every e4m3 byte (NaN codes give NaN)."""
+    """float64 value of every e4m3 byte (NaN codes give NaN).
+
+    Source: ursb.me Field Note "llm-inference-life", blurb (fp8 e4m3); the
+    bit layout is the format reading stated in this module's header.
+    """
     c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
     sign = np.where(c & 0x80, -1.0, 1.0)
     e = (c >> 3) & 0xF
@@ -40,7 +44,11 @@ def e4m3_decode(codes) -> np.ndarray:
 
 def e4m3_encode(x) -> np.ndarray:
     """Round float64 values (exact float32 values in practice) to e4m3 codes:
-    nearest, ties to even, magnitudes above 448 saturate to 448."""
+    nearest, ties to even, magnitudes above 448 saturate to 448.
+
+    Source: as e4m3_decode; rounding and saturation are the readings stated
+    in this module's header.
+    """
     x = np.asarray(x, dtype=np.float64)
     sign = np.signbit(x)
     a = np.minimum(np.abs(x), E4M3_MAX)
@@ -63,11 +71,18 @@ def e4m3_encode(x) -> np.ndarray:
 
 def quantize(x, scale: float) -> np.ndarray:
     """Codes of x (bf16 / float32 values) for a pool with this scale: the
-    float32 quotient x / scale, then e4m3_encode."""
+    float32 quotient x / scale, then e4m3_encode.
+
+    Source: "从零构建LLM 推理引擎", card "量化" (fewer bits per KV entry); the per-pool scale is
+    the reading stated in this module's header.
+    """
     q = np.asarray(x, dtype=np.float32) / np.float32(scale)
     return e4m3_encode(q.astype(np.float64))
 
 
 def dequantize(codes, scale: float) -> np.ndarray:
-    """float64 values a pool of codes stands for."""
+    """float64 values a pool of codes stands for.
+
+    Source: "从零构建LLM 推理引擎", card "量化"; an entry stands for code * scale.
+    """
     return e4m3_decode(codes) * float(np.float32(scale))

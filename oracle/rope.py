@@ -37,19 +37,32 @@ ERR_POS_OOB = "position_out_of_range"  # position < 0 or >= max_position
 
 
 def inv_freq(rotary_dim: int, theta: float) -> np.ndarray:
-    """theta ** (-2 i / rotary_dim) for i < rotary_dim / 2, float64."""
+    """theta ** (-2 i / rotary_dim) for i < rotary_dim / 2, float64.
+
+    Source: "AI Infra入门干货总结：大模型是如何高效推理的", "附1：模型配置参数" (rope_theta); the schedule itself is the
+    reading stated in this module's header.
+    """
     i = np.arange(rotary_dim // 2, dtype=np.float64)
     return np.power(np.float64(theta), -2.0 * i / rotary_dim)
 
 
 def cos_sin_table(max_position: int, rotary_dim: int, theta: float) -> np.ndarray:
-    """[max_position, rotary_dim] float64: cos of every angle, then sin."""
+    """[max_position, rotary_dim] float64: cos of every angle, then sin.
+
+    Source: "AI Infra入门干货总结：大模型是如何高效推理的", "Reshape & Cache" (a cos_sin_cache of shape
+    [max_position, rotary_dim] indexed by position).
+    """
     ang = np.outer(np.arange(max_position, dtype=np.float64), inv_freq(rotary_dim, theta))
     return np.concatenate([np.cos(ang), np.sin(ang)], axis=1)
 
 
 def pair_index(rotary_dim: int, neox: bool):
-    """(first, second) dimension of each rotated pair i < rotary_dim / 2."""
+    """(first, second) dimension of each rotated pair i < rotary_dim / 2.
+
+    Source: ursb.me Field Note "llm-inference-life", blurb (dimensions taken
+    in pairs, each pair turned like a complex number); which dimensions form
+    a pair is the reading stated in this module's header.
+    """
     half = rotary_dim // 2
     i = np.arange(half)
     if neox:
