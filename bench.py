@@ -119,6 +119,43 @@ def max_over_ranks(x: float, world: int, dev) -> float:
     return float(t.item())
 
 
+def own_peaks(dev, copy_bytes: int = 1 << 30, gemm_n: int = 8192, iters: int = 10):
+    """This process's own reference rates, reported as context beside the
+    measured peaks: a device-to-device copy (read + write bytes over time) and
+    a bf16 torch matmul (2 n^3 FLOP), each timed with CUDA events after three
+    warm-up runs.  Never raises: a failure is reported in the result."""
+    try:
+        stream = torch.cuda.current_stream()
+        a = torch.empty(copy_bytes, dtype=torch.uint8, device=dev)
+        b = torch.empty_like(a)
+
+        def timed(fn):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(iters):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / 1e3 / iters
+
+        copy_s = timed(lambda: b.copy_(a))
+        del a, b
+        x = torch.randn(gemm_n, gemm_n, device=dev).to(torch.bfloat16)
+        y = torch.randn(gemm_n, gemm_n, device=dev).to(torch.bfloat16)
+        z = torch.empty(gemm_n, gemm_n, dtype=torch.bfloat16, device=dev)
+        gemm_s = timed(lambda: torch.matmul(x, y, out=z))
+        del x, y, z
+        return {"copy_gbs": round(2 * copy_bytes / copy_s / 1e9, 1),
+                "bf16_gemm_tflops": round(2 * gemm_n ** 3 / gemm_s / 1e12, 1),
+                "how": f"{copy_bytes >> 20} MiB device-to-device copy, {gemm_n}^3 bf16 "
+                       f"torch.matmul; CUDA events, mean of {iters} after 3 warm-up"}
+    except Exception as e:  # context only: never costs the benchmark line
+        return {"error": f"{type(e).__name__}: {e}"[:200]}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -486,6 +523,9 @@ def run_ours(args, rank, world, local):
                                    "frac": round(bc["attention"] / attn_s / 1e9 /
                                                  peaks["hbm_gbs"], 4),
                                    "bytes": bc["attention"]}}
+    own = own_peaks(dev) if world == 1 else None
+    if own is not None and "copy_gbs" in own:
+        roofline["own_peaks"] = dict(own, frac_of_own_copy=round(achieved / own["copy_gbs"], 4))
     extra = dict(extra_kv)
     prefill_roofline = None
     if args.workload in ("mixed", "mixed_prefill"):
@@ -506,6 +546,8 @@ def run_ours(args, rank, world, local):
                               f"{n_t} launches, L2 flushed before each",
                 "ms": round(tiles_ms, 4), "algorithmic_flops_per_launch": fl,
                 "traffic": kernel_traffic("attn_tc.cu", f"attn_tc_kernel_{args.workload}.md")}
+            if own is not None and "bf16_gemm_tflops" in own:
+                prefill_roofline["frac_of_own_gemm"] = round(tf / own["bf16_gemm_tflops"], 4)
 
     # ---- end to end: host buffers in, result back to the host, each step
     e2e = None
