@@ -1,8 +1,12 @@
-"""Block sizes 64, 128 and 256, which the library accepts beside 8, 16 and 32:
-decode and mixed steps on every kernel path (fp32 generic kernel, bf16
-mma.sync partitions and tensor-core prefill tiles, e4m3 pools, the
-shared-prefix cascade) against the fp64 oracle.  A 16-key stage then covers
-part of one block, and a request's last block is mostly empty.
+"""Shapes the library accepts beyond the parity suites, against the fp64 oracle:
+
+  * block sizes 64, 128 and 256 (beside 8, 16 and 32) on every kernel path:
+    fp32 generic kernel, bf16 mma.sync partitions and tensor-core prefill
+    tiles, e4m3 pools, the shared-prefix cascade.  A 16-key stage then
+    covers part of one block, and a request's last block is mostly empty;
+  * one KV head (MQA) and an odd number of KV heads, where each decode work
+    item carries a single KV head (the one-head variant of the mma.sync
+    kernel) and the tensor-core tiles take all query heads of the one group.
 
 This file is collected after every other GPU test.
 """
@@ -84,4 +88,31 @@ def test_fp8_decode_large_blocks(cuda_device, bs):
 def test_shared_prefix_large_blocks(cuda_device, bs):
     # 24 requests whose tables start with the same 1024 tokens of blocks
     w = W.shared_prefix_decode(bs, num_seqs=24, prefix_tokens=1024, block_size=bs)
+    _run_and_check(w, cuda_device)
+
+
+@pytest.mark.parametrize("dtype,hq,hkv,d", [("bf16", 8, 1, 128), ("bf16", 16, 1, 64),
+                                            ("bf16", 12, 3, 128), ("bf16", 5, 5, 64),
+                                            ("f32", 8, 1, 64)])
+def test_decode_single_kv_head_per_item(cuda_device, dtype, hq, hkv, d):
+    rng = np.random.default_rng([hq, hkv, d])
+    lens = [1, 15, 16, 17, 700, 2500] + rng.integers(1, 1200, 3).tolist()
+    w = W.custom(f"decode_mqa_{hq}_{hkv}_{d}_{dtype}", lens, [1] * len(lens), hq, hkv, d, 16,
+                 dtype, seed=hq * 7 + hkv + d, extra_blocks=2)
+    _run_and_check(w, cuda_device)
+
+
+@pytest.mark.parametrize("hq,hkv,d", [(8, 1, 128), (16, 1, 64), (12, 3, 128)])
+def test_mixed_step_single_kv_head_per_item(cuda_device, hq, hkv, d):
+    lens = [400, 130, 1, 37, 900]
+    qlens = [150, 130, 1, 1, 1]
+    w = W.custom(f"mixed_mqa_{hq}_{hkv}_{d}", lens, qlens, hq, hkv, d, 16, "bf16",
+                 seed=hq * 7 + hkv + d + 1)
+    _run_and_check(w, cuda_device)
+
+
+def test_fp8_decode_single_kv_head(cuda_device):
+    lens = [1, 16, 17, 900, 2500]
+    w = W.with_fp8_cache(W.custom("fp8_mqa", lens, [1] * len(lens), 8, 1, 128, 16, "bf16",
+                                  seed=77))
     _run_and_check(w, cuda_device)
