@@ -111,8 +111,10 @@ def test_mixed_step_single_kv_head_per_item(cuda_device, hq, hkv, d):
     _run_and_check(w, cuda_device)
 
 
-def test_fp8_decode_single_kv_head(cuda_device):
+@pytest.mark.parametrize("hq,hkv", [(8, 1), (16, 4)])
+def test_fp8_decode_head_groups(cuda_device, hq, hkv):
+    # e4m3 decode with one and with four KV heads per work item
     lens = [1, 16, 17, 900, 2500]
-    w = W.with_fp8_cache(W.custom("fp8_mqa", lens, [1] * len(lens), 8, 1, 128, 16, "bf16",
-                                  seed=77))
+    w = W.with_fp8_cache(W.custom(f"fp8_heads_{hq}_{hkv}", lens, [1] * len(lens), hq, hkv, 128,
+                                  16, "bf16", seed=77 + hkv))
     _run_and_check(w, cuda_device)
