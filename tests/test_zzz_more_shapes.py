@@ -118,3 +118,25 @@ def test_fp8_decode_head_groups(cuda_device, hq, hkv):
     w = W.with_fp8_cache(W.custom(f"fp8_heads_{hq}_{hkv}", lens, [1] * len(lens), hq, hkv, 128,
                                   16, "bf16", seed=77 + hkv))
     _run_and_check(w, cuda_device)
+
+
+def test_fp8_query_beyond_f16_range_sets_its_error_bit(cuda_device):
+    """Over e4m3 pools the tensor-core decode path takes queries as f16: a
+    query entry beyond +-65504 sets PA_ERRBIT_Q_RANGE.  The requests whose
+    queries are in range are still exact."""
+    dev = cuda_device
+    w = W.with_fp8_cache(W.custom("fp8_q_range", [40, 300, 77], [1, 1, 1], 8, 2, 128, 16, "bf16",
+                                  seed=91))
+    host = W.make_tensors(w, "cpu", where="host")
+    host["q"][1, 3, 5] = 1.0e6                       # request 1 only (bf16 holds ~1e6)
+    t = {k: v.to(dev) for k, v in host.items()}
+    idx = W.index_tensors(w, dev)
+    err = P.new_error_word(dev)
+    out = P.step(t["q"], t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], idx["block_tables"],
+                 idx["query_start_loc"], idx["seq_lens"], w.scale, decode_only=True, err=err,
+                 kv_scales=w.kv_scales)
+    torch.cuda.synchronize()
+    assert P.read_error(err) == P.ERRBIT_Q_RANGE
+    _, _, _, ref, _, _ = oracle_full_fp8(w, host)
+    keep = [0, 2]
+    assert_close(f64(out)[keep], ref[keep], "bf16", w.name)
