@@ -25,9 +25,11 @@
  *                     slots from explicit (request, position) pairs
  *   PA_FP8_E4M3       e4m3 cache pools with one scale per pool ("从零构建LLM
  *                     推理引擎", card "量化")
- *   pa_decode_no_alloc, pa_kernel_timing_enable / _read
+ *   pa_decode_no_alloc, pa_kernel_timing_enable / _read,
+ *   pa_selftest_wait_timeout
  *                     entry points with no counterpart on the pages (a decode
- *                     for callers that cannot allocate; per-launch timing)
+ *                     for callers that cannot allocate; per-launch timing; a
+ *                     check that a bounded device wait ends and reports)
  *
  * Conventions shared by every call
  *   - All tensor arguments are DEVICE pointers of the current CUDA device,
@@ -296,8 +298,12 @@ pa_status pa_mixed_step(const void* q, const void* key_cache, const void* value_
  *   sizes exceeds PA_DECODE_NO_ALLOC_MAX_BYTES (nothing is launched).
  *   The first call on a device looks up the array's address on that device
  *   (cudaGetSymbolAddress) and caches it; make that first call before any
- *   stream capture.  All calls share the array: two calls whose kernels
- *   overlap on the GPU race.  Nothing in it needs clearing between calls.
+ *   stream capture.  The cached address belongs to the device's current
+ *   context: after a cudaDeviceReset of that device, this entry point must
+ *   not be called again in the same process (it would hand the kernels the
+ *   old context's address).  All calls share the array: two calls whose
+ *   kernels overlap on the GPU race.  Nothing in it needs clearing between
+ *   calls.
  */
 #define PA_DECODE_NO_ALLOC_MAX_BYTES (32u << 20) /* 32 MiB of device memory per GPU */
 
@@ -338,6 +344,27 @@ pa_status pa_kernel_timing_read(float* ms);
  * were, PA_ERR_CUDA if a CUDA call failed (e.g. an earlier kernel faulted).
  */
 pa_status pa_read_error(int32_t* err_word, int32_t* host_bits, void* stream);
+
+/*
+ * pa_selftest_wait_timeout -- a check of the library's failure detection
+ * (the pages have no counterpart).  Every mbarrier wait in the attention
+ * kernels is bounded: when it runs out it sets PA_ERRBIT_TIMEOUT and the
+ * kernel leaves its role, so a stalled pipeline ends its launch instead of
+ * hanging the device.  A correct call never reaches that exit; this entry
+ * point does, on purpose and harmlessly: it launches one warp whose lane 0
+ * waits, through the same bounded-wait routine, on a shared-memory mbarrier
+ * that nothing arrives at.
+ *   limit_us   the wait's limit in microseconds, 1 .. 100000 (100 ms)
+ *   err_word   device int32; PA_ERRBIT_TIMEOUT is OR-ed into it when the
+ *              wait gives up (required)
+ *   waited_ns  device uint64 or NULL: the wait's duration by the GPU's global
+ *              timer, from its start to its end
+ * Returns PA_ERR_INVALID_ARG for a limit outside the range or a NULL
+ * err_word (nothing is launched), PA_ERR_CUDA if the launch failed, PA_OK
+ * otherwise.  Asynchronous on `stream`; pa_read_error collects the bit.
+ */
+pa_status pa_selftest_wait_timeout(uint32_t limit_us, int32_t* err_word,
+                                   unsigned long long* waited_ns, void* stream);
 
 #ifdef __cplusplus
 }

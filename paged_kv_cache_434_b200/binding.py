@@ -31,7 +31,7 @@ EXPORTS = ("pa_status_str", "pa_version", "pa_slot_mapping", "pa_cache_write",
            "pa_decode_workspace_size", "pa_decode", "pa_mixed_step_workspace_size",
            "pa_mixed_step", "pa_read_error", "pa_decode_no_alloc", "pa_kernel_timing_enable",
            "pa_kernel_timing_read", "pa_rope_cos_sin_cache", "pa_rope_cache_write",
-           "pa_copy_blocks", "pa_slot_mapping_positions")
+           "pa_copy_blocks", "pa_slot_mapping_positions", "pa_selftest_wait_timeout")
 
 
 class PagedAttentionError(RuntimeError):
@@ -73,6 +73,7 @@ _SIGNATURES = {
     "pa_copy_blocks": ([_vp, _vp, _vp, _i64, _desc_p, _vp, _vp], ctypes.c_int),
     "pa_slot_mapping_positions": ([_vp, _i32, _i32, _vp, _vp, _i64, _i32, _i64, _vp, _vp, _vp],
                                   ctypes.c_int),
+    "pa_selftest_wait_timeout": ([ctypes.c_uint32, _vp, _vp, _vp], ctypes.c_int),
     "pa_rope_cache_write": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                              _i32, _i64, _i32, _desc_p, _vp, _vp], ctypes.c_int),
 }
@@ -439,3 +440,17 @@ def decode_no_alloc(q, k_cache, v_cache, block_tables, seq_lens, scale: float, o
         _cuda(seq_lens, "seq_lens", torch.int32, 1), float(scale), _cuda(out, "out"), B, H, W,
         _dt(out), ctypes.byref(desc), _err_ptr(err), _stream()), "pa_decode_no_alloc")
     return out
+
+
+def selftest_wait_timeout(limit_us: int, err, waited_ns=None) -> None:
+    """pa_selftest_wait_timeout: one warp waits, through the kernels' bounded
+    wait, on an mbarrier nothing arrives at.  The wait must give up after
+    `limit_us` microseconds (1 .. 100000) and OR PA_ERRBIT_TIMEOUT into `err`.
+    `waited_ns` (an int64 CUDA tensor of one element, or None) receives the
+    wait's duration by the GPU's global timer.  Asynchronous on the current
+    stream."""
+    ptr = None
+    if waited_ns is not None:
+        ptr = _cuda(waited_ns, "waited_ns", torch.int64)
+    _check(_lib().pa_selftest_wait_timeout(int(limit_us), _err_ptr(err), ptr, _stream()),
+           "pa_selftest_wait_timeout")

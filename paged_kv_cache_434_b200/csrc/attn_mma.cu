@@ -79,7 +79,7 @@ __device__ __forceinline__ uint32_t swz(int key, int chunk) {
 template <int D, int HG, bool F8>
 __global__ void __launch_bounds__((HG + 1) * 32, 1)
     attn_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                    AttnGeom g, WsView ws, int box_rows, int heads_per_box, int after_tiles) {
+                    AttnGeom g, WsView ws, int box_rows, int by_token, int after_tiles) {
   static_assert(!F8 || D == 128, "e4m3 pools: head_dim 128");
   using C = mmak::Cfg<D, HG, F8>;
   constexpr int NS = C::NS;
@@ -169,14 +169,15 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         if (done || (si.flags & mmak::kBad)) {
           mbar_arrive(&full[stage]);
         } else {
-          const int boxes = rows1 >= 0 ? 2 : 1;
-          const uint32_t box_bytes = static_cast<uint32_t>(box_rows) * 128u;
-          mbar_arrive_expect_tx(&full[stage], 2u * HG * NH * boxes * box_bytes);
           uint8_t* kbase = stages + stage * C::kStageBytes;
           uint8_t* vbase = kbase + C::kTensorBytes;
           const int head0 = item.y * HG;
-          if (heads_per_box == HG) {
-            // (dim, token, head) map: one box per half and tensor
+          // The branch follows the kind of map the host encoded (by_token), and
+          // each branch announces exactly the bytes of the boxes it issues.
+          if (by_token) {
+            // (dim, token, head) map, box [64 | 128 codes, 16 tokens, HG heads]:
+            // one box per half and tensor
+            mbar_arrive_expect_tx(&full[stage], 2u * NH * HG * C::kTile);
 #pragma unroll
             for (int dh = 0; dh < NH; ++dh) {
               const int toff = dh * HG * C::kTile;
@@ -184,7 +185,11 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
               tma_load_3d_hint(vbase + toff, &tmV, &full[stage], dh * 64, rows0, head0, policy);
             }
           } else {
-            // (dim, head, token) map: one box per head, half, tensor and block
+            // (dim, head, token) map, box [64 | 128 codes, 1 head, box_rows
+            // tokens]: one box per head, half, tensor and block
+            const int boxes = rows1 >= 0 ? 2 : 1;
+            const uint32_t box_bytes = static_cast<uint32_t>(box_rows) * 128u;
+            mbar_arrive_expect_tx(&full[stage], 2u * HG * NH * boxes * box_bytes);
 #pragma unroll
             for (int hh = 0; hh < HG; ++hh) {
 #pragma unroll
@@ -599,10 +604,11 @@ static cudaError_t launch_mma_t(const AttnGeom& g, const WsView& ws, int num_sms
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::kThreads, C::kSmem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
+  // the kernel's choice of box coordinates must follow the map just encoded
+  const int by_token = heads_per_box > 1 ? 1 : 0;
   return launch_pdl<attn_mma_kernel<D, HG, F8>>(dim3(num_sms * per_sm), dim3(C::kThreads),
-                                                C::kSmem,
-                                            s, tk, tv, g, ws, box_rows, heads_per_box,
-                                            after_tiles);
+                                                C::kSmem, s, tk, tv, g, ws, box_rows, by_token,
+                                                after_tiles);
 }
 
 cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,

@@ -10,7 +10,9 @@
 //
 // Set-up: the first call on a device looks up the array's device address with
 // cudaGetSymbolAddress while that device is current, and caches it per device.
-// That first call should come before any stream capture.  In host code the
+// That first call should come before any stream capture.  The cached address
+// belongs to the context it was looked up in: after a cudaDeviceReset of the
+// device the entry point must not be called again in that process.  In host code the
 // array's name is only a host-side stand-in, never a device address, so the
 // looked-up pointer is what the kernels receive.
 //

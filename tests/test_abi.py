@@ -280,6 +280,7 @@ def test_binding_constants_match_the_header():
 
 
 _CTYPES_OF = {"int32_t": "c_int", "int64_t": "c_long", "float": "c_float", "double": "c_double",
+              "uint32_t": "c_uint",
               "size_t": "c_ulong", "int": "c_int"}
 
 

@@ -7,7 +7,7 @@ pattern must be intact: no kernel writes before or after the buffer it was
 given, even when the workspace is exactly the size the library asked for.
 The results inside are checked against the oracle as in the parity suites.
 
-This file is collected after every other GPU test.
+The `late` mark runs this file after the other GPU tests except the no-alloc ones.
 """
 
 import numpy as np
@@ -19,7 +19,7 @@ import paged_kv_cache_434_b200 as P
 from paged_kv_cache_434_b200 import workloads as W
 from _util import assert_close, bits, f64, fp8_codes, oracle_full, oracle_full_fp8
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.late(3)]
 
 GUARD = 4096   # bytes on each side; a multiple of 256 keeps the inner buffer 256-byte aligned
 FILL = 0xA5

@@ -11,7 +11,7 @@ Checked against the oracle, through the same step the benchmark times:
   * attention on sampled requests, against the fp64 oracle over the pools'
     dequantised values, within the bf16-input tolerance.
 
-This file is collected after the parity suites.
+The `late` mark runs this file after the parity suites.
 """
 
 import numpy as np
@@ -23,7 +23,7 @@ import paged_kv_cache_434_b200 as P
 from paged_kv_cache_434_b200 import workloads as W
 from _util import assert_close, f64, oracle_rows
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.late(1)]
 
 
 def _dequantised_blocks(w, pool_u8, seqs, table):

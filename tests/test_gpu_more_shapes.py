@@ -8,7 +8,7 @@
     item carries a single KV head (the one-head variant of the mma.sync
     kernel) and the tensor-core tiles take all query heads of the one group.
 
-This file is collected after every other GPU test.
+The `late` mark runs this file after the parity suites.
 """
 
 import numpy as np
@@ -19,7 +19,7 @@ import paged_kv_cache_434_b200 as P
 from paged_kv_cache_434_b200 import workloads as W
 from _util import assert_close, bits, f64, fp8_codes, oracle_full, oracle_full_fp8
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.late(2)]
 
 BLOCK_SIZES = [64, 128, 256]
 
@@ -91,27 +91,31 @@ def test_shared_prefix_large_blocks(cuda_device, bs):
     _run_and_check(w, cuda_device)
 
 
+# Block size 16 takes one [dims x 16 keys] box per head and half; block size 8
+# takes two [dims x 8 keys] boxes per head and half (a stage spans two blocks).
+@pytest.mark.parametrize("bs", [16, 8])
 @pytest.mark.parametrize("dtype,hq,hkv,d", [("bf16", 8, 1, 128), ("bf16", 16, 1, 64),
                                             ("bf16", 12, 3, 128), ("bf16", 5, 5, 64),
                                             ("f32", 8, 1, 64)])
-def test_decode_single_kv_head_per_item(cuda_device, dtype, hq, hkv, d):
-    rng = np.random.default_rng([hq, hkv, d])
-    lens = [1, 15, 16, 17, 700, 2500] + rng.integers(1, 1200, 3).tolist()
-    w = W.custom(f"decode_mqa_{hq}_{hkv}_{d}_{dtype}", lens, [1] * len(lens), hq, hkv, d, 16,
-                 dtype, seed=hq * 7 + hkv + d, extra_blocks=2)
+def test_decode_single_kv_head_per_item(cuda_device, bs, dtype, hq, hkv, d):
+    rng = np.random.default_rng([hq, hkv, d, bs])
+    lens = [1, 7, 8, 9, 15, 16, 17, 700, 2500] + rng.integers(1, 1200, 3).tolist()
+    w = W.custom(f"decode_mqa_{hq}_{hkv}_{d}_{dtype}_bs{bs}", lens, [1] * len(lens), hq, hkv, d,
+                 bs, dtype, seed=hq * 7 + hkv + d + bs, extra_blocks=2)
     _run_and_check(w, cuda_device)
 
 
+@pytest.mark.parametrize("bs", [16, 8])
 @pytest.mark.parametrize("hq,hkv,d", [(8, 1, 128), (16, 1, 64), (12, 3, 128)])
-def test_mixed_step_single_kv_head_per_item(cuda_device, hq, hkv, d):
-    lens = [400, 130, 1, 37, 900]
-    qlens = [150, 130, 1, 1, 1]
-    w = W.custom(f"mixed_mqa_{hq}_{hkv}_{d}", lens, qlens, hq, hkv, d, 16, "bf16",
-                 seed=hq * 7 + hkv + d + 1)
+def test_mixed_step_single_kv_head_per_item(cuda_device, bs, hq, hkv, d):
+    lens = [400, 130, 1, 37, 900, 9]
+    qlens = [150, 130, 1, 1, 1, 1]
+    w = W.custom(f"mixed_mqa_{hq}_{hkv}_{d}_bs{bs}", lens, qlens, hq, hkv, d, bs, "bf16",
+                 seed=hq * 7 + hkv + d + bs + 1)
     _run_and_check(w, cuda_device)
 
 
-@pytest.mark.parametrize("hq,hkv", [(8, 1), (16, 4)])
+@pytest.mark.parametrize("hq,hkv", [(8, 1), (12, 3), (16, 4)])
 def test_fp8_decode_head_groups(cuda_device, hq, hkv):
     # e4m3 decode with one and with four KV heads per work item
     lens = [1, 16, 17, 900, 2500]
