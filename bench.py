@@ -75,6 +75,8 @@ def parse_args(argv=None):
                     help="time budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default workload only: skip the mixed-step and shared-prefix objects")
     return ap.parse_args(argv)
 
 
@@ -408,13 +410,15 @@ def time_prefill_tiles(P, w, t, flush, steps):
     return statistics.mean(ms), len(ms)
 
 
-def run_ours(args, rank, world, local):
+def measure(args, name, rank, world, local, with_e2e=True, with_cpu=True):
+    """Time one workload's step on this rank's GPU and return its JSON line
+    (every rank computes it; the collectives inside run on every rank)."""
     import paged_kv_cache_434_b200 as P
     from paged_kv_cache_434_b200 import workloads as W
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = workload_for(args.workload, args.seed + rank)
+    w = workload_for(name, args.seed + rank)
     t = W.make_tensors(w, dev)
     idx = W.index_tensors(w, dev)
     T = w.num_tokens
@@ -493,8 +497,8 @@ def run_ours(args, rank, world, local):
     kernel_ms = {k: round(statistics.mean(v), 4) for k, v in kt.items()}
 
     bc = byte_counts(w)
-    metric, unit = metric_of(args.workload)
-    if args.workload in ("mixed", "mixed_prefill"):
+    metric, unit = metric_of(name)
+    if name in ("mixed", "mixed_prefill"):
         value = job_throughput(T, args.steps, world, total_s)
     else:
         value = job_throughput(bc["step"], args.steps, world, total_s) / 1e9
@@ -516,7 +520,8 @@ def run_ours(args, rank, world, local):
                 "timed_over": f"the decode-partition launch alone: CUDA events on its stream, "
                               f"mean of {n_k} launches, L2 flushed before each",
                 "ms": round(dk_s * 1e3, 4),
-                "traffic": kernel_traffic(src, f"{dominant}_{args.workload}.md"),
+                "traffic": kernel_traffic(src, f"{dominant}_{name}.md"),
+                "traffic_source": "from profiles/ (ncu summary of the same kernel source)",
                 "algorithmic_bytes_per_launch": dk_bytes,
                 "attention_call": {"ms": round(attn_s * 1e3, 4),
                                    "achieved": round(bc["attention"] / attn_s / 1e9, 1),
@@ -528,7 +533,7 @@ def run_ours(args, rank, world, local):
         roofline["own_peaks"] = dict(own, frac_of_own_copy=round(achieved / own["copy_gbs"], 4))
     extra = dict(extra_kv)
     prefill_roofline = None
-    if args.workload in ("mixed", "mixed_prefill"):
+    if name in ("mixed", "mixed_prefill"):
         fl = prefill_flops(w)
         extra["prefill_flops_per_step"] = fl
         tiles = time_prefill_tiles(P, w, t, flush, args.steps)
@@ -545,13 +550,14 @@ def run_ours(args, rank, world, local):
                               f"the q_b > 1 requests alone, CUDA events on its stream, mean of "
                               f"{n_t} launches, L2 flushed before each",
                 "ms": round(tiles_ms, 4), "algorithmic_flops_per_launch": fl,
-                "traffic": kernel_traffic("attn_tc.cu", f"attn_tc_kernel_{args.workload}.md")}
+                "traffic": kernel_traffic("attn_tc.cu", f"attn_tc_kernel_{name}.md"),
+                "traffic_source": "from profiles/ (ncu summary of the same kernel source)"}
             if own is not None and "bf16_gemm_tflops" in own:
                 prefill_roofline["frac_of_own_gemm"] = round(tf / own["bf16_gemm_tflops"], 4)
 
     # ---- end to end: host buffers in, result back to the host, each step
     e2e = None
-    if not args.no_e2e:
+    if with_e2e and not args.no_e2e:
         names = ["q", "k_new", "v_new"]
         host = {n: t[n].cpu().pin_memory() for n in names}
         host_idx = {n: idx[n].cpu().pin_memory() for n in ("block_tables", "seq_lens",
@@ -578,47 +584,96 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / 1e3, world, dev)
-        e2e_val = (T * args.steps * world / e2e_s if args.workload in ("mixed", "mixed_prefill")
+        e2e_val = (T * args.steps * world / e2e_s if name in ("mixed", "mixed_prefill")
                    else bc["step"] * args.steps * world / e2e_s / 1e9)
         e2e = {"value": round(e2e_val, 2), "unit": unit, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_s * 1e3 / args.steps, 4)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if with_cpu and rank == 0 and world == 1 and not args.no_cpu_baseline:
         units, el, desc, threads = oracle_sample(w, (t["k_cache"], t["v_cache"]),
                                                  args.cpu_seconds)
-        v = units / el / (1 if args.workload in ("mixed", "mixed_prefill") else 1e9)
+        v = units / el / (1 if name in ("mixed", "mixed_prefill") else 1e9)
         cpu = {"value": round(v, 4), "unit": unit, "cores": threads, "kind": "oracle",
                "sample": desc}
 
+    line = {
+        "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(total_s * 1e3 / args.steps, 4),
+        "ms_per_step_p10_p50_p90": [round(float(x), 4) for x in
+                                    np.percentile(step_ms, [10, 50, 90])],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": ("e4m3 pools, f16 tensor-core products" if w.kv_dtype == "fp8" else w.dtype),
+        "data": "synthetic: seeded N(0,1) Q/K/V rounded to the dtype, seeded lengths and "
+                "randomly permuted physical blocks",
+        "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_tokens": T,
+                   "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+                   "head_dim": w.head_dim, "block_size": w.block_size,
+                   "num_blocks": w.num_blocks,
+                   "kv_bytes_unique": bc["kv"], "step_bytes": bc["step"],
+                   "l2": "flushed before every step (512 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world} (independent batches per GPU)",
+                   **extra},
+        "roofline": roofline,
+        **({"prefill_roofline": prefill_roofline} if prefill_roofline else {}),
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "kernel_ms": kernel_ms,
+        "gpu_launches": (2 + len(kernel_ms)) * args.steps,
+        "clocks": clk,
+        "wall_s_timed_region": round(wall, 3),
+    }
+    return line
+
+
+def _in_step_tiles(line):
+    """The tensor-core tile launch of the full mixed step, on the SMs the
+    planner gave it (per-launch timing pass), as a fraction of the bf16 peak."""
+    fl = line["config"].get("prefill_flops_per_step")
+    ms = line["kernel_ms"].get("tiles")
+    if not fl or not ms:
+        return None
+    peaks = load_peaks()
+    tf = fl / (ms / 1e3) / 1e12
+    return {"bound": "tensor", "kernel": "attn_tc_kernel", "achieved": round(tf, 1),
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(tf / peaks["bf16_tflops"], 4), "ms": ms,
+            "timed_over": "the tile launch inside the full mixed step, on the SMs the planner "
+                          "leaves to the tiles (the decode partitions run on the others); CUDA "
+                          "events on its stream in the per-launch timing pass"}
+
+
+def run_ours(args, rank, world, local):
+    line = measure(args, args.workload, rank, world, local)
+    if args.workload == "llama8b_decode" and not args.no_extras:
+        # The other half of the metric (a mixed continuous-batching step) and the
+        # shared-prefix decode batch, measured in the same process after the
+        # headline, each with its own timed region, clocks and launch count.
+        torch.cuda.empty_cache()
+        m = measure(args, "mixed", rank, world, local, with_cpu=False)
+        line["mixed_step"] = {
+            k: m[k] for k in ("metric", "value", "unit", "ms_per_step", "e2e", "kernel_ms",
+                              "gpu_launches", "clocks")}
+        line["mixed_step"]["config"] = {k: m["config"][k] for k in (
+            "workload", "num_seqs", "num_tokens", "prefill_flops_per_step")}
+        line["mixed_step"]["prefill_roofline"] = {"alone": m.get("prefill_roofline"),
+                                                  "in_step": _in_step_tiles(m)}
+        line["mixed_step"]["decode_roofline"] = m["roofline"]
+        torch.cuda.empty_cache()
+        sp = measure(args, "shared_prefix", rank, world, local, with_cpu=False)
+        line["shared_prefix"] = {
+            k: sp[k] for k in ("metric", "value", "unit", "ms_per_step", "e2e", "kernel_ms",
+                               "gpu_launches", "clocks")}
+        line["shared_prefix"]["config"] = {k: sp["config"][k] for k in (
+            "workload", "num_seqs", "num_heads", "num_kv_heads", "block_size",
+            "kv_bytes_unique")}
+        line["shared_prefix"]["attention_call"] = dict(
+            sp["roofline"]["attention_call"],
+            note="per attention call, on unique bytes: each physical block once (the shared "
+                 "prefix once), Q read and fp32 O written, against the HBM copy peak")
+        line["shared_prefix"]["suffix_partitions"] = sp["roofline"]
     if rank == 0:
-        line = {
-            "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
-            "steps": args.steps, "warmup": max(args.warmup, 3),
-            "ms_per_step": round(total_s * 1e3 / args.steps, 4),
-            "ms_per_step_p10_p50_p90": [round(float(x), 4) for x in
-                                        np.percentile(step_ms, [10, 50, 90])],
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": ("e4m3 pools, f16 tensor-core products" if w.kv_dtype == "fp8" else w.dtype),
-            "data": "synthetic: seeded N(0,1) Q/K/V rounded to the dtype, seeded lengths and "
-                    "randomly permuted physical blocks",
-            "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_tokens": T,
-                       "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
-                       "head_dim": w.head_dim, "block_size": w.block_size,
-                       "num_blocks": w.num_blocks,
-                       "kv_bytes_unique": bc["kv"], "step_bytes": bc["step"],
-                       "l2": "flushed before every step (512 MiB write, outside the events)",
-                       "parallelism": f"replicas x{world} (independent batches per GPU)",
-                       **extra},
-            "roofline": roofline,
-            **({"prefill_roofline": prefill_roofline} if prefill_roofline else {}),
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "kernel_ms": kernel_ms,
-            "gpu_launches": (2 + len(kernel_ms)) * args.steps,
-            "clocks": clk,
-            "wall_s_timed_region": round(wall, 3),
-        }
         print(json.dumps(line), flush=True)
 
 

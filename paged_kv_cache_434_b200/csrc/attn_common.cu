@@ -29,7 +29,7 @@ namespace pa {
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 WsLayout ws_layout(int64_t num_qrows, int num_heads, int head_dim, int head_groups,
-                   int64_t max_parts, int64_t max_tiles) {
+                   int64_t max_parts, int64_t max_tiles, int max_ctas) {
   WsLayout L{};
   L.num_qrows = num_qrows;
   L.max_parts = max_parts;
@@ -54,6 +54,11 @@ WsLayout ws_layout(int64_t num_qrows, int num_heads, int head_dim, int head_grou
   off = align_up(off + num_qrows * num_heads * max_parts * head_dim * sizeof(float), 256);
   L.tiles = off;
   off = align_up(off + max_tiles * sizeof(int4), 256);
+  L.max_ctas = max_ctas;
+  L.sk = off;
+  off = align_up(off + static_cast<size_t>(max_ctas) * sizeof(int4), 256);
+  L.row_ustart = off;
+  off = align_up(off + num_qrows * sizeof(int64_t), 256);
   L.total = off;
   return L;
 }
@@ -70,6 +75,9 @@ WsView ws_view(void* base, const WsLayout& L) {
   v.part_ml = reinterpret_cast<float2*>(p + L.part_ml);
   v.part_o = reinterpret_cast<float*>(p + L.part_o);
   v.tiles = reinterpret_cast<int4*>(p + L.tiles);
+  v.sk = reinterpret_cast<int4*>(p + L.sk);
+  v.row_ustart = reinterpret_cast<int64_t*>(p + L.row_ustart);
+  v.max_ctas = static_cast<int32_t>(L.max_ctas);
   v.max_parts = L.max_parts;
   v.max_items = L.max_items;
   v.max_tiles = L.max_tiles;
@@ -162,6 +170,250 @@ __device__ int shared_prefix_blocks(const AttnGeom& g, int max_cols, int* s_bad)
   return r;
 }
 
+// Exclusive prefix of v over the CTA's threads in thread order; *total gets
+// the sum.  s_scan holds 33 values.
+template <typename T>
+__device__ __forceinline__ T block_exclusive_scan(T v, T* s_scan, T* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  T incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const T n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) s_scan[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const T w = s_scan[lane];
+    T wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const T n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    s_scan[lane] = wi - w;
+    if (lane == 31) s_scan[32] = wi;
+  }
+  __syncthreads();
+  *total = s_scan[32];
+  return s_scan[warp] + incl - v;
+}
+
+// Decode batches of up to kFastRows requests, in one pass: each thread holds
+// up to kFastPerThread consecutive requests' lengths in registers, so the
+// partition plan needs no re-reads of the workspace and few barriers.
+//   * Balanced ranges (no tiles beside the batch, one head group per row):
+//     the units are cut into num_sms ranges of equal work; CTA c streams range
+//     c, so every CTA ends at the same time and a row is split only where a
+//     range boundary falls inside it (its pieces are its partitions).  Taken
+//     when no row is cut into more pieces than the partial slots hold.
+//   * Otherwise rows are cut into uniform partitions of P stages, and the
+//     items are listed by the whole CTA (item i finds its row by binary search
+//     over the rows' first items).
+// Returns false, having written nothing, when every block table starts with
+// the same block and the batch qualifies for the shared-prefix cascade: the
+// general planner then looks for the prefix.
+constexpr int kFastPerThread = 4;
+constexpr int kFastRows = kPlanThreads * kFastPerThread;
+
+__device__ bool plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsView& ws,
+                                 int* s_rowpos, int* s_scan, long long* s_scan64,
+                                 long long* s_sum, int* s_max, int* s_P, int* s_merge,
+                                 int* s_merge_big) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int B = g.num_seqs;
+  const int per = (B + kPlanThreads - 1) / kPlanThreads;  // <= kFastPerThread
+  const int r0 = tid * per;
+  const int64_t max_keys = static_cast<int64_t>(g.max_blocks) * g.block_size;
+  const bool look_shared = a.cascade && B >= kCascadeMinSeqs && g.max_blocks > 0;
+  const int ref0 = look_shared ? g.block_tables[0] : 0;
+  int L[kFastPerThread], c0[kFastPerThread];
+#pragma unroll
+  for (int k = 0; k < kFastPerThread; ++k) {
+    const int r = r0 + k;
+    L[k] = 0;
+    c0[k] = ref0;
+    if (k < per && r < B) {
+      L[k] = g.seq_lens[r];
+      if (look_shared) c0[k] = g.block_tables[static_cast<int64_t>(r) * g.max_blocks];
+    }
+  }
+  bool same = true, all_ok = true;
+  int min_len = 0x7fffffff;
+#pragma unroll
+  for (int k = 0; k < kFastPerThread; ++k) {
+    if (k >= per || r0 + k >= B) continue;
+    const bool ok = L[k] >= 0 && L[k] <= max_keys;
+    all_ok &= ok;
+    same &= c0[k] == ref0;
+    if (ok) min_len = min(min_len, L[k]);
+  }
+  if (look_shared &&
+      __syncthreads_and(same && all_ok && (min_len == 0x7fffffff || min_len > kCascadeMinPrefix)))
+    return false;
+
+  // invalid requests: error bits, rows left unwritten (L = -1 from here on)
+  long long units_sum = 0;
+  int units_max = 0;
+#pragma unroll
+  for (int k = 0; k < kFastPerThread; ++k) {
+    if (k >= per || r0 + k >= B) continue;
+    int bits = 0;
+    if (L[k] < 0) bits |= PA_ERRBIT_QUERY_TOO_LONG;
+    if (L[k] > max_keys) bits |= PA_ERRBIT_SEQ_TOO_LONG;
+    if (bits) {
+      if (g.err_word) atomicOr(g.err_word, bits);
+      L[k] = -1;
+      continue;
+    }
+    const int units = (L[k] + kStageTokens - 1) / kStageTokens;
+    units_sum += units;
+    units_max = max(units_max, units);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    units_sum += __shfl_xor_sync(0xffffffffu, units_sum, o);
+    units_max = max(units_max, __shfl_xor_sync(0xffffffffu, units_max, o));
+  }
+  if (lane == 0) {
+    s_sum[warp] = units_sum;
+    s_max[warp] = units_max;
+  }
+  __shared__ long long s_total;
+  __syncthreads();
+  const long long cap =
+      max(1LL, static_cast<long long>(ws.max_parts) - (a.cascade ? kMaxPrefixChunks : 0));
+  if (tid == 0) {
+    long long total = 0;
+    int mx = 0;
+    for (int w = 0; w < kPlanThreads / 32; ++w) {
+      total += s_sum[w];
+      mx = max(mx, s_max[w]);
+    }
+    s_total = total;
+    const long long by_target =
+        (total * a.head_groups + a.target_items - 1) / max(a.target_items, 1);
+    const long long by_cap = (mx + cap - 1) / cap;
+    const long long P = max(static_cast<long long>(a.min_part_stages), max(by_target, by_cap));
+    *s_P = static_cast<int>(max(P, 1LL));
+    *s_merge = 0;
+    *s_merge_big = 0;
+  }
+  __syncthreads();
+  const int P = *s_P;
+  const long long U = s_total;
+  const int C = a.num_sms;
+
+  // pieces of each row: balanced ranges, if every row fits the partial slots
+  int np[kFastPerThread];
+  long long us0 = 0;
+  bool balanced = a.balanced && a.head_groups == 1 && U > 0 && C <= ws.max_ctas;
+  if (balanced) {
+    long long my_units = 0;
+#pragma unroll
+    for (int k = 0; k < kFastPerThread; ++k)
+      if (k < per && r0 + k < B && L[k] > 0) my_units += (L[k] + kStageTokens - 1) / kStageTokens;
+    long long dummy;
+    us0 = block_exclusive_scan<long long>(my_units, s_scan64, &dummy);
+    bool fits = U / C < (1LL << 30);
+    long long us = us0;
+#pragma unroll
+    for (int k = 0; k < kFastPerThread; ++k) {
+      np[k] = -1;
+      if (k >= per || r0 + k >= B || L[k] < 0) continue;
+      const long long n_st = (L[k] + kStageTokens - 1) / kStageTokens;
+      np[k] = n_st == 0 ? 0 : range_of(us + n_st - 1, U, C) - range_of(us, U, C) + 1;
+      fits &= np[k] <= cap;
+      us += n_st;
+    }
+    balanced = __syncthreads_and(fits);
+  }
+  if (balanced) {
+    long long us = us0;
+#pragma unroll
+    for (int k = 0; k < kFastPerThread; ++k) {
+      const int r = r0 + k;
+      if (k >= per || r >= B) continue;
+      ws.row_ustart[r] = us;
+      if (L[k] < 0) continue;
+      const long long n_st = (L[k] + kStageTokens - 1) / kStageTokens;
+      const long long ue = us + n_st;
+      // the ranges that start inside this row
+      for (long long c = (us * C + U - 1) / U; c < C; ++c) {
+        const long long x = range_start(c, U, C);
+        if (x >= ue) break;
+        ws.sk[c] = make_int4(r, 0, static_cast<int>(x - us),
+                             static_cast<int>(range_start(c + 1, U, C) - x));
+      }
+      us = ue;
+    }
+  } else {
+    int my_items = 0;
+#pragma unroll
+    for (int k = 0; k < kFastPerThread; ++k) {
+      np[k] = -1;
+      if (k >= per || r0 + k >= B || L[k] < 0) continue;
+      const int units = (L[k] + kStageTokens - 1) / kStageTokens;
+      np[k] = (units + P - 1) / P;
+      my_items += np[k] * a.head_groups;
+    }
+    int n_items = 0;
+    int pos = block_exclusive_scan<int>(my_items, s_scan, &n_items);
+#pragma unroll
+    for (int k = 0; k < kFastPerThread; ++k) {
+      const int r = r0 + k;
+      if (k >= per || r >= B) continue;
+      s_rowpos[r] = pos;
+      if (np[k] > 0) pos += np[k] * a.head_groups;
+    }
+    if (tid == 0) {
+      s_rowpos[B] = n_items;
+      ws.ctrl[1] = n_items;
+    }
+    __syncthreads();
+    // items {row, head group, partition}, row-major, spread over the CTA
+    for (int i = tid; i < n_items; i += kPlanThreads) {
+      int lo = 0, hi = B;  // the row r with s_rowpos[r] <= i < s_rowpos[r + 1]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_rowpos[mid] <= i) lo = mid;
+        else hi = mid;
+      }
+      const int k = i - s_rowpos[lo];
+      ws.items[i] = make_int4(lo, k % a.head_groups, k / a.head_groups, 0);
+    }
+  }
+  // rows: info, partition counts, and the merge pass's list (rows with no key
+  // get zeros there; rows of more than one partition are merged)
+#pragma unroll
+  for (int k = 0; k < kFastPerThread; ++k) {
+    const int r = r0 + k;
+    if (k >= per || r >= B) continue;
+    ws.qrow_bad[r] = 0;
+    ws.nparts[r] = np[k];
+    ws.qrow_info[r] = np[k] >= 0 ? make_int4(r, L[k], 1, 0) : make_int4(-1, 0, 0, 0);
+    if (np[k] > 32) ws.merge_rows[g.num_qrows - 1 - atomicAdd(s_merge_big, 1)] = r;
+    else if (np[k] >= 0 && np[k] != 1) ws.merge_rows[atomicAdd(s_merge, 1)] = r;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    ws.ctrl[0] = 0;
+    if (balanced) ws.ctrl[1] = 0;
+    ws.ctrl[2] = P * kStageTokens;
+    ws.ctrl[3] = 0;
+    ws.ctrl[4] = 0;  // no tiles, no shared prefix
+    ws.ctrl[5] = *s_merge;
+    ws.ctrl[6] = 0;
+    ws.ctrl[7] = 0;
+    ws.ctrl[8] = 0;
+    ws.ctrl[9] = *s_merge_big;
+    ws.ctrl[10] = balanced ? C : 0;
+    ws.ctrl[11] = balanced ? static_cast<int>(U & 0xffffffffLL) : 0;
+    ws.ctrl[12] = balanced ? static_cast<int>(U >> 32) : 0;
+  }
+  return true;
+}
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs a, WsView ws) {
   grid_launch_dependents();
   grid_dependency_wait();  // seq_lens / tables / the workspace may come from the previous launch
@@ -175,9 +427,18 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   __shared__ int s_big[kMaxBig];
   __shared__ int s_bigpos[kMaxBig];
   __shared__ int s_hist[kTileBins];
+  __shared__ int s_rowpos[kFastRows + 1];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool decode_mode = g.query_start_loc == nullptr;
   const int64_t max_keys = static_cast<int64_t>(g.max_blocks) * g.block_size;
+
+  if (decode_mode && g.num_seqs <= kFastRows && g.num_qrows == g.num_seqs) {
+    __shared__ int s_scan33[33];
+    __shared__ long long s_scan64[33];
+    if (plan_decode_fast(g, a, ws, s_rowpos, s_scan33, s_scan64, s_sum, s_max, &s_P, &s_merge,
+                         &s_merge_big))
+      return;
+  }
 
   // 0. rows no request covers stay unwritten
   for (int r = tid; r < g.num_qrows; r += kPlanThreads) {
@@ -523,6 +784,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     ws.ctrl[6] = prefix_tokens;
     ws.ctrl[7] = prefix_chunks;
     ws.ctrl[8] = s_ntc;
+    ws.ctrl[10] = 0;  // items from the list
   }
 }
 
@@ -768,29 +1030,29 @@ __device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView&
 #pragma unroll
   for (int e = 0; e < V; ++e) acc[e] = 0.f;
   const float* po = ws.part_o + base * D + lane * V;
-  int k = 0;
-  for (; k + 3 < np; k += 4) {
-    float x[4][V], ck[4];
+  // up to 16 partial rows in flight per lane: a row of at most 32 partitions
+  // takes at most two round trips to L2
+  constexpr int kBatch = 16;
+  for (int k0 = 0; k0 < np; k0 += kBatch) {
+    float x[kBatch][V];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      ck[u] = __shfl_sync(0xffffffffu, c, k + u);
-      if constexpr (V == 4) {  // one 16-byte load per partition
-        const float4 t4 = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(k + u) * D);
+    for (int u = 0; u < kBatch; ++u) {
+      const bool ok = k0 + u < np;
+      if constexpr (V == 4) {
+        const float4 t4 = ok ? *reinterpret_cast<const float4*>(po + static_cast<int64_t>(k0 + u) * D)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
         x[u][0] = t4.x, x[u][1] = t4.y, x[u][2] = t4.z, x[u][3] = t4.w;
       } else {
 #pragma unroll
-        for (int e = 0; e < V; ++e) x[u][e] = po[static_cast<int64_t>(k + u) * D + e];
+        for (int e = 0; e < V; ++e) x[u][e] = ok ? po[static_cast<int64_t>(k0 + u) * D + e] : 0.f;
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < kBatch; ++u) {
+      const float cu = __shfl_sync(0xffffffffu, c, min(k0 + u, 31));
 #pragma unroll
-      for (int e = 0; e < V; ++e) acc[e] = fmaf(x[u][e], ck[u], acc[e]);
-  }
-  for (; k < np; ++k) {
-    const float ck = __shfl_sync(0xffffffffu, c, k);
-#pragma unroll
-    for (int e = 0; e < V; ++e) acc[e] = fmaf(po[static_cast<int64_t>(k) * D + e], ck, acc[e]);
+      for (int e = 0; e < V; ++e) acc[e] = fmaf(x[u][e], cu, acc[e]);
+    }
   }
   const float inv = 1.f / den;
 #pragma unroll

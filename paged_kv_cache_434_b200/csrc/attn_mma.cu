@@ -45,7 +45,8 @@ struct StageInfo {
   int part;
   int nvalid;
   int flags;
-  int pad0, pad1;
+  int np;  // partitions of the item's row
+  int pad1;
 };
 
 // F8: e4m3 pools (head_dim 128).  A stage then holds [16 keys x 128 codes]
@@ -128,17 +129,64 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     uint32_t phase = 0;
     int round = 0;  // completed passes over the ring
     bool ok = true;
+    // Work source: this CTA's balanced range of (row, stage) units when the
+    // planner cut the batch into ranges (C > 0), else items taken from the
+    // planner's list one at a time.
+    const int C = __ldcg(&ws.ctrl[10]);
+    const long long U = static_cast<long long>(static_cast<unsigned>(__ldcg(&ws.ctrl[11]))) |
+                        (static_cast<long long>(__ldcg(&ws.ctrl[12])) << 32);
+    int sk_r = 0, sk_s = 0, sk_left = 0;
+    if (C > 0 && static_cast<int>(blockIdx.x) < C) {
+      const int4 st = __ldcg(&ws.sk[blockIdx.x]);
+      sk_r = st.x, sk_s = st.z, sk_left = st.w;
+    }
     for (;;) {
-      const int it = atomicAdd(&ws.ctrl[0], 1);
-      const bool done = it >= n_items;
+      bool done;
       int4 item = make_int4(0, 0, 0, 0), qi = make_int4(0, 0, 0, 0);
-      if (!done) {
-        item = __ldcg(&ws.items[it]);
-        qi = __ldcg(&ws.qrow_info[item.x]);
+      int lo, hi, np = 1;
+      if (C > 0) {
+        // the next piece of the range: stages [sk_s, sk_s + take) of row sk_r
+        int n_st = 0, take = 0;
+        done = sk_left <= 0;
+        while (!done) {
+          qi = __ldcg(&ws.qrow_info[sk_r]);
+          n_st = qi.z ? (qi.y - qi.w + kStageTokens - 1) / kStageTokens : 0;
+          if (sk_s < n_st) {
+            take = min(sk_left, n_st - sk_s);
+            break;
+          }
+          sk_s = 0;  // a row without (more) units: the next row
+          if (++sk_r >= g.num_qrows) done = true;
+        }
+        if (!done) {
+          const long long u0 = __ldcg(&ws.row_ustart[sk_r]);
+          const int cf = range_of(u0, U, C);
+          np = range_of(u0 + n_st - 1, U, C) - cf + 1;
+          item = make_int4(sk_r, 0, static_cast<int>(blockIdx.x) - cf, 0);
+          lo = qi.w + sk_s * kStageTokens;
+          hi = min(min(lo + take * kStageTokens, qi.y), g.max_blocks * g.block_size);
+          sk_left -= take;
+          sk_s += take;
+          if (sk_s == n_st) {
+            sk_s = 0;
+            ++sk_r;
+          }
+        } else {
+          lo = 0;
+          hi = 1;
+        }
+      } else {
+        const int it = atomicAdd(&ws.ctrl[0], 1);
+        done = it >= n_items;
+        if (!done) {
+          item = __ldcg(&ws.items[it]);
+          qi = __ldcg(&ws.qrow_info[item.x]);
+          np = __ldcg(&ws.nparts[item.x]);
+        }
+        lo = qi.w + item.z * P;  // partitions start after a shared prefix
+        // lo >= hi: empty item, skipped; never past the table
+        hi = done ? lo + 1 : min(min(lo + P, qi.y), g.max_blocks * g.block_size);
       }
-      const int lo = qi.w + item.z * P;  // partitions start after a shared prefix
-      // lo >= hi: empty item, skipped; never past the table
-      const int hi = done ? lo + 1 : min(min(lo + P, qi.y), g.max_blocks * g.block_size);
       const int32_t* table = g.block_tables + static_cast<int64_t>(qi.x) * g.max_blocks;
       for (int key0 = lo; key0 < hi; key0 += kStageTokens) {
         if (round > 0 && !mbar_wait_bounded(&empty[stage], phase ^ 1, kWaitLimitNs)) {
@@ -150,6 +198,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         si.b = qi.x;
         si.hg = item.y;
         si.part = item.z;
+        si.np = np;
         si.nvalid = min(kStageTokens, hi - key0);
         si.flags = done ? mmak::kEnd
                         : ((key0 == lo ? mmak::kFirst : 0) |
@@ -465,7 +514,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_BLOCK_OOB);
         }
       } else {
-        const int np = __ldcg(&ws.nparts[r]);
+        const int np = si.np;
         if (np == 1) {
           const float i0 = vsc / l0, i1 = vsc / l1;
           const int64_t ob = (static_cast<int64_t>(r) * g.num_heads + head) * D;

@@ -664,9 +664,9 @@ static cudaError_t launch_tc_t(const AttnGeom& g, const WsView& ws, int num_sms,
                                        ws);
 }
 
-cudaError_t launch_attn_tc(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {
-  if (g.head_dim == 128) return launch_tc_t<128>(g, ws, num_sms, s);
-  return launch_tc_t<64>(g, ws, num_sms, s);
+cudaError_t launch_attn_tc(const AttnGeom& g, const WsView& ws, int grid, cudaStream_t s) {
+  if (g.head_dim == 128) return launch_tc_t<128>(g, ws, grid, s);
+  return launch_tc_t<64>(g, ws, grid, s);
 }
 
 }  // namespace pa

@@ -57,6 +57,7 @@ struct AttnPlan {
   bool use_tc;       // tcgen05 tiles: prefill requests, or a decode batch's shared prefix
   bool cascade;      // decode: shared-prefix tiles + suffix partitions
   int tile_tokens;
+  int tc_grid;       // CTAs of the tensor-core tile launch
   int heads_per_group;
   int head_groups;
   int num_sms;
@@ -101,6 +102,17 @@ static AttnPlan make_plan(int64_t num_qrows, int num_heads, int max_blocks,
   p.use_tc = (mixed && tc_ok) || p.cascade;
   p.max_parts = mp + (p.cascade ? kMaxPrefixChunks : 0);  // shared-prefix chunks
   p.tile_tokens = p.use_tc ? tc_tokens_per_tile(probe) : 0;
+  // A decode batch's shared-prefix tiles take at most one SM in two (the
+  // suffix partitions stream on the others from the start) unless there are
+  // more (request group, KV head) tiles than that: a grid of half the SMs
+  // leaves the other half to the partitions at once, also when the planner
+  // finds no shared prefix and the tile CTAs only exit.
+  p.tc_grid = p.num_sms;
+  if (p.cascade && p.tile_tokens > 0) {
+    const int64_t base =
+        (num_qrows + p.tile_tokens - 1) / p.tile_tokens * static_cast<int64_t>(c->num_kv_heads);
+    if (2 * base <= p.num_sms) p.tc_grid = (p.num_sms + 1) / 2;
+  }
   // ws_layout's terms in double first: arguments whose exact workspace would
   // not fit a size_t are refused instead of getting a wrapped, too small size
   const double rows = static_cast<double>(num_qrows), parts = static_cast<double>(p.max_parts);
@@ -110,7 +122,7 @@ static AttnPlan make_plan(int64_t num_qrows, int num_heads, int max_blocks,
                : 0.0;
   const double bytes = 64.0 * 4 + rows * (16 + 3 * 4) + rows * p.head_groups * parts * 16 +
                        rows * num_heads * parts * (8 + 4.0 * c->head_dim) + tiles * 16 +
-                       9 * 256;
+                       p.num_sms * 16.0 + rows * 8 + 11 * 256;
   p.size_ok = bytes <= kMaxWorkspaceBytes;
   p.max_tiles = (p.use_tc && p.size_ok)
                     ? ((num_qrows + p.tile_tokens - 1) / p.tile_tokens + num_seqs) *
@@ -207,7 +219,7 @@ class TimedCall {
 static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* workspace,
                                size_t ws_bytes, cudaStream_t s) {
   const WsLayout L = ws_layout(p.num_qrows, g.num_heads, g.head_dim, p.head_groups, p.max_parts,
-                               p.max_tiles);
+                               p.max_tiles, p.num_sms);
   if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return PA_ERR_WORKSPACE;
   if (g.num_qrows == 0 || g.num_seqs == 0) return PA_OK;
@@ -221,13 +233,14 @@ static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* works
   a.tile_tokens = p.tile_tokens;
   a.cascade = p.cascade ? 1 : 0;
   a.num_sms = p.num_sms;
+  a.balanced = p.use_mma ? 1 : 0;
   TimedCall tm(s);
   tm.begin(PA_TK_PLAN);
   if (launch_plan(g, a, ws, s) != cudaSuccess) return PA_ERR_CUDA;
   tm.end(PA_TK_PLAN);
   if (p.use_tc) {
     tm.begin(PA_TK_TILES);
-    if (launch_attn_tc(g, ws, p.num_sms, s) != cudaSuccess) return PA_ERR_CUDA;
+    if (launch_attn_tc(g, ws, p.tc_grid, s) != cudaSuccess) return PA_ERR_CUDA;
     tm.end(PA_TK_TILES);
   }
   tm.begin(PA_TK_DECODE);
@@ -311,7 +324,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t max
   const AttnPlan p = make_plan(num_seqs, num_heads, max_blocks_per_seq, cache, true);
   if (!p.size_ok) return 0;
   return ws_layout(p.num_qrows, num_heads, cache->head_dim, p.head_groups, p.max_parts,
-                   p.max_tiles)
+                   p.max_tiles, p.num_sms)
       .total;
 }
 
@@ -345,7 +358,7 @@ size_t pa_mixed_step_workspace_size(int32_t num_seqs, int64_t num_tokens, int32_
       make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true, num_seqs, true);
   if (!p.size_ok) return 0;
   return ws_layout(p.num_qrows, num_heads, cache->head_dim, p.head_groups, p.max_parts,
-                   p.max_tiles)
+                   p.max_tiles, p.num_sms)
       .total;
 }
 

@@ -43,44 +43,6 @@ def oracle_full(w, host):
     return slots, kb, vb, out, err_w | err_a, valid
 
 
-def oracle_rows(w, host_blocks, k_new, v_new, q, rows):
-    """Oracle for selected flattened query rows of a large workload.
-
-    host_blocks[b] = (k_blocks, v_blocks) float64 [n_b, bs, Hkv, D] copied from
-    the device pool right after generation (before any kernel ran) for every
-    request b that owns a sampled row.  k_new / v_new / q are CPU tensors of the
-    step's new tokens and queries.  Returns {row: [Hq, D] float64}.
-    """
-    qsl = w.query_start_loc
-    owner = np.searchsorted(qsl, np.asarray(rows), side="right") - 1
-    res = {}
-    for r, b in zip(rows, owner):
-        b = int(b)
-        kb, vb = host_blocks[b]
-        n = kb.shape[0]
-        table = np.arange(n, dtype=np.int32)[None, :]
-        t0, t1 = int(qsl[b]), int(qsl[b + 1])
-        q_b, L = t1 - t0, int(w.seq_lens[b])
-        slots = oracle.slot_mapping(table, [0, q_b], [L], w.block_size)
-        kk, vv, _ = oracle.cache_write(kb, vb, f64(k_new[t0:t1]), f64(v_new[t0:t1]), slots)
-        pos = L - q_b + (int(r) - t0)
-        K = oracle.gather(kk, table[0], pos + 1)
-        V = oracle.gather(vv, table[0], pos + 1)
-        res[int(r)] = oracle.attend_two_pass(f64(q[r:r + 1]), K, V, w.scale, pos)[0]
-    return res
-
-
-def snapshot_blocks(w, pools, seqs):
-    """Copy the blocks each request in `seqs` uses, as float64 on the host."""
-    k_cache, v_cache = pools
-    out = {}
-    for b in seqs:
-        n = (int(w.seq_lens[b]) + w.block_size - 1) // w.block_size
-        ids = torch.from_numpy(w.block_tables[b, :n].astype(np.int64)).to(k_cache.device)
-        out[int(b)] = (f64(k_cache.index_select(0, ids)), f64(v_cache.index_select(0, ids)))
-    return out
-
-
 def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
     err = np.abs(got - ref)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
@@ -112,3 +74,46 @@ def oracle_full_fp8(w, host):
     out, err_a, valid = oracle.paged_mixed_step(f64(host["q"]), k64, v64, w.block_tables, qsl,
                                                 w.seq_lens, w.scale)
     return slots, kc, vc, out, err_w | err_a, valid
+
+
+def device_blocks(w, pools, seqs):
+    """Device copies of the blocks each request in `seqs` uses, taken before
+    the step runs (the oracle applies the step's cache write itself).  Kept on
+    the device so that whole outputs of full-size workloads can be checked one
+    request at a time without holding every request's history on the host."""
+    k_cache, v_cache = pools
+    out = {}
+    for b in seqs:
+        n = (int(w.seq_lens[b]) + w.block_size - 1) // w.block_size
+        ids = torch.from_numpy(w.block_tables[b, :n].astype(np.int64)).to(k_cache.device)
+        out[int(b)] = (k_cache.index_select(0, ids), v_cache.index_select(0, ids))
+    return out
+
+
+def oracle_request(w, blocks, k_new, v_new, q, b, dequant=None):
+    """Oracle output of every query row of request b: [q_b, Hq, D] float64.
+
+    blocks = (k_blocks, v_blocks) of the request as copied before the step
+    (pool dtype, any device); k_new / v_new / q are CPU tensors of the step's
+    new tokens and queries.  The request's new tokens are written into its
+    blocks with the oracle's slot function and cache write, the history is
+    gathered through the (renumbered) block table, and all q_b queries attend
+    at once.  dequant(codes) turns e4m3 codes into float64 values."""
+    qsl = w.query_start_loc
+    kb, vb = blocks
+    t0, t1 = int(qsl[b]), int(qsl[b + 1])
+    q_b, L = t1 - t0, int(w.seq_lens[b])
+    n = kb.shape[0]
+    table = np.arange(n, dtype=np.int32)[None, :]
+    slots = oracle.slot_mapping(table, [0, q_b], [L], w.block_size)
+    if dequant is None:
+        kk, vv, _ = oracle.cache_write(f64(kb), f64(vb), f64(k_new[t0:t1]), f64(v_new[t0:t1]),
+                                       slots)
+    else:
+        kq = oracle.quantize(f64(k_new[t0:t1]).astype(np.float32), w.kv_scale)
+        vq = oracle.quantize(f64(v_new[t0:t1]).astype(np.float32), w.kv_scale)
+        kc, vc, _ = oracle.cache_write(fp8_codes(kb), fp8_codes(vb), kq, vq, slots)
+        kk, vv = dequant(kc), dequant(vc)
+    K = oracle.gather(kk, table[0], L)
+    V = oracle.gather(vv, table[0], L)
+    return oracle.attend_two_pass(f64(q[t0:t1]), K, V, w.scale, L - q_b)

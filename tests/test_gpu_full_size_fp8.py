@@ -8,8 +8,8 @@ Checked against the oracle, through the same step the benchmark times:
   * the codes of every written row, bit for bit against the oracle's
     quantisation of the new K/V rows;
   * a sample of unwritten rows, unchanged;
-  * attention on sampled requests, against the fp64 oracle over the pools'
-    dequantised values, within the bf16-input tolerance.
+  * attention on every row of every request, against the fp64 oracle over
+    the pools' dequantised values, within the bf16-input tolerance.
 
 The `late` mark runs this file after the parity suites.
 """
@@ -21,32 +21,19 @@ import torch
 import oracle
 import paged_kv_cache_434_b200 as P
 from paged_kv_cache_434_b200 import workloads as W
-from _util import assert_close, f64, oracle_rows
+from _util import assert_close, device_blocks, f64, oracle_request
 
 pytestmark = [pytest.mark.gpu, pytest.mark.late(1)]
 
 
-def _dequantised_blocks(w, pool_u8, seqs, table):
-    """The blocks each request of `seqs` uses, as the float64 values their
-    codes stand for (`table` holds the oracle's value of each of the 256 codes)."""
-    out = {}
-    for b in seqs:
-        n = (int(w.seq_lens[b]) + w.block_size - 1) // w.block_size
-        ids = torch.from_numpy(w.block_tables[b, :n].astype(np.int64)).to(pool_u8[0].device)
-        out[int(b)] = tuple(table[p.index_select(0, ids).cpu().numpy()] for p in pool_u8)
-    return out
-
-
-def _full_size_fp8(w, dev, sample_rows):
+def _full_size_fp8(w, dev, reqs):
     assert w.kv_dtype == "fp8"
     t = W.make_tensors(w, dev, where="device")
     idx = W.index_tensors(w, dev)
     Hkv, D = w.num_kv_heads, w.head_dim
     kc = t["k_cache"].view(torch.uint8)
     vc = t["v_cache"].view(torch.uint8)
-    table = oracle.dequantize(np.arange(256, dtype=np.uint8), w.kv_scale)
-    owners = sorted(set(np.searchsorted(w.query_start_loc, sample_rows, side="right") - 1))
-    blocks = _dequantised_blocks(w, (kc, vc), owners, table)
+    blocks = device_blocks(w, (t["k_cache"], t["v_cache"]), reqs)
     # untouched-row sample, taken before the step
     gen = np.random.default_rng(99)
     probe = torch.from_numpy(gen.integers(0, w.num_blocks * w.block_size, 4096)).to(dev)
@@ -72,20 +59,22 @@ def _full_size_fp8(w, dev, sample_rows):
     keep = torch.tensor([i for i, s in enumerate(probe.tolist()) if s not in written], device=dev)
     assert torch.equal(kc_rows.index_select(0, probe)[keep], before[keep])
 
-    # the new rows enter attention as the values of their codes
-    k_new = torch.from_numpy(table[k_codes])
-    v_new = torch.from_numpy(table[v_codes])
-    ref = oracle_rows(w, blocks, k_new, v_new, t["q"].cpu(), sample_rows)
-    got = f64(out[torch.tensor(sample_rows, device=dev)])
-    return assert_close(got, np.stack([ref[r] for r in sample_rows]), "bf16", w.name)
+    # every row of the chosen requests; the oracle quantises the new rows and
+    # attends over the values the codes stand for
+    k_new, v_new, q = t["k_new"].cpu(), t["v_new"].cpu(), t["q"].cpu()
+    qsl = w.query_start_loc
+    got, ref = [], []
+    for b in reqs:
+        ref.append(oracle_request(w, blocks.pop(int(b)), k_new, v_new, q, int(b),
+                                  dequant=lambda c: oracle.dequantize(c, w.kv_scale)))
+        got.append(f64(out[int(qsl[b]):int(qsl[b + 1])]))
+    return assert_close(np.concatenate(got), np.concatenate(ref), "bf16", w.name)
 
 
 def test_full_llama8b_decode_fp8(cuda_device):
     w = W.llama8b_decode_fp8(0)
-    rows = sorted({0, 1, int(np.argmax(w.seq_lens)), int(np.argmin(w.seq_lens)), 63})
-    _full_size_fp8(w, cuda_device, rows)
+    _full_size_fp8(w, cuda_device, range(w.num_seqs))     # all 64 requests
 
 
 def test_full_long_context_fp8(cuda_device):
-    # the shortest (32K) and the longest (128K) request
-    _full_size_fp8(W.long_context_decode_fp8(0), cuda_device, [0, 3])
+    _full_size_fp8(W.long_context_decode_fp8(0), cuda_device, [0, 1, 2, 3])

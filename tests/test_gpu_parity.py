@@ -11,7 +11,7 @@ import oracle
 import paged_kv_cache_434_b200 as P
 from paged_kv_cache_434_b200 import workloads as W
 
-from _util import assert_close, bits, f64, oracle_full, oracle_rows, snapshot_blocks
+from _util import assert_close, bits, device_blocks, f64, oracle_full, oracle_request
 
 pytestmark = pytest.mark.gpu
 
@@ -258,13 +258,13 @@ def test_error_bits_bad_inputs(cuda_device):
 
 # ---------------------------------------------------------------- full-size workloads
 
-def _full_size(w, dev, sample_rows, out_dtype=torch.float32):
-    """Run a full-size workload through the step; check slots/writes by
-    properties that hold at any size and attention on sampled rows."""
+def _full_size(w, dev, reqs, out_dtype=torch.float32):
+    """Run a full-size workload through the step; check slots and cache writes
+    by properties that hold at any size, and EVERY output row of the requests
+    in `reqs` against the oracle, element by element."""
     t = W.make_tensors(w, dev, where="device")
     idx = W.index_tensors(w, dev)
-    owners = sorted(set(np.searchsorted(w.query_start_loc, sample_rows, side="right") - 1))
-    blocks = snapshot_blocks(w, (t["k_cache"], t["v_cache"]), owners)
+    blocks = device_blocks(w, (t["k_cache"], t["v_cache"]), reqs)
     # untouched-slot sample, taken before the step
     gen = np.random.default_rng(99)
     probe = torch.from_numpy(gen.integers(0, w.num_blocks * w.block_size, 4096)).to(dev)
@@ -288,17 +288,19 @@ def _full_size(w, dev, sample_rows, out_dtype=torch.float32):
     written = set(ref_slots.tolist())
     keep = torch.tensor([i for i, s in enumerate(probe.tolist()) if s not in written], device=dev)
     assert torch.equal(kc_flat.index_select(0, probe)[keep], before[keep])
-    # attention on sampled rows
-    ref = oracle_rows(w, blocks, t["k_new"].cpu(), t["v_new"].cpu(), t["q"].cpu(), sample_rows)
-    got = f64(out[torch.tensor(sample_rows, device=dev)])
-    refm = np.stack([ref[r] for r in sample_rows])
-    return assert_close(got, refm, w.dtype, w.name), out
+    # attention: every row of the chosen requests
+    k_new, v_new, q = t["k_new"].cpu(), t["v_new"].cpu(), t["q"].cpu()
+    qsl = w.query_start_loc
+    got, ref = [], []
+    for b in reqs:
+        ref.append(oracle_request(w, blocks.pop(int(b)), k_new, v_new, q, int(b)))
+        got.append(f64(out[int(qsl[b]):int(qsl[b + 1])]))
+    return assert_close(np.concatenate(got), np.concatenate(ref), w.dtype, w.name), out
 
 
 def test_full_llama8b_decode(cuda_device):
     w = W.llama8b_decode(0)
-    rows = [0, 1, int(np.argmax(w.seq_lens)), int(np.argmin(w.seq_lens)), 63]
-    _full_size(w, cuda_device, rows)
+    _full_size(w, cuda_device, range(w.num_seqs))          # all 64 requests
 
 
 def test_full_long_context_split_kv(cuda_device):
@@ -307,22 +309,27 @@ def test_full_long_context_split_kv(cuda_device):
 
 def test_full_shared_prefix_decode(cuda_device):
     w = W.shared_prefix_decode(0)
-    _full_size(w, cuda_device, [0, 17, 64, 127])
+    _full_size(w, cuda_device, range(w.num_seqs))          # all 128 requests
 
 
+def _mixed_requests(w, n_decode=256, seed=7):
+    """Both prefill chunks (every one of their 4096 rows) and n_decode decode
+    requests drawn by a seeded generator."""
+    big = [b for b in range(w.num_seqs) if w.query_lens[b] > 1]
+    dec = [b for b in range(w.num_seqs) if w.query_lens[b] == 1]
+    pick = np.random.default_rng(seed).choice(dec, size=n_decode, replace=False)
+    return sorted(big + [int(b) for b in pick])
+
+
+@pytest.mark.late(1)
 def test_full_mixed_step(cuda_device):
     w = W.mixed_step(0)
-    # chunk A (prefix 4096): first, middle, last query; chunk B: first, last; decodes
-    rows = [0, 1, 1023, 2047, 2048, 2049, 4095, 4096, 6000, 8191]
-    _full_size(w, cuda_device, rows)
+    reqs = _mixed_requests(w)
+    assert sum(int(w.query_lens[b]) for b in reqs) == 4096 + 256
+    _full_size(w, cuda_device, reqs)
 
 
+@pytest.mark.late(1)
 def test_full_mixed_step_shuffled(cuda_device):
     w = W.mixed_step(1, shuffle=True)
-    qsl = w.query_start_loc
-    big = [b for b in range(w.num_seqs) if w.query_lens[b] > 1]
-    rows = []
-    for b in big:
-        rows += [int(qsl[b]), int(qsl[b]) + 1, int(qsl[b + 1]) - 1]
-    rows += [int(qsl[5]), int(qsl[w.num_seqs - 1])]
-    _full_size(w, cuda_device, sorted(set(rows)))
+    _full_size(w, cuda_device, _mixed_requests(w, seed=8))
