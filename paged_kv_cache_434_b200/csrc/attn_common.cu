@@ -29,7 +29,7 @@ namespace pa {
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 WsLayout ws_layout(int64_t num_qrows, int num_heads, int head_dim, int head_groups,
-                   int64_t max_parts, int64_t max_tiles, int max_ctas) {
+                   int64_t max_parts, int64_t max_tiles) {
   WsLayout L{};
   L.num_qrows = num_qrows;
   L.max_parts = max_parts;
@@ -54,11 +54,6 @@ WsLayout ws_layout(int64_t num_qrows, int num_heads, int head_dim, int head_grou
   off = align_up(off + num_qrows * num_heads * max_parts * head_dim * sizeof(float), 256);
   L.tiles = off;
   off = align_up(off + max_tiles * sizeof(int4), 256);
-  L.max_ctas = max_ctas;
-  L.sk = off;
-  off = align_up(off + static_cast<size_t>(max_ctas) * sizeof(int4), 256);
-  L.row_ustart = off;
-  off = align_up(off + num_qrows * sizeof(int64_t), 256);
   L.total = off;
   return L;
 }
@@ -75,9 +70,6 @@ WsView ws_view(void* base, const WsLayout& L) {
   v.part_ml = reinterpret_cast<float2*>(p + L.part_ml);
   v.part_o = reinterpret_cast<float*>(p + L.part_o);
   v.tiles = reinterpret_cast<int4*>(p + L.tiles);
-  v.sk = reinterpret_cast<int4*>(p + L.sk);
-  v.row_ustart = reinterpret_cast<int64_t*>(p + L.row_ustart);
-  v.max_ctas = static_cast<int32_t>(L.max_ctas);
   v.max_parts = L.max_parts;
   v.max_items = L.max_items;
   v.max_tiles = L.max_tiles;
@@ -201,23 +193,27 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T* s_scan, T* total) {
 
 // Decode batches of up to kFastRows requests, in one pass: each thread holds
 // up to kFastPerThread consecutive requests' lengths in registers, so the
-// partition plan needs no re-reads of the workspace and few barriers.
-//   * Balanced ranges (no tiles beside the batch, one head group per row):
-//     the units are cut into num_sms ranges of equal work; CTA c streams range
-//     c, so every CTA ends at the same time and a row is split only where a
-//     range boundary falls inside it (its pieces are its partitions).  Taken
-//     when no row is cut into more pieces than the partial slots hold.
-//   * Otherwise rows are cut into uniform partitions of P stages, and the
-//     items are listed by the whole CTA (item i finds its row by binary search
-//     over the rows' first items).
-// Returns false, having written nothing, when every block table starts with
-// the same block and the batch qualifies for the shared-prefix cascade: the
-// general planner then looks for the prefix.
+// plan needs no re-reads of the workspace and few barriers.
+//   * Shared prefix (batches of >= kCascadeMinSeqs requests whose tables all
+//     start with the same block): the longest common run of leading blocks is
+//     found by comparing (request, column) pairs against row 0 in shared
+//     memory; a run of >= kCascadeMinPrefix tokens is attended by tensor-core
+//     tiles (listed here) and the rows keep only their suffix.
+//   * Partitions in decreasing sizes: work W = stages x head groups; each row
+//     is cut into big pieces of Pb ~ 0.85 W / (2 SMs) stages (85 % of its
+//     stages, whole pieces only) and small pieces of Pb / 4 for the rest.
+//     The item list holds every big piece before every small one, and the
+//     partition kernel takes items in list order from a global counter: the
+//     big pieces spread the work, the small ones even out the end, whatever
+//     the SMs' start times and streaming rates.  Rows that would need more
+//     pieces than the partial slots hold fall back to uniform pieces.
+//   * Items are written by the whole CTA: item i finds its row by binary
+//     search over the rows' first items in shared memory.
 constexpr int kFastPerThread = 4;
 constexpr int kFastRows = kPlanThreads * kFastPerThread;
 
-__device__ bool plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsView& ws,
-                                 int* s_rowpos, int* s_scan, long long* s_scan64,
+__device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsView& ws,
+                                 int* s_rowpos, int* s_ref, int ref_cap, int* s_scan,
                                  long long* s_sum, int* s_max, int* s_P, int* s_merge,
                                  int* s_merge_big) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -248,9 +244,48 @@ __device__ bool plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
     same &= c0[k] == ref0;
     if (ok) min_len = min(min_len, L[k]);
   }
-  if (look_shared &&
-      __syncthreads_and(same && all_ok && (min_len == 0x7fffffff || min_len > kCascadeMinPrefix)))
-    return false;
+
+  // Shared prefix: row 0's entries go to shared memory; the (request, column)
+  // pairs are compared column chunk by column chunk, about eight loads per
+  // thread per chunk, until a chunk holds a mismatch.  The run is limited so
+  // that each request keeps at least one key of its own.
+  __shared__ int s_first, s_minlen;
+  int prefix_blocks = 0;
+  if (look_shared) {
+    const int w_min = __reduce_min_sync(0xffffffffu, all_ok ? min_len : 0);
+    if (tid == 0) s_minlen = 0x7fffffff;
+    __syncthreads();
+    if (lane == 0) atomicMin(&s_minlen, w_min);
+    const bool cand = __syncthreads_and(same && all_ok) && s_minlen > kCascadeMinPrefix &&
+                      s_minlen != 0x7fffffff;
+    if (cand) {
+      const int max_cols = min(min((s_minlen - 1) / g.block_size, g.max_blocks), ref_cap);
+      for (int c = tid; c < max_cols; c += kPlanThreads) s_ref[c] = g.block_tables[c];
+      if (tid == 0) s_first = max_cols;
+      __syncthreads();
+      const int W = max(1, 8 * kPlanThreads / B);  // columns per chunk
+      for (int cb = 1; cb < max_cols; cb += W) {
+        const int ce = min(cb + W, max_cols), wc = ce - cb;
+        int mine = 0x7fffffff;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int idx = tid + k * kPlanThreads;
+          if (idx < wc * B) {
+            const int b = idx / wc, j = cb + idx % wc;
+            if (g.block_tables[static_cast<int64_t>(b) * g.max_blocks + j] != s_ref[j])
+              mine = min(mine, j);
+          }
+        }
+        mine = __reduce_min_sync(0xffffffffu, mine);
+        if (lane == 0 && mine != 0x7fffffff) atomicMin(&s_first, mine);
+        __syncthreads();
+        if (s_first < ce) break;  // s_first only falls: every thread sees the same answer
+      }
+      const int pb = s_first;
+      if (pb * g.block_size >= kCascadeMinPrefix) prefix_blocks = pb;
+    }
+  }
+  const int prefix = prefix_blocks * g.block_size;
 
   // invalid requests: error bits, rows left unwritten (L = -1 from here on)
   long long units_sum = 0;
@@ -266,7 +301,7 @@ __device__ bool plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
       L[k] = -1;
       continue;
     }
-    const int units = (L[k] + kStageTokens - 1) / kStageTokens;
+    const int units = (L[k] - prefix + kStageTokens - 1) / kStageTokens;
     units_sum += units;
     units_max = max(units_max, units);
   }
@@ -279,7 +314,7 @@ __device__ bool plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
     s_sum[warp] = units_sum;
     s_max[warp] = units_max;
   }
-  __shared__ long long s_total;
+  __shared__ int s_Pb, s_Ps;
   __syncthreads();
   const long long cap =
       max(1LL, static_cast<long long>(ws.max_parts) - (a.cascade ? kMaxPrefixChunks : 0));
@@ -290,97 +325,127 @@ __device__ bool plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
       total += s_sum[w];
       mx = max(mx, s_max[w]);
     }
-    s_total = total;
-    const long long by_target =
-        (total * a.head_groups + a.target_items - 1) / max(a.target_items, 1);
+    const long long work = total * a.head_groups;
+    const long long by_target = (work + a.target_items - 1) / max(a.target_items, 1);
     const long long by_cap = (mx + cap - 1) / cap;
     const long long P = max(static_cast<long long>(a.min_part_stages), max(by_target, by_cap));
-    *s_P = static_cast<int>(max(P, 1LL));
+    *s_P = static_cast<int>(min(max(P, 1LL), static_cast<long long>(kMaxItemStages)));
+    const long long pb = max(static_cast<long long>(a.min_part_stages),
+                             work * 85 / (100 * 2 * max(a.num_sms, 1)));
+    s_Pb = static_cast<int>(min(pb, static_cast<long long>(kMaxItemStages)));
+    s_Ps = max(a.min_part_stages, s_Pb / 4);
     *s_merge = 0;
     *s_merge_big = 0;
   }
   __syncthreads();
-  const int P = *s_P;
-  const long long U = s_total;
-  const int C = a.num_sms;
-
-  // pieces of each row: balanced ranges, if every row fits the partial slots
-  int np[kFastPerThread];
-  long long us0 = 0;
-  bool balanced = a.balanced && a.head_groups == 1 && U > 0 && C <= ws.max_ctas;
-  if (balanced) {
-    long long my_units = 0;
-#pragma unroll
-    for (int k = 0; k < kFastPerThread; ++k)
-      if (k < per && r0 + k < B && L[k] > 0) my_units += (L[k] + kStageTokens - 1) / kStageTokens;
-    long long dummy;
-    us0 = block_exclusive_scan<long long>(my_units, s_scan64, &dummy);
-    bool fits = U / C < (1LL << 30);
-    long long us = us0;
+  // pieces per row: big + small, unless some row would need too many
+  int nb[kFastPerThread], ns[kFastPerThread];
+  bool fits = true;
+  {
+    const int Pb = s_Pb, Ps = s_Ps;
 #pragma unroll
     for (int k = 0; k < kFastPerThread; ++k) {
-      np[k] = -1;
+      nb[k] = ns[k] = 0;
       if (k >= per || r0 + k >= B || L[k] < 0) continue;
-      const long long n_st = (L[k] + kStageTokens - 1) / kStageTokens;
-      np[k] = n_st == 0 ? 0 : range_of(us + n_st - 1, U, C) - range_of(us, U, C) + 1;
-      fits &= np[k] <= cap;
-      us += n_st;
+      const int n = (L[k] - prefix + kStageTokens - 1) / kStageTokens;
+      nb[k] = static_cast<int>(static_cast<long long>(n) * 85 / 100 / Pb);
+      ns[k] = (n - nb[k] * Pb + Ps - 1) / Ps;
+      fits &= nb[k] + ns[k] <= cap;
     }
-    balanced = __syncthreads_and(fits);
   }
-  if (balanced) {
-    long long us = us0;
+  const bool guided = __syncthreads_and(fits);
+  const int Pb = guided ? s_Pb : *s_P, Ps = guided ? s_Ps : *s_P;
+  if (!guided) {
 #pragma unroll
     for (int k = 0; k < kFastPerThread; ++k) {
-      const int r = r0 + k;
-      if (k >= per || r >= B) continue;
-      ws.row_ustart[r] = us;
-      if (L[k] < 0) continue;
-      const long long n_st = (L[k] + kStageTokens - 1) / kStageTokens;
-      const long long ue = us + n_st;
-      // the ranges that start inside this row
-      for (long long c = (us * C + U - 1) / U; c < C; ++c) {
-        const long long x = range_start(c, U, C);
-        if (x >= ue) break;
-        ws.sk[c] = make_int4(r, 0, static_cast<int>(x - us),
-                             static_cast<int>(range_start(c + 1, U, C) - x));
-      }
-      us = ue;
-    }
-  } else {
-    int my_items = 0;
-#pragma unroll
-    for (int k = 0; k < kFastPerThread; ++k) {
-      np[k] = -1;
+      nb[k] = 0;
       if (k >= per || r0 + k >= B || L[k] < 0) continue;
-      const int units = (L[k] + kStageTokens - 1) / kStageTokens;
-      np[k] = (units + P - 1) / P;
-      my_items += np[k] * a.head_groups;
+      ns[k] = ((L[k] - prefix + kStageTokens - 1) / kStageTokens + Ps - 1) / Ps;
     }
-    int n_items = 0;
-    int pos = block_exclusive_scan<int>(my_items, s_scan, &n_items);
+  }
+  // item positions: every big piece first, then every small piece
+  int my_big = 0, my_small = 0;
+#pragma unroll
+  for (int k = 0; k < kFastPerThread; ++k) {
+    my_big += nb[k] * a.head_groups;
+    my_small += ns[k] * a.head_groups;
+  }
+  int n_big = 0, n_small = 0;
+  const int big0 = block_exclusive_scan<int>(my_big, s_scan, &n_big);
+  const int small0 = block_exclusive_scan<int>(my_small, s_scan, &n_small);
+  // big items, spread over the CTA by binary search over the rows' first items
+  {
+    int pos = big0;
 #pragma unroll
     for (int k = 0; k < kFastPerThread; ++k) {
       const int r = r0 + k;
       if (k >= per || r >= B) continue;
       s_rowpos[r] = pos;
-      if (np[k] > 0) pos += np[k] * a.head_groups;
+      pos += nb[k] * a.head_groups;
     }
-    if (tid == 0) {
-      s_rowpos[B] = n_items;
-      ws.ctrl[1] = n_items;
-    }
+    if (tid == 0) s_rowpos[B] = n_big;
     __syncthreads();
-    // items {row, head group, partition}, row-major, spread over the CTA
-    for (int i = tid; i < n_items; i += kPlanThreads) {
+    for (int i = tid; i < n_big; i += kPlanThreads) {
       int lo = 0, hi = B;  // the row r with s_rowpos[r] <= i < s_rowpos[r + 1]
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (s_rowpos[mid] <= i) lo = mid;
         else hi = mid;
       }
-      const int k = i - s_rowpos[lo];
-      ws.items[i] = make_int4(lo, k % a.head_groups, k / a.head_groups, 0);
+      const int k = i - s_rowpos[lo], piece = k / a.head_groups;
+      ws.items[i] = make_int4(lo, (k % a.head_groups) | (Pb << kItemSizeShift), piece,
+                              piece * Pb);
+    }
+    __syncthreads();
+  }
+  // small items, after them
+  {
+    int pos = small0;
+#pragma unroll
+    for (int k = 0; k < kFastPerThread; ++k) {
+      const int r = r0 + k;
+      if (k >= per || r >= B) continue;
+      s_rowpos[r] = pos;
+      pos += ns[k] * a.head_groups;
+    }
+    if (tid == 0) s_rowpos[B] = n_small;
+    __syncthreads();
+    for (int i = tid; i < n_small; i += kPlanThreads) {
+      int lo = 0, hi = B;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_rowpos[mid] <= i) lo = mid;
+        else hi = mid;
+      }
+      const int row = lo, k = i - s_rowpos[row], piece = k / a.head_groups;
+      // the row's big pieces, from the owning thread's registers, are not at
+      // hand here: recompute them from its length
+      const int Lr = g.seq_lens[row];
+      const int n = (Lr - prefix + kStageTokens - 1) / kStageTokens;
+      const int nbr = guided ? static_cast<int>(static_cast<long long>(n) * 85 / 100 / Pb) : 0;
+      ws.items[n_big + i] =
+          make_int4(row, (k % a.head_groups) | (Ps << kItemSizeShift), nbr + piece,
+                    nbr * Pb + piece * Ps);
+    }
+  }
+  // shared-prefix tiles: groups of tile_tokens requests x one KV head x a
+  // chunk of the prefix keys, at most one tile per two SMs, so that the suffix
+  // partitions start at once on the SMs the tiles leave free (longer tiles on
+  // half the SMs measured 11 % faster than one wave of shorter tiles)
+  int prefix_chunks = 0, n_tiles = 0;
+  if (prefix > 0) {
+    const int per_tile = a.tile_tokens;
+    const int groups = (B + per_tile - 1) / per_tile;
+    const int kv_tiles = (prefix + 127) / 128;
+    const int base = groups * g.num_kv_heads;
+    const int want = min(min(kMaxPrefixChunks, kv_tiles), max(1, a.num_sms / (2 * base)));
+    const int per_chunk = (kv_tiles + want - 1) / want;
+    prefix_chunks = (kv_tiles + per_chunk - 1) / per_chunk;  // no empty chunk
+    n_tiles = static_cast<int>(min(static_cast<int64_t>(base) * prefix_chunks, ws.max_tiles));
+    for (int idx = tid; idx < n_tiles; idx += kPlanThreads) {
+      const int c = idx / base, rest = idx % base;
+      const int grp = rest / g.num_kv_heads, hk = rest % g.num_kv_heads;
+      ws.tiles[idx] = make_int4(grp * per_tile, hk, min(per_tile, B - grp * per_tile), c);
     }
   }
   // rows: info, partition counts, and the merge pass's list (rows with no key
@@ -389,29 +454,26 @@ __device__ bool plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
   for (int k = 0; k < kFastPerThread; ++k) {
     const int r = r0 + k;
     if (k >= per || r >= B) continue;
+    const int n = L[k] < 0 ? -1 : nb[k] + ns[k] + (prefix > 0 ? prefix_chunks : 0);
     ws.qrow_bad[r] = 0;
-    ws.nparts[r] = np[k];
-    ws.qrow_info[r] = np[k] >= 0 ? make_int4(r, L[k], 1, 0) : make_int4(-1, 0, 0, 0);
-    if (np[k] > 32) ws.merge_rows[g.num_qrows - 1 - atomicAdd(s_merge_big, 1)] = r;
-    else if (np[k] >= 0 && np[k] != 1) ws.merge_rows[atomicAdd(s_merge, 1)] = r;
+    ws.nparts[r] = n;
+    ws.qrow_info[r] = n >= 0 ? make_int4(r, L[k], 1, prefix) : make_int4(-1, 0, 0, 0);
+    if (n > 32) ws.merge_rows[g.num_qrows - 1 - atomicAdd(s_merge_big, 1)] = r;
+    else if (n >= 0 && n != 1) ws.merge_rows[atomicAdd(s_merge, 1)] = r;
   }
   __syncthreads();
   if (tid == 0) {
     ws.ctrl[0] = 0;
-    if (balanced) ws.ctrl[1] = 0;
-    ws.ctrl[2] = P * kStageTokens;
+    ws.ctrl[1] = n_big + n_small;
+    ws.ctrl[2] = Pb * kStageTokens;
     ws.ctrl[3] = 0;
-    ws.ctrl[4] = 0;  // no tiles, no shared prefix
+    ws.ctrl[4] = n_tiles;
     ws.ctrl[5] = *s_merge;
-    ws.ctrl[6] = 0;
-    ws.ctrl[7] = 0;
-    ws.ctrl[8] = 0;
+    ws.ctrl[6] = prefix;
+    ws.ctrl[7] = prefix_chunks;
+    ws.ctrl[8] = prefix > 0 ? a.num_sms : 0;  // every tile CTA works
     ws.ctrl[9] = *s_merge_big;
-    ws.ctrl[10] = balanced ? C : 0;
-    ws.ctrl[11] = balanced ? static_cast<int>(U & 0xffffffffLL) : 0;
-    ws.ctrl[12] = balanced ? static_cast<int>(U >> 32) : 0;
   }
-  return true;
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs a, WsView ws) {
@@ -434,10 +496,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
 
   if (decode_mode && g.num_seqs <= kFastRows && g.num_qrows == g.num_seqs) {
     __shared__ int s_scan33[33];
-    __shared__ long long s_scan64[33];
-    if (plan_decode_fast(g, a, ws, s_rowpos, s_scan33, s_scan64, s_sum, s_max, &s_P, &s_merge,
-                         &s_merge_big))
-      return;
+    plan_decode_fast(g, a, ws, s_rowpos, s_hist, kTileBins, s_scan33, s_sum, s_max, &s_P,
+                     &s_merge, &s_merge_big);
+    return;
   }
 
   // 0. rows no request covers stay unwritten
@@ -637,7 +698,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
         max(1LL, static_cast<long long>(ws.max_parts) - (a.cascade ? kMaxPrefixChunks : 0));
     long long by_cap = (mx + cap - 1) / cap;
     long long P = max(static_cast<long long>(a.min_part_stages), max(by_target, by_cap));
-    s_P = static_cast<int>(max(P, 1LL));
+    s_P = static_cast<int>(min(max(P, 1LL), static_cast<long long>(kMaxItemStages)));
     // CTAs the tensor-core tiles run on.  With decode partitions in the same
     // call, the tiles take only as many SMs as finish them in about half the
     // time the (HBM-bound) partitions need, and the partitions start at once
@@ -718,7 +779,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
       }
     }
     for (int p = 0; p < np; ++p)
-      for (int hg = 0; hg < a.head_groups; ++hg) ws.items[pos++] = make_int4(r, hg, p, 0);
+      for (int hg = 0; hg < a.head_groups; ++hg)
+        ws.items[pos++] = make_int4(r, hg | (P << kItemSizeShift), p, p * P);
   }
   __syncthreads();
   const int nbig_rows = min(s_nbig, kMaxBig);
@@ -728,7 +790,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     const int units = (info.y - info.w + kStageTokens - 1) / kStageTokens;
     const int n_it = (units + P - 1) / P * a.head_groups;
     for (int i = tid; i < n_it; i += kPlanThreads)
-      ws.items[s_bigpos[k] + i] = make_int4(r, i % a.head_groups, i / a.head_groups, 0);
+      ws.items[s_bigpos[k] + i] = make_int4(r, (i % a.head_groups) | (P << kItemSizeShift),
+                                            i / a.head_groups, (i / a.head_groups) * P);
   }
 
   // 4. tiles, longest first
@@ -784,7 +847,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     ws.ctrl[6] = prefix_tokens;
     ws.ctrl[7] = prefix_chunks;
     ws.ctrl[8] = s_ntc;
-    ws.ctrl[10] = 0;  // items from the list
   }
 }
 
@@ -860,7 +922,6 @@ __global__ void __launch_bounds__(kGenWarps * 32) attn_generic_kernel(AttnGeom g
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = g.num_heads / g.num_kv_heads;
   const int n_items = ws.ctrl[1];
-  const int P = ws.ctrl[2];
   using QT = typename QueryType<T>::type;
   const QT* q = static_cast<const QT*>(g.q);
   const T* kc = static_cast<const T*>(g.k_cache);
@@ -875,10 +936,11 @@ __global__ void __launch_bounds__(kGenWarps * 32) attn_generic_kernel(AttnGeom g
     const int it = s_item;
     if (it >= n_items) break;
     const int4 item = ws.items[it];
-    const int r = item.x, hk = item.y, p = item.z;
+    const int r = item.x, hk = item.y & kItemHgMask, p = item.z;
     const int4 info = ws.qrow_info[r];
     const int b = info.x, key_len = info.y;
-    const int lo = info.w + p * P, hi = min(lo + P, key_len);
+    const int lo = info.w + item.w * kStageTokens;
+    const int hi = min(lo + (item.y >> kItemSizeShift) * kStageTokens, key_len);
     for (int idx = tid; idx < G * D; idx += blockDim.x) {
       const int gq = idx / D, d = idx % D;
       s_q[gq][d] = to_f32(q[(static_cast<int64_t>(r) * g.num_heads + hk * G + gq) * D + d]);
@@ -1001,10 +1063,10 @@ cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms
 // planner's list.  Pass 1: one warp per (row, query head) whose partitions fit
 // in a warp (<= 32): lane k holds partition k's (m, l), the weights
 // 2^(m_k - M) are shuffled to all lanes and each lane accumulates D/32 output
-// columns.  Pass 2: one 8-warp CTA per remaining (row, head): max and
+// columns.  Pass 2: one 16-warp CTA per remaining (row, head): max and
 // denominator reduced over the CTA, then each warp accumulates every 8th
 // partition (4 in flight) and the warp sums are combined.
-constexpr int kMergeWarps = 8;
+constexpr int kMergeWarps = 16;
 constexpr int kMergeCached = 2048;  // partition weights kept in shared memory
 
 template <int D>
@@ -1157,9 +1219,11 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(AttnGeom g, WsV
 }
 
 cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {
+  // one CTA of 16 warps per SM, warps looping over the pairs: a grid of
+  // eight small CTAs per SM took ~10 us just to be launched
   int64_t blocks = static_cast<int64_t>(g.num_qrows) * g.num_heads;
   if (blocks == 0) return cudaSuccess;
-  if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > num_sms) blocks = num_sms;
   const dim3 grid(static_cast<unsigned>(blocks)), block(kMergeWarps * 32);
   if (g.head_dim == 64) return launch_pdl<merge_kernel<64>>(grid, block, 0, s, g, ws);
   return launch_pdl<merge_kernel<128>>(grid, block, 0, s, g, ws);

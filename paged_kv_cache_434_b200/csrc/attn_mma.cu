@@ -53,21 +53,23 @@ struct StageInfo {
 // per head and tensor (one 128-byte swizzled row per key, the same 2 KiB tile
 // size).  K fragments are widened in registers straight from an ldmatrix of
 // the codes (the dimension order inside each 16-dim step is permuted, and the
-// query fragments follow the same order); V codes are widened to f16 in a
-// scratch of the warp's own, laid out as the bf16 path's two [16 x 64]
-// halves, for the transposed loads of the P V product.
+// query fragments follow the same order).  V fragments come from a transposed
+// ldmatrix of the codes too: a lane receives the code pairs (dims 2g, 2g+1)
+// of keys 2t and 2t+1, and one byte permute turns them into the key pairs of
+// dim 2g and of dim 2g+1 -- the B operands of two n8 tiles that hold the even
+// and the odd dims of a 16-dim chunk.  The output rows are put back in dim
+// order when they are stored.
 template <int D, int HG, bool F8 = false>
 struct Cfg {
   static constexpr int NH = F8 ? 1 : D / 64;            // tiles per head and tensor in a stage
   static constexpr int kTile = 2048;                    // [16 keys x 128 bytes]
   static constexpr int kTensorBytes = HG * NH * kTile;  // K (or V) part of a stage
   static constexpr int kStageBytes = 2 * kTensorBytes;
-  static constexpr int kScratch = F8 ? HG * (D / 64) * kTile : 0;  // f16 V per warp
-  static constexpr int kBudget = 200 * 1024 - kScratch;
+  static constexpr int kBudget = 200 * 1024;
   static constexpr int NS0 = kBudget / kStageBytes;
   static constexpr int NS = NS0 > 6 ? 6 : (NS0 < 2 ? 2 : NS0);
   static constexpr int kThreads = (HG + 1) * 32;
-  static constexpr int kSmem = NS * kStageBytes + kScratch + 1024 /*align*/ + 1024 /*info+bars*/;
+  static constexpr int kSmem = NS * kStageBytes + 1024 /*align*/ + 1024 /*info+bars*/;
 };
 
 // byte offset of (key, 16-byte chunk) inside one 128B-swizzled [16 x 64] tile
@@ -89,9 +91,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* stages = smem;
-  uint8_t* scratch = smem + NS * C::kStageBytes;  // F8: f16 V tiles, 4 KiB per warp
-  mmak::StageInfo* info =
-      reinterpret_cast<mmak::StageInfo*>(smem + NS * C::kStageBytes + C::kScratch);
+  mmak::StageInfo* info = reinterpret_cast<mmak::StageInfo*>(smem + NS * C::kStageBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(info + NS);
   uint64_t* empty = full + NS;
   __shared__ int s_abort;
@@ -118,7 +118,6 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   if (!after_tiles) grid_dependency_wait();
 
   const int n_items = __ldcg(&ws.ctrl[1]);
-  const int P = __ldcg(&ws.ctrl[2]);
   const int G = g.num_heads / g.num_kv_heads;
 
   if (warp == HG) {
@@ -129,64 +128,23 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     uint32_t phase = 0;
     int round = 0;  // completed passes over the ring
     bool ok = true;
-    // Work source: this CTA's balanced range of (row, stage) units when the
-    // planner cut the batch into ranges (C > 0), else items taken from the
-    // planner's list one at a time.
-    const int C = __ldcg(&ws.ctrl[10]);
-    const long long U = static_cast<long long>(static_cast<unsigned>(__ldcg(&ws.ctrl[11]))) |
-                        (static_cast<long long>(__ldcg(&ws.ctrl[12])) << 32);
-    int sk_r = 0, sk_s = 0, sk_left = 0;
-    if (C > 0 && static_cast<int>(blockIdx.x) < C) {
-      const int4 st = __ldcg(&ws.sk[blockIdx.x]);
-      sk_r = st.x, sk_s = st.z, sk_left = st.w;
-    }
     for (;;) {
-      bool done;
+      const int it = atomicAdd(&ws.ctrl[0], 1);
+      const bool done = it >= n_items;
       int4 item = make_int4(0, 0, 0, 0), qi = make_int4(0, 0, 0, 0);
-      int lo, hi, np = 1;
-      if (C > 0) {
-        // the next piece of the range: stages [sk_s, sk_s + take) of row sk_r
-        int n_st = 0, take = 0;
-        done = sk_left <= 0;
-        while (!done) {
-          qi = __ldcg(&ws.qrow_info[sk_r]);
-          n_st = qi.z ? (qi.y - qi.w + kStageTokens - 1) / kStageTokens : 0;
-          if (sk_s < n_st) {
-            take = min(sk_left, n_st - sk_s);
-            break;
-          }
-          sk_s = 0;  // a row without (more) units: the next row
-          if (++sk_r >= g.num_qrows) done = true;
-        }
-        if (!done) {
-          const long long u0 = __ldcg(&ws.row_ustart[sk_r]);
-          const int cf = range_of(u0, U, C);
-          np = range_of(u0 + n_st - 1, U, C) - cf + 1;
-          item = make_int4(sk_r, 0, static_cast<int>(blockIdx.x) - cf, 0);
-          lo = qi.w + sk_s * kStageTokens;
-          hi = min(min(lo + take * kStageTokens, qi.y), g.max_blocks * g.block_size);
-          sk_left -= take;
-          sk_s += take;
-          if (sk_s == n_st) {
-            sk_s = 0;
-            ++sk_r;
-          }
-        } else {
-          lo = 0;
-          hi = 1;
-        }
-      } else {
-        const int it = atomicAdd(&ws.ctrl[0], 1);
-        done = it >= n_items;
-        if (!done) {
-          item = __ldcg(&ws.items[it]);
-          qi = __ldcg(&ws.qrow_info[item.x]);
-          np = __ldcg(&ws.nparts[item.x]);
-        }
-        lo = qi.w + item.z * P;  // partitions start after a shared prefix
-        // lo >= hi: empty item, skipped; never past the table
-        hi = done ? lo + 1 : min(min(lo + P, qi.y), g.max_blocks * g.block_size);
+      int np = 1;
+      if (!done) {
+        item = __ldcg(&ws.items[it]);
+        qi = __ldcg(&ws.qrow_info[item.x]);
+        np = __ldcg(&ws.nparts[item.x]);
       }
+      // keys [key_start + 16 first, + 16 stages) of the row (after a shared
+      // prefix, if any); lo >= hi: empty item, skipped; never past the table
+      const int lo = qi.w + item.w * kStageTokens;
+      const int hi = done ? lo + 1
+                          : min(min(lo + (item.y >> kItemSizeShift) * kStageTokens, qi.y),
+                                g.max_blocks * g.block_size);
+      item.y &= kItemHgMask;
       const int32_t* table = g.block_tables + static_cast<int64_t>(qi.x) * g.max_blocks;
       for (int key0 = lo; key0 < hi; key0 += kStageTokens) {
         if (round > 0 && !mbar_wait_bounded(&empty[stage], phase ^ 1, kWaitLimitNs)) {
@@ -336,37 +294,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
     } else {
       uint32_t kt = smem_u32(stages + stage * C::kStageBytes) + hh * C::kTile;
       uint32_t vt = kt + C::kTensorBytes;
-      constexpr uint32_t kHalf = F8 ? C::kTile : HG * C::kTile;  // between the two halves
-      if constexpr (F8) {
-        // widen this head's V codes to f16 in the warp's scratch (keys past
-        // the end of the request become zeros: the pool may hold NaN codes)
-        const uint8_t* v8 = stages + stage * C::kStageBytes + C::kTensorBytes + hh * C::kTile;
-        uint8_t* vs = scratch + hh * (2 * C::kTile);
-        __syncwarp();  // the previous stage's fragments have been read
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = lane + 32 * u;  // 128 chunks of 16 codes
-          const int key = i >> 3, c = i & 7;
-          const uint4 w8 = *reinterpret_cast<const uint4*>(v8 + mmak::swz(key, c));
-          uint32_t h[8];
-          const uint32_t w[4] = {w8.x, w8.y, w8.z, w8.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            h[2 * j] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] & 0xffffu));
-            h[2 * j + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] >> 16));
-          }
-          if (key >= si.nvalid) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) h[j] = 0u;
-          }
-          uint8_t* dst = vs + (c >> 2) * C::kTile;
-          *reinterpret_cast<uint4*>(dst + mmak::swz(key, 2 * (c & 3))) =
-              make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4*>(dst + mmak::swz(key, 2 * (c & 3) + 1)) =
-              make_uint4(h[4], h[5], h[6], h[7]);
-        }
-        vt = smem_u32(vs);
-      }
+      constexpr uint32_t kHalf = HG * C::kTile;  // between the two halves (bf16)
       // ---- S = Q K^T over 16 keys
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
       if constexpr (F8) {
@@ -385,9 +313,6 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
             mma_f16_16816((m & 1) ? s1 : s0, qa[kk + (m >> 1)], lo, hi);
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);  // codes of K and V consumed
-        released = true;
       } else {
         const int mi = lane >> 3;
         const int key = (lane & 7) + ((mi >> 1) << 3);
@@ -479,7 +404,32 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         __syncwarp();
       }
       // ---- O += P V
-      {
+      if constexpr (F8) {
+        // matrices: keys 0-7 / 8-15 of code chunk 2q, then of chunk 2q + 1
+        const int mi = lane >> 3;
+        const int key = (lane & 7) + ((mi & 1) << 3);
+        // keys past the end of the request: their (possibly NaN) codes are
+        // zeroed after widening, as halves of the key pairs (2t, 2t+1) and
+        // (2t+8, 2t+9) this lane holds
+        const int t2 = 2 * (lane & 3);
+        const uint32_t mk0 = (t2 < nv ? 0x0000ffffu : 0u) | (t2 + 1 < nv ? 0xffff0000u : 0u);
+        const uint32_t mk1 = (t2 + 8 < nv ? 0x0000ffffu : 0u) | (t2 + 9 < nv ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t r[4];
+          ldmatrix_x4_trans(vt + mmak::swz(key, 2 * q + (mi >> 1)), r[0], r[1], r[2], r[3]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {  // code chunk 2q + h: even dims, then odd dims
+            const uint32_t lo = prmt_b32(r[2 * h], 0x3120u), hi = prmt_b32(r[2 * h + 1], 0x3120u);
+            const uint32_t e0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo & 0xffffu)) & mk0;
+            const uint32_t e1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi & 0xffffu)) & mk1;
+            const uint32_t d0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo >> 16)) & mk0;
+            const uint32_t d1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi >> 16)) & mk1;
+            mma_f16_16816(o[2 * (2 * q + h)], pa, e0, e1);
+            mma_f16_16816(o[2 * (2 * q + h) + 1], pa, d0, d1);
+          }
+        }
+      } else {
         const int mi = lane >> 3;
         const int key = (lane & 7) + ((mi & 1) << 3);
 #pragma unroll
@@ -488,13 +438,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           const int chunk = 2 * c16 + (mi >> 1);
           uint32_t b0, b1, b2, b3;
           ldmatrix_x4_trans(vt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
-          if constexpr (F8) {
-            mma_f16_16816(o[2 * n2], pa, b0, b1);
-            mma_f16_16816(o[2 * n2 + 1], pa, b2, b3);
-          } else {
-            mma_bf16_16816(o[2 * n2], pa, b0, b1);
-            mma_bf16_16816(o[2 * n2 + 1], pa, b2, b3);
-          }
+          mma_bf16_16816(o[2 * n2], pa, b0, b1);
+          mma_bf16_16816(o[2 * n2 + 1], pa, b2, b3);
         }
       }
       if (!F8 && nv < kStageTokens) fence_proxy_async_smem();
@@ -515,7 +460,54 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         }
       } else {
         const int np = si.np;
-        if (np == 1) {
+        if (F8) {
+          // o[2c] holds the even dims of chunk c, o[2c + 1] the odd ones: this
+          // lane's four values of a row are dims 16c + 4t .. 16c + 4t + 3
+          const int t4 = 4 * (lane & 3);
+          const bool direct = np == 1;
+          const float i0 = direct ? vsc / l0 : vsc, i1 = direct ? vsc / l1 : vsc;
+          float* dst0 = nullptr;
+          float* dst1 = nullptr;
+          __nv_bfloat16* bdst0 = nullptr;
+          __nv_bfloat16* bdst1 = nullptr;
+          if (direct) {
+            const int64_t ob = (static_cast<int64_t>(r) * g.num_heads + head) * D;
+            if (g.out_dtype == PA_F32) {
+              dst0 = static_cast<float*>(g.out) + ob + qr * D;
+              dst1 = dst0 + 8 * D;
+            } else {
+              bdst0 = static_cast<__nv_bfloat16*>(g.out) + ob + qr * D;
+              bdst1 = bdst0 + 8 * D;
+            }
+          } else {
+            const int64_t slot0 =
+                (static_cast<int64_t>(r) * g.num_heads + head) * ws.max_parts + si.part;
+            const int64_t sl0 = slot0 + static_cast<int64_t>(qr) * ws.max_parts;
+            const int64_t sl1 = slot0 + static_cast<int64_t>(qr + 8) * ws.max_parts;
+            if ((lane & 3) == 0 && qr < G) ws.part_ml[sl0] = make_float2(m0, l0);
+            if ((lane & 3) == 0 && qr + 8 < G) ws.part_ml[sl1] = make_float2(m1, l1);
+            dst0 = ws.part_o + sl0 * D;
+            dst1 = ws.part_o + sl1 * D;
+          }
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            const float4 v0 = make_float4(o[2 * c][0] * i0, o[2 * c + 1][0] * i0,
+                                          o[2 * c][1] * i0, o[2 * c + 1][1] * i0);
+            const float4 v1 = make_float4(o[2 * c][2] * i1, o[2 * c + 1][2] * i1,
+                                          o[2 * c][3] * i1, o[2 * c + 1][3] * i1);
+            if (bdst0) {
+              if (qr < G)
+                *reinterpret_cast<uint2*>(bdst0 + c * 16 + t4) =
+                    make_uint2(pack_bf16x2(v0.x, v0.y), pack_bf16x2(v0.z, v0.w));
+              if (qr + 8 < G)
+                *reinterpret_cast<uint2*>(bdst1 + c * 16 + t4) =
+                    make_uint2(pack_bf16x2(v1.x, v1.y), pack_bf16x2(v1.z, v1.w));
+            } else {
+              if (qr < G) *reinterpret_cast<float4*>(dst0 + c * 16 + t4) = v0;
+              if (qr + 8 < G) *reinterpret_cast<float4*>(dst1 + c * 16 + t4) = v1;
+            }
+          }
+        } else if (np == 1) {
           const float i0 = vsc / l0, i1 = vsc / l1;
           const int64_t ob = (static_cast<int64_t>(r) * g.num_heads + head) * D;
           if (g.out_dtype == PA_F32) {

@@ -509,9 +509,9 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
               float x0, x1;
               f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), sl2, nm2),
                         x0, x1);
-              // every exponential on the XU (ex2.approx): moving a share of them to a
-              // polynomial on the FMA pipe measured slower (that pipe also carries the
-              // scaling, maxima and sums)
+              // every exponential on the XU (ex2.approx): sending a quarter, three
+              // eighths or half of them (by column pairs) to a cubic on the FMA pipe
+              // measured 3 %, 15 % and 20 % slower -- the softmax is not XU-bound
               const float p0 = fast_exp2(x0);
               const float p1 = fast_exp2(x1);
               acc[(e >> 1) & 3] = f2_add(acc[(e >> 1) & 3], f2_pack(p0, p1));

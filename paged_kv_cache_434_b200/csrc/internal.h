@@ -25,10 +25,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 //                         [7] key chunks the shared prefix is split into,
 //                         [8] CTAs of the tensor-core tile kernel that work,
 //                         [9] rows to merge with more than 32 partitions
-//                         (listed from the back of merge_rows),
-//                         [10] decode partitions in balanced ranges: the
-//                         number C of ranges (0: items from the list),
-//                         [11]/[12] total units U of those ranges (low, high)
+//                         (listed from the back of merge_rows)
 //   qrow_info int4[R]     {request b, key_len, valid, key_start}: the row's
 //                         partitions cover keys [key_start, key_len); keys
 //                         below key_start (a shared prefix) come from tiles
@@ -37,21 +34,25 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 //   qrow_bad  int32[R]    set when a block id outside the pool was met
 //   merge_rows int32[R]   rows the merge pass must write (0 or >1 partitions):
 //                         up to 32 partitions from the front, more from the back
-//   items     int4[I]     {qrow, head group, partition, 0}
+//   items     int4[I]     {qrow, head group | stages << kItemSizeShift,
+//                         partition, first stage}: keys [key_start + 16 first,
+//                         + 16 stages) of the row, clipped to its length
 //   part_ml   float2[R*H*P]   per (row, query head, partition): (m, l),
 //                         m in log2 units (score * scale * log2 e)
 //   part_o    float[R*H*P*D]  unnormalised partial outputs
 //   tiles     int4[Tl]    tensor-core tiles: prefill {request b, kv head, first
 //                         token, tokens}; shared prefix {first request, kv
 //                         head, requests, key chunk}
-//   sk        int4[C]     balanced ranges: CTA c starts at {row, 0, stage}
-//                         and streams `units` 16-key stages, rows in order
-//   row_ustart int64[R]   first unit of each row in that order
 struct WsLayout {
-  size_t ctrl, qrow_info, nparts, qrow_bad, merge_rows, items, part_ml, part_o, tiles, sk,
-      row_ustart, total;
-  int64_t num_qrows, max_parts, max_items, max_tiles, max_ctas;
+  size_t ctrl, qrow_info, nparts, qrow_bad, merge_rows, items, part_ml, part_o, tiles, total;
+  int64_t num_qrows, max_parts, max_items, max_tiles;
 };
+
+// Item field packing: head group in the low bits of .y, the item's length in
+// 16-key stages above them.
+constexpr int kItemSizeShift = 12;
+constexpr int kItemHgMask = (1 << kItemSizeShift) - 1;
+constexpr int kMaxItemStages = (1 << (31 - kItemSizeShift)) - 1;
 
 struct WsView {
   int32_t* ctrl;
@@ -63,29 +64,13 @@ struct WsView {
   float2* part_ml;
   float* part_o;
   int4* tiles;
-  int4* sk;
-  int64_t* row_ustart;
   int64_t max_parts;
   int64_t max_items;
   int64_t max_tiles;
-  int32_t max_ctas;  // balanced ranges the workspace has room for
 };
 
 WsLayout ws_layout(int64_t num_qrows, int num_heads, int head_dim, int head_groups,
-                   int64_t max_parts, int64_t max_tiles, int max_ctas);
-
-// Balanced ranges of the decode partitions: units (16-key stages) in (row,
-// stage) order, cut into C ranges; range c is [u0(c), u0(c + 1)) with
-// u0(c) = floor(c U / C), and range_of(u) is the range holding unit u.  The
-// pieces of a row are its partitions, numbered by range.
-__device__ __forceinline__ long long range_start(long long c, long long U, int C) {
-  return c * U / C;
-}
-__device__ __forceinline__ int range_of(long long u, long long U, int C) {
-  int c = static_cast<int>(u * C / U);
-  if (c + 1 < C && range_start(c + 1, U, C) <= u) ++c;
-  return c;
-}
+                   int64_t max_parts, int64_t max_tiles);
 WsView ws_view(void* base, const WsLayout& L);
 
 // ---------------------------------------------------------------- geometry
@@ -122,8 +107,6 @@ struct PlanArgs {
   int32_t tile_tokens;      // tokens (rows of a request) per tensor-core tile pair
   int32_t cascade;          // decode: attend a prefix shared by all requests once
   int32_t num_sms;
-  int32_t balanced;         // 1: a decode batch without tiles (one head group
-                            // per row) may be cut into num_sms balanced ranges
 };
 
 // Shared-prefix cascade: only worth it for long prefixes and enough requests.

@@ -122,7 +122,7 @@ static AttnPlan make_plan(int64_t num_qrows, int num_heads, int max_blocks,
                : 0.0;
   const double bytes = 64.0 * 4 + rows * (16 + 3 * 4) + rows * p.head_groups * parts * 16 +
                        rows * num_heads * parts * (8 + 4.0 * c->head_dim) + tiles * 16 +
-                       p.num_sms * 16.0 + rows * 8 + 11 * 256;
+                       9 * 256;
   p.size_ok = bytes <= kMaxWorkspaceBytes;
   p.max_tiles = (p.use_tc && p.size_ok)
                     ? ((num_qrows + p.tile_tokens - 1) / p.tile_tokens + num_seqs) *
@@ -219,7 +219,7 @@ class TimedCall {
 static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* workspace,
                                size_t ws_bytes, cudaStream_t s) {
   const WsLayout L = ws_layout(p.num_qrows, g.num_heads, g.head_dim, p.head_groups, p.max_parts,
-                               p.max_tiles, p.num_sms);
+                               p.max_tiles);
   if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return PA_ERR_WORKSPACE;
   if (g.num_qrows == 0 || g.num_seqs == 0) return PA_OK;
@@ -233,7 +233,6 @@ static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* works
   a.tile_tokens = p.tile_tokens;
   a.cascade = p.cascade ? 1 : 0;
   a.num_sms = p.num_sms;
-  a.balanced = p.use_mma ? 1 : 0;
   TimedCall tm(s);
   tm.begin(PA_TK_PLAN);
   if (launch_plan(g, a, ws, s) != cudaSuccess) return PA_ERR_CUDA;
@@ -324,7 +323,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t max
   const AttnPlan p = make_plan(num_seqs, num_heads, max_blocks_per_seq, cache, true);
   if (!p.size_ok) return 0;
   return ws_layout(p.num_qrows, num_heads, cache->head_dim, p.head_groups, p.max_parts,
-                   p.max_tiles, p.num_sms)
+                   p.max_tiles)
       .total;
 }
 
@@ -358,7 +357,7 @@ size_t pa_mixed_step_workspace_size(int32_t num_seqs, int64_t num_tokens, int32_
       make_plan(num_tokens, num_heads, max_blocks_per_seq, cache, true, num_seqs, true);
   if (!p.size_ok) return 0;
   return ws_layout(p.num_qrows, num_heads, cache->head_dim, p.head_groups, p.max_parts,
-                   p.max_tiles, p.num_sms)
+                   p.max_tiles)
       .total;
 }
 

@@ -198,6 +198,12 @@ __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// Byte permute of one word: result byte i is byte ((sel >> 4i) & 3) of a.
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(a), "r"(sel));
+  return d;
+}
 // Two e4m3 codes (low byte first) to two halves of an f16x2 (exact).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
   uint32_t r;
@@ -242,7 +248,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-
 // ------------------------------------------------------------------ tcgen05 (sm_100a)
 // Tensor memory: 128 lanes x 512 columns of 32-bit cells per SM.  A warp may
 // only touch lanes [32 * (warp % 4), +32).  Address = (lane << 16) | column.
