@@ -5,7 +5,8 @@
 A step is the whole hot path for one batch: slot mapping of the new tokens,
 the cache write (reshape_and_cache) and the attention call (pa_decode for
 decode batches, pa_mixed_step for a chunked-prefill step).  Inputs are
-resident in HBM when timing starts; L2 is flushed (a 512 MiB write) before
+resident in HBM when timing starts; L2 is flushed (a 512 MiB write, then a
+512 MiB read, so no dirty line is written back during the step) before
 every step and only the step itself sits between its CUDA events.  With
 torchrun (N > 1) every rank runs its own batch on its own GPU (sequences are
 independent: weak scaling, no collective on the data path); the time is the
@@ -61,6 +62,23 @@ WORKLOADS = {
     "graph_decode": ("llama8b_decode", 2),  # a small decode step replayed from a CUDA graph
 }
 FLUSH_BYTES = 512 << 20
+L2_NOTE = ("flushed before every step, outside the events: a 512 MiB write, then a 512 MiB "
+           "read, so that L2 holds clean lines and no write-back of the flush competes with "
+           "the step")
+
+
+class L2Flush:
+    """Evicts L2 between steps: writes a buffer larger than L2, then reads
+    another, so that the dirty lines of the write are written back before the
+    step instead of during it."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+
+    def fill_(self, v=1):
+        self.w.fill_(v)
+        self.r.sum()
 
 
 def parse_args(argv=None):
@@ -431,7 +449,7 @@ def measure(args, name, rank, world, local, with_e2e=True, with_cpu=True):
                 P.mixed_step_workspace_size(w.num_seqs, T, w.num_heads, w.max_blocks_per_seq,
                                             t["k_cache"]))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -612,7 +630,7 @@ def measure(args, name, rank, world, local, with_e2e=True, with_cpu=True):
                    "head_dim": w.head_dim, "block_size": w.block_size,
                    "num_blocks": w.num_blocks,
                    "kv_bytes_unique": bc["kv"], "step_bytes": bc["step"],
-                   "l2": "flushed before every step (512 MiB write, outside the events)",
+                   "l2": L2_NOTE,
                    "parallelism": f"replicas x{world} (independent batches per GPU)",
                    **extra},
         "roofline": roofline,
@@ -721,7 +739,7 @@ def run_rope(args, rank, world, local):
     table = P.rope_cos_sin_cache(x["max_pos"], w.head_dim, ROPE_THETA, device=dev)
     q_out = torch.empty_like(x["q"])
     err = P.new_error_word(dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -806,7 +824,7 @@ def run_rope(args, rank, world, local):
                        "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
                        "head_dim": w.head_dim, "rotary_dim": w.head_dim, "rope_theta": ROPE_THETA,
                        "pairing": "split-half (neox)", "step_bytes": nbytes,
-                       "l2": "flushed before every step (512 MiB write, outside the events)",
+                       "l2": L2_NOTE,
                        "parallelism": f"replicas x{world} (independent batches per GPU)"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": clk, "wall_s_timed_region": round(wall, 3)}),
@@ -953,7 +971,7 @@ def run_cow(args, rank, world, local):
     torch.cuda.set_device(dev)
     kc, vc, m = cow_inputs(dev, args.seed + rank)
     err = P.new_error_word(dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
     step = lambda: P.copy_blocks(kc, vc, m, err=err)
     for _ in range(max(args.warmup, 3)):
@@ -1023,7 +1041,7 @@ def run_cow(args, rank, world, local):
             "config": {"workload": "cow_copy_llama3_8b_2048_pairs", "pairs": COW_PAIRS,
                        "num_blocks": COW_BLOCKS, "block_size": 16, "num_kv_heads": 8,
                        "head_dim": 128, "step_bytes": nbytes,
-                       "l2": "flushed before every step (512 MiB write, outside the events)",
+                       "l2": L2_NOTE,
                        "parallelism": f"replicas x{world} (independent pools per GPU)"},
             "roofline": {"bound": "hbm", "kernel": "copy_blocks_kernel", "achieved": round(achieved, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -1058,7 +1076,7 @@ def run_graph(args, rank, world, local):
     slots = torch.empty(T, dtype=torch.int64, device=dev)
     out = torch.empty(T, w.num_heads, w.head_dim, dtype=torch.float32, device=dev)
     err = P.new_error_word(dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step():
         P.step(t["q"], t["k_new"], t["v_new"], t["k_cache"], t["v_cache"], idx["block_tables"],
@@ -1141,7 +1159,7 @@ def run_graph(args, rank, world, local):
             "config": {"workload": w.name, "num_seqs": w.num_seqs, "seq_lens": GRAPH_LENS,
                        "num_heads": 32, "num_kv_heads": 8, "head_dim": 128, "block_size": 16,
                        "step_bytes": bc["step"],
-                       "l2": "flushed before every step (512 MiB write, outside the events)",
+                       "l2": L2_NOTE,
                        "parallelism": f"replicas x{world}"},
             "eager_us_per_step": round(statistics.mean(e_ms) * 1e3, 2),
             "l2_warm_back_to_back_us": {"graph": round(statistics.mean(g_hot) * 1e3, 2),

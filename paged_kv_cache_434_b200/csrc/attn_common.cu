@@ -196,12 +196,13 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T* s_scan, T* total) {
 // plan needs no re-reads of the workspace and few barriers.
 //   * Shared prefix (batches of >= kCascadeMinSeqs requests whose tables all
 //     start with the same block): the longest common run of leading blocks is
-//     found by comparing (request, column) pairs against row 0 in shared
-//     memory; a run of >= kCascadeMinPrefix tokens is attended by tensor-core
-//     tiles (listed here) and the rows keep only their suffix.
+//     found by comparing (request, column) pairs against row 0; a run of
+//     >= kCascadeMinPrefix tokens is attended by tensor-core tiles (listed
+//     here) and the rows keep only their suffix.
 //   * Partitions in decreasing sizes: work W = stages x head groups; each row
-//     is cut into big pieces of Pb ~ 0.85 W / (2 SMs) stages (85 % of its
-//     stages, whole pieces only) and small pieces of Pb / 4 for the rest.
+//     is cut into big pieces of Pb ~ 0.4 W / SMs stages (within 80 % of its
+//     stages, whole pieces only) and small pieces of Ps ~ 0.05 W / SMs for
+//     the rest: about two big and four small pieces per SM overall.
 //     The item list holds every big piece before every small one, and the
 //     partition kernel takes items in list order from a global counter: the
 //     big pieces spread the work, the small ones even out the end, whatever
@@ -212,8 +213,37 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T* s_scan, T* total) {
 constexpr int kFastPerThread = 4;
 constexpr int kFastRows = kPlanThreads * kFastPerThread;
 
+// The pieces of a row of n stages: nb big ones of pb stages (whole pieces
+// within 80 % of the row), then ns small ones of ps.  A row that would need
+// more than `cap` pieces gets larger pieces of its own (at most cap / 2 big
+// and the rest small).  The same arithmetic wherever a row's pieces are
+// counted or listed.
+struct RowPieces {
+  int pb, nb, ps, ns;
+};
+__device__ __forceinline__ RowPieces row_pieces(int n, int Pb, int Ps, int cap) {
+  RowPieces p;
+  if (cap < 2) {  // one piece per row
+    p.pb = max(n, 1), p.nb = n > 0 ? 1 : 0, p.ps = 1, p.ns = 0;
+    return p;
+  }
+  const int big = static_cast<int>(static_cast<float>(n) * 0.8f);
+  p.pb = Pb;
+  p.nb = big / Pb;
+  p.ps = Ps;
+  p.ns = (n - p.nb * Pb + Ps - 1) / Ps;
+  if (p.nb + p.ns <= cap) return p;
+  const int hb = cap / 2, hs = cap - hb;
+  p.pb = max(Pb, (big + hb - 1) / hb);
+  p.nb = big / p.pb;
+  const int rem = n - p.nb * p.pb;
+  p.ps = max(Ps, (rem + hs - 1) / hs);
+  p.ns = (rem + p.ps - 1) / p.ps;
+  return p;
+}
+
 __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsView& ws,
-                                 int* s_rowpos, int* s_ref, int ref_cap, int* s_scan,
+                                 int* s_rowpos, int* s_scan,
                                  long long* s_sum, int* s_max, int* s_P, int* s_merge,
                                  int* s_merge_big) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -245,10 +275,11 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
     if (ok) min_len = min(min_len, L[k]);
   }
 
-  // Shared prefix: row 0's entries go to shared memory; the (request, column)
-  // pairs are compared column chunk by column chunk, about eight loads per
-  // thread per chunk, until a chunk holds a mismatch.  The run is limited so
-  // that each request keeps at least one key of its own.
+  // Shared prefix: the (request, column) pairs are compared with row 0 column
+  // chunk by column chunk -- each thread loads both entries of its pairs, 16
+  // pairs per thread in a chunk, the chunks growing fourfold -- until a chunk
+  // holds a mismatch (the tables are often cold: one round trip per chunk).
+  // The run is limited so that each request keeps at least one key of its own.
   __shared__ int s_first, s_minlen;
   int prefix_blocks = 0;
   if (look_shared) {
@@ -259,21 +290,31 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
     const bool cand = __syncthreads_and(same && all_ok) && s_minlen > kCascadeMinPrefix &&
                       s_minlen != 0x7fffffff;
     if (cand) {
-      const int max_cols = min(min((s_minlen - 1) / g.block_size, g.max_blocks), ref_cap);
-      for (int c = tid; c < max_cols; c += kPlanThreads) s_ref[c] = g.block_tables[c];
+      const int max_cols = min((s_minlen - 1) / g.block_size, g.max_blocks);
       if (tid == 0) s_first = max_cols;
       __syncthreads();
-      const int W = max(1, 8 * kPlanThreads / B);  // columns per chunk
-      for (int cb = 1; cb < max_cols; cb += W) {
+      constexpr int kPairs = 16;  // pairs per thread and chunk
+      int W = max(1, kPairs * kPlanThreads / B);  // columns per chunk
+      for (int cb = 1; cb < max_cols; cb += W, W *= 4) {
         const int ce = min(cb + W, max_cols), wc = ce - cb;
+        const int64_t pairs = static_cast<int64_t>(wc) * B;
         int mine = 0x7fffffff;
+        for (int64_t i0 = 0; i0 < pairs; i0 += kPairs * kPlanThreads) {
+          int v[kPairs], ref[kPairs];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int idx = tid + k * kPlanThreads;
-          if (idx < wc * B) {
-            const int b = idx / wc, j = cb + idx % wc;
-            if (g.block_tables[static_cast<int64_t>(b) * g.max_blocks + j] != s_ref[j])
-              mine = min(mine, j);
+          for (int k = 0; k < kPairs; ++k) {
+            const int64_t idx = i0 + tid + static_cast<int64_t>(k) * kPlanThreads;
+            v[k] = ref[k] = 0;
+            if (idx < pairs) {
+              const int b = static_cast<int>(idx / wc), j = cb + static_cast<int>(idx % wc);
+              v[k] = g.block_tables[static_cast<int64_t>(b) * g.max_blocks + j];
+              ref[k] = g.block_tables[j];
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kPairs; ++k) {
+            const int64_t idx = i0 + tid + static_cast<int64_t>(k) * kPlanThreads;
+            if (idx < pairs && v[k] != ref[k]) mine = min(mine, cb + static_cast<int>(idx % wc));
           }
         }
         mine = __reduce_min_sync(0xffffffffu, mine);
@@ -316,52 +357,48 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
   }
   __shared__ int s_Pb, s_Ps;
   __syncthreads();
-  const long long cap =
-      max(1LL, static_cast<long long>(ws.max_parts) - (a.cascade ? kMaxPrefixChunks : 0));
-  if (tid == 0) {
-    long long total = 0;
-    int mx = 0;
-    for (int w = 0; w < kPlanThreads / 32; ++w) {
-      total += s_sum[w];
-      mx = max(mx, s_max[w]);
+  // partial slots a row's own pieces may use (the last kMaxPrefixChunks are
+  // the shared prefix's, when there is one)
+  const int cap = static_cast<int>(
+      max(1LL, static_cast<long long>(ws.max_parts) - (prefix > 0 ? kMaxPrefixChunks : 0)));
+  if (warp == 0) {
+    long long total = s_sum[lane];
+    int mx = s_max[lane];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    const long long work = total * a.head_groups;
-    const long long by_target = (work + a.target_items - 1) / max(a.target_items, 1);
-    const long long by_cap = (mx + cap - 1) / cap;
-    const long long P = max(static_cast<long long>(a.min_part_stages), max(by_target, by_cap));
-    *s_P = static_cast<int>(min(max(P, 1LL), static_cast<long long>(kMaxItemStages)));
-    const long long pb = max(static_cast<long long>(a.min_part_stages),
-                             work * 85 / (100 * 2 * max(a.num_sms, 1)));
-    s_Pb = static_cast<int>(min(pb, static_cast<long long>(kMaxItemStages)));
-    s_Ps = max(a.min_part_stages, s_Pb / 4);
-    *s_merge = 0;
-    *s_merge_big = 0;
+    if (lane == 0) {
+      // the sizes are heuristics: float arithmetic (no 64-bit division)
+      const double work = static_cast<double>(total) * a.head_groups;
+      const double by_target = ceil(work / max(a.target_items, 1));
+      const int by_cap = (mx + cap - 1) / cap;
+      const double P = fmax(static_cast<double>(a.min_part_stages), fmax(by_target, by_cap));
+      *s_P = static_cast<int>(fmin(fmax(P, 1.0), 1e9));
+      // big pieces: 80 % of the work, about two per SM; small pieces: the
+      // rest, about four per SM
+      const double C = max(a.num_sms, 1);
+      s_Pb = static_cast<int>(fmin(fmax(0.4 * work / C, static_cast<double>(a.min_part_stages)),
+                                   1e9));
+      s_Ps = static_cast<int>(fmin(fmax(0.05 * work / C, static_cast<double>(a.min_part_stages)),
+                                   static_cast<double>(s_Pb)));
+      *s_merge = 0;
+      *s_merge_big = 0;
+    }
   }
   __syncthreads();
-  // pieces per row: big + small, unless some row would need too many
+  // pieces per row: whole big pieces within 80 % of its stages, small pieces
+  // for the rest
+  const int Pb = s_Pb, Ps = s_Ps;
   int nb[kFastPerThread], ns[kFastPerThread];
-  bool fits = true;
-  {
-    const int Pb = s_Pb, Ps = s_Ps;
 #pragma unroll
-    for (int k = 0; k < kFastPerThread; ++k) {
-      nb[k] = ns[k] = 0;
-      if (k >= per || r0 + k >= B || L[k] < 0) continue;
-      const int n = (L[k] - prefix + kStageTokens - 1) / kStageTokens;
-      nb[k] = static_cast<int>(static_cast<long long>(n) * 85 / 100 / Pb);
-      ns[k] = (n - nb[k] * Pb + Ps - 1) / Ps;
-      fits &= nb[k] + ns[k] <= cap;
-    }
-  }
-  const bool guided = __syncthreads_and(fits);
-  const int Pb = guided ? s_Pb : *s_P, Ps = guided ? s_Ps : *s_P;
-  if (!guided) {
-#pragma unroll
-    for (int k = 0; k < kFastPerThread; ++k) {
-      nb[k] = 0;
-      if (k >= per || r0 + k >= B || L[k] < 0) continue;
-      ns[k] = ((L[k] - prefix + kStageTokens - 1) / kStageTokens + Ps - 1) / Ps;
-    }
+  for (int k = 0; k < kFastPerThread; ++k) {
+    nb[k] = ns[k] = 0;
+    if (k >= per || r0 + k >= B || L[k] < 0) continue;
+    const RowPieces rp = row_pieces((L[k] - prefix + kStageTokens - 1) / kStageTokens, Pb, Ps, cap);
+    nb[k] = rp.nb;
+    ns[k] = rp.ns;
   }
   // item positions: every big piece first, then every small piece
   int my_big = 0, my_small = 0;
@@ -393,8 +430,10 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
         else hi = mid;
       }
       const int k = i - s_rowpos[lo], piece = k / a.head_groups;
-      ws.items[i] = make_int4(lo, (k % a.head_groups) | (Pb << kItemSizeShift), piece,
-                              piece * Pb);
+      const int n = (g.seq_lens[lo] - prefix + kStageTokens - 1) / kStageTokens;
+      const RowPieces rp = row_pieces(n, Pb, Ps, cap);
+      ws.items[i] = make_int4(lo, (k % a.head_groups) | (piece << kItemPartShift), rp.pb,
+                              piece * rp.pb);
     }
     __syncthreads();
   }
@@ -418,14 +457,13 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
         else hi = mid;
       }
       const int row = lo, k = i - s_rowpos[row], piece = k / a.head_groups;
-      // the row's big pieces, from the owning thread's registers, are not at
+      // the row's piece sizes, from the owning thread's registers, are not at
       // hand here: recompute them from its length
-      const int Lr = g.seq_lens[row];
-      const int n = (Lr - prefix + kStageTokens - 1) / kStageTokens;
-      const int nbr = guided ? static_cast<int>(static_cast<long long>(n) * 85 / 100 / Pb) : 0;
+      const int n = (g.seq_lens[row] - prefix + kStageTokens - 1) / kStageTokens;
+      const RowPieces rp = row_pieces(n, Pb, Ps, cap);
       ws.items[n_big + i] =
-          make_int4(row, (k % a.head_groups) | (Ps << kItemSizeShift), nbr + piece,
-                    nbr * Pb + piece * Ps);
+          make_int4(row, (k % a.head_groups) | ((rp.nb + piece) << kItemPartShift), rp.ps,
+                    rp.nb * rp.pb + piece * rp.ps);
     }
   }
   // shared-prefix tiles: groups of tile_tokens requests x one KV head x a
@@ -465,7 +503,7 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
   if (tid == 0) {
     ws.ctrl[0] = 0;
     ws.ctrl[1] = n_big + n_small;
-    ws.ctrl[2] = Pb * kStageTokens;
+    ws.ctrl[2] = Pb * kStageTokens;  // (informative: items carry their own length)
     ws.ctrl[3] = 0;
     ws.ctrl[4] = n_tiles;
     ws.ctrl[5] = *s_merge;
@@ -496,7 +534,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
 
   if (decode_mode && g.num_seqs <= kFastRows && g.num_qrows == g.num_seqs) {
     __shared__ int s_scan33[33];
-    plan_decode_fast(g, a, ws, s_rowpos, s_hist, kTileBins, s_scan33, s_sum, s_max, &s_P,
+    plan_decode_fast(g, a, ws, s_rowpos, s_scan33, s_sum, s_max, &s_P,
                      &s_merge, &s_merge_big);
     return;
   }
@@ -695,10 +733,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     }
     long long by_target = (total * a.head_groups + a.target_items - 1) / max(a.target_items, 1);
     const long long cap =
-        max(1LL, static_cast<long long>(ws.max_parts) - (a.cascade ? kMaxPrefixChunks : 0));
+        max(1LL, static_cast<long long>(ws.max_parts) - (prefix_tokens > 0 ? kMaxPrefixChunks : 0));
     long long by_cap = (mx + cap - 1) / cap;
     long long P = max(static_cast<long long>(a.min_part_stages), max(by_target, by_cap));
-    s_P = static_cast<int>(min(max(P, 1LL), static_cast<long long>(kMaxItemStages)));
+    s_P = static_cast<int>(max(P, 1LL));
     // CTAs the tensor-core tiles run on.  With decode partitions in the same
     // call, the tiles take only as many SMs as finish them in about half the
     // time the (HBM-bound) partitions need, and the partitions start at once
@@ -780,7 +818,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     }
     for (int p = 0; p < np; ++p)
       for (int hg = 0; hg < a.head_groups; ++hg)
-        ws.items[pos++] = make_int4(r, hg | (P << kItemSizeShift), p, p * P);
+        ws.items[pos++] = make_int4(r, hg | (p << kItemPartShift), P, p * P);
   }
   __syncthreads();
   const int nbig_rows = min(s_nbig, kMaxBig);
@@ -790,8 +828,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     const int units = (info.y - info.w + kStageTokens - 1) / kStageTokens;
     const int n_it = (units + P - 1) / P * a.head_groups;
     for (int i = tid; i < n_it; i += kPlanThreads)
-      ws.items[s_bigpos[k] + i] = make_int4(r, (i % a.head_groups) | (P << kItemSizeShift),
-                                            i / a.head_groups, (i / a.head_groups) * P);
+      ws.items[s_bigpos[k] + i] =
+          make_int4(r, (i % a.head_groups) | ((i / a.head_groups) << kItemPartShift), P,
+                    (i / a.head_groups) * P);
   }
 
   // 4. tiles, longest first
@@ -936,11 +975,13 @@ __global__ void __launch_bounds__(kGenWarps * 32) attn_generic_kernel(AttnGeom g
     const int it = s_item;
     if (it >= n_items) break;
     const int4 item = ws.items[it];
-    const int r = item.x, hk = item.y & kItemHgMask, p = item.z;
+    const int r = item.x, hk = item.y & kItemHgMask, p = item.y >> kItemPartShift;
     const int4 info = ws.qrow_info[r];
     const int b = info.x, key_len = info.y;
-    const int lo = info.w + item.w * kStageTokens;
-    const int hi = min(lo + (item.y >> kItemSizeShift) * kStageTokens, key_len);
+    const int64_t lo64 = info.w + static_cast<int64_t>(item.w) * kStageTokens;
+    const int lo = static_cast<int>(lo64);
+    const int hi = static_cast<int>(min(lo64 + static_cast<int64_t>(item.z) * kStageTokens,
+                                        static_cast<int64_t>(key_len)));
     for (int idx = tid; idx < G * D; idx += blockDim.x) {
       const int gq = idx / D, d = idx % D;
       s_q[gq][d] = to_f32(q[(static_cast<int64_t>(r) * g.num_heads + hk * G + gq) * D + d]);
@@ -1063,10 +1104,10 @@ cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms
 // planner's list.  Pass 1: one warp per (row, query head) whose partitions fit
 // in a warp (<= 32): lane k holds partition k's (m, l), the weights
 // 2^(m_k - M) are shuffled to all lanes and each lane accumulates D/32 output
-// columns.  Pass 2: one 16-warp CTA per remaining (row, head): max and
+// columns.  Pass 2: one 32-warp CTA per remaining (row, head): max and
 // denominator reduced over the CTA, then each warp accumulates every 8th
 // partition (4 in flight) and the warp sums are combined.
-constexpr int kMergeWarps = 16;
+constexpr int kMergeWarps = 32;
 constexpr int kMergeCached = 2048;  // partition weights kept in shared memory
 
 template <int D>
@@ -1092,9 +1133,9 @@ __device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView&
 #pragma unroll
   for (int e = 0; e < V; ++e) acc[e] = 0.f;
   const float* po = ws.part_o + base * D + lane * V;
-  // up to 16 partial rows in flight per lane: a row of at most 32 partitions
-  // takes at most two round trips to L2
-  constexpr int kBatch = 16;
+  // up to 8 partial rows in flight per lane (and 32 warps per SM): a row of
+  // at most 32 partitions takes at most four round trips to L2
+  constexpr int kBatch = 8;
   for (int k0 = 0; k0 < np; k0 += kBatch) {
     float x[kBatch][V];
 #pragma unroll
@@ -1122,7 +1163,7 @@ __device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView&
 }
 
 template <int D>
-__global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(AttnGeom g, WsView ws) {
+__global__ void __launch_bounds__(kMergeWarps * 32, 1) merge_kernel(AttnGeom g, WsView ws) {
   constexpr int V = D / 32;
   __shared__ float s_c[kMergeCached];
   __shared__ float s_red[kMergeWarps];
@@ -1219,7 +1260,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(AttnGeom g, WsV
 }
 
 cudaError_t launch_merge(const AttnGeom& g, const WsView& ws, int num_sms, cudaStream_t s) {
-  // one CTA of 16 warps per SM, warps looping over the pairs: a grid of
+  // one CTA of 32 warps per SM, warps looping over the pairs: a grid of
   // eight small CTAs per SM took ~10 us just to be launched
   int64_t blocks = static_cast<int64_t>(g.num_qrows) * g.num_heads;
   if (blocks == 0) return cudaSuccess;

@@ -141,10 +141,12 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       // keys [key_start + 16 first, + 16 stages) of the row (after a shared
       // prefix, if any); lo >= hi: empty item, skipped; never past the table
       const int lo = qi.w + item.w * kStageTokens;
-      const int hi = done ? lo + 1
-                          : min(min(lo + (item.y >> kItemSizeShift) * kStageTokens, qi.y),
-                                g.max_blocks * g.block_size);
-      item.y &= kItemHgMask;
+      const int hi =
+          done ? lo + 1
+               : static_cast<int>(min(static_cast<int64_t>(lo) + static_cast<int64_t>(item.z) *
+                                                                   kStageTokens,
+                                      static_cast<int64_t>(min(qi.y, g.max_blocks * g.block_size))));
+      const int hg = item.y & kItemHgMask, part = item.y >> kItemPartShift;
       const int32_t* table = g.block_tables + static_cast<int64_t>(qi.x) * g.max_blocks;
       for (int key0 = lo; key0 < hi; key0 += kStageTokens) {
         if (round > 0 && !mbar_wait_bounded(&empty[stage], phase ^ 1, kWaitLimitNs)) {
@@ -154,8 +156,8 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         mmak::StageInfo si;
         si.qrow = item.x;
         si.b = qi.x;
-        si.hg = item.y;
-        si.part = item.z;
+        si.hg = hg;
+        si.part = part;
         si.np = np;
         si.nvalid = min(kStageTokens, hi - key0);
         si.flags = done ? mmak::kEnd
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         } else {
           uint8_t* kbase = stages + stage * C::kStageBytes;
           uint8_t* vbase = kbase + C::kTensorBytes;
-          const int head0 = item.y * HG;
+          const int head0 = hg * HG;
           // The branch follows the kind of map the host encoded (by_token), and
           // each branch announces exactly the bytes of the boxes it issues.
           if (by_token) {

@@ -34,9 +34,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 //   qrow_bad  int32[R]    set when a block id outside the pool was met
 //   merge_rows int32[R]   rows the merge pass must write (0 or >1 partitions):
 //                         up to 32 partitions from the front, more from the back
-//   items     int4[I]     {qrow, head group | stages << kItemSizeShift,
-//                         partition, first stage}: keys [key_start + 16 first,
-//                         + 16 stages) of the row, clipped to its length
+//   items     int4[I]     {qrow, head group | partition << 16, stages, first
+//                         stage}: keys [key_start + 16 first, + 16 stages) of
+//                         the row, clipped to its length
 //   part_ml   float2[R*H*P]   per (row, query head, partition): (m, l),
 //                         m in log2 units (score * scale * log2 e)
 //   part_o    float[R*H*P*D]  unnormalised partial outputs
@@ -48,11 +48,10 @@ struct WsLayout {
   int64_t num_qrows, max_parts, max_items, max_tiles;
 };
 
-// Item field packing: head group in the low bits of .y, the item's length in
-// 16-key stages above them.
-constexpr int kItemSizeShift = 12;
-constexpr int kItemHgMask = (1 << kItemSizeShift) - 1;
-constexpr int kMaxItemStages = (1 << (31 - kItemSizeShift)) - 1;
+// Item field packing: head group in the low 16 bits of .y, the partition index
+// in the high 16 (partitions per row stay far below 2^15).
+constexpr int kItemPartShift = 16;
+constexpr int kItemHgMask = (1 << kItemPartShift) - 1;
 
 struct WsView {
   int32_t* ctrl;
