@@ -212,6 +212,7 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T* s_scan, T* total) {
 //     search over the rows' first items in shared memory.
 constexpr int kFastPerThread = 4;
 constexpr int kFastRows = kPlanThreads * kFastPerThread;
+constexpr int kMinSmallStages = 4;
 
 // The pieces of a row of n stages: nb big ones of pb stages (whole pieces
 // within 80 % of the row), then ns small ones of ps.  A row that would need
@@ -381,7 +382,9 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
       const double C = max(a.num_sms, 1);
       s_Pb = static_cast<int>(fmin(fmax(0.4 * work / C, static_cast<double>(a.min_part_stages)),
                                    1e9));
-      s_Ps = static_cast<int>(fmin(fmax(0.05 * work / C, static_cast<double>(a.min_part_stages)),
+      // (at least kMinSmallStages: smaller pieces cost more in the merge than
+      // they gain at the end)
+      s_Ps = static_cast<int>(fmin(fmax(0.05 * work / C, static_cast<double>(kMinSmallStages)),
                                    static_cast<double>(s_Pb)));
       *s_merge = 0;
       *s_merge_big = 0;
