@@ -304,6 +304,9 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         // lane holds 4 codes (dims 4j..4j+3) of one key per matrix
         const int mi = lane >> 3;
         const int key = (lane & 7) + ((mi & 1) << 3);
+        // two accumulator chains per half (even and odd 16-dim steps): the
+        // dependent mma chain of a stage is half as long
+        float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int kk = 0; kk < D / 16; kk += 2) {
           uint32_t r[4];
@@ -312,8 +315,14 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           for (int m = 0; m < 4; ++m) {
             const uint32_t lo = e4m3x2_to_f16x2(static_cast<uint16_t>(r[m] & 0xffffu));
             const uint32_t hi = e4m3x2_to_f16x2(static_cast<uint16_t>(r[m] >> 16));
-            mma_f16_16816((m & 1) ? s1 : s0, qa[kk + (m >> 1)], lo, hi);
+            float* acc = (m >> 1) ? ((m & 1) ? t1 : t0) : ((m & 1) ? s1 : s0);
+            mma_f16_16816(acc, qa[kk + (m >> 1)], lo, hi);
           }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          s0[e] += t0[e];
+          s1[e] += t1[e];
         }
       } else {
         const int mi = lane >> 3;
@@ -414,6 +423,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
         // zeroed after widening, as halves of the key pairs (2t, 2t+1) and
         // (2t+8, 2t+9) this lane holds
         const int t2 = 2 * (lane & 3);
+        const bool tail = nv < kStageTokens;  // only a request's last stage
         const uint32_t mk0 = (t2 < nv ? 0x0000ffffu : 0u) | (t2 + 1 < nv ? 0xffff0000u : 0u);
         const uint32_t mk1 = (t2 + 8 < nv ? 0x0000ffffu : 0u) | (t2 + 9 < nv ? 0xffff0000u : 0u);
 #pragma unroll
@@ -423,10 +433,14 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {  // code chunk 2q + h: even dims, then odd dims
             const uint32_t lo = prmt_b32(r[2 * h], 0x3120u), hi = prmt_b32(r[2 * h + 1], 0x3120u);
-            const uint32_t e0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo & 0xffffu)) & mk0;
-            const uint32_t e1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi & 0xffffu)) & mk1;
-            const uint32_t d0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo >> 16)) & mk0;
-            const uint32_t d1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi >> 16)) & mk1;
+            uint32_t e0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo & 0xffffu));
+            uint32_t e1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi & 0xffffu));
+            uint32_t d0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo >> 16));
+            uint32_t d1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi >> 16));
+            if (tail) {
+              e0 &= mk0, d0 &= mk0;
+              e1 &= mk1, d1 &= mk1;
+            }
             mma_f16_16816(o[2 * (2 * q + h)], pa, e0, e1);
             mma_f16_16816(o[2 * (2 * q + h) + 1], pa, d0, d1);
           }
