@@ -82,6 +82,42 @@ def test_fp8_every_code_decodes_exactly(cuda_device):
             assert np.array_equal(out[b, h], want[b]), (b, h)
 
 
+def test_fp8_every_key_code_scores_exactly(cuda_device):
+    """Two keys per request: key 0 holds one K code in one dim (the dim moves
+    with the code, so every k slot of the tensor-core fragments is used), key 1
+    is zero, and only key 0's V row is non-zero (1.0 in the same dim).  The
+    output there is v_scale * sigmoid(q . k), for all 254 finite e4m3 codes,
+    the subnormal ones (zero exponent) included."""
+    dev = cuda_device
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    n, d, hkv, hq, bs = len(codes), 128, 2, 8, 16
+    vals = oracle.e4m3_decode(codes).astype(np.float64)
+    dims = np.arange(n) % d
+    kp = np.zeros((n, bs, hkv, d), dtype=np.uint8)
+    vp = np.zeros((n, bs, hkv, d), dtype=np.uint8)
+    q = np.zeros((n, hq, d), dtype=np.float32)
+    heads = (np.arange(hq) - 3.5) * 0.5                  # scores of both signs
+    for b in range(n):
+        kp[b, 0, :, dims[b]] = codes[b]
+        vp[b, 0, :, dims[b]] = 0x38                       # 1.0
+        q[b, :, dims[b]] = heads / (vals[b] if vals[b] != 0 else 1.0)
+    qb = torch.from_numpy(q).to(torch.bfloat16)
+    k_scale, v_scale, sm = 1.0, 0.5, 1.0
+    out = P.decode(qb.to(dev), torch.from_numpy(kp).view(torch.float8_e4m3fn).to(dev),
+                   torch.from_numpy(vp).view(torch.float8_e4m3fn).to(dev),
+                   torch.arange(n, dtype=torch.int32, device=dev).view(n, 1),
+                   torch.full((n,), 2, dtype=torch.int32, device=dev), sm,
+                   kv_scales=(k_scale, v_scale)).cpu().numpy().astype(np.float64)
+    qd = qb.float().numpy().astype(np.float64)
+    for b in range(n):
+        s0 = qd[b, :, dims[b]] * vals[b] * k_scale * sm
+        want = v_scale / (1.0 + np.exp(-s0))
+        got = out[b, :, dims[b]]
+        assert np.allclose(got, want, rtol=2e-3, atol=1e-6), (hex(codes[b]), got, want)
+        rest = np.delete(out[b], dims[b], axis=1)
+        assert np.all(rest == 0), hex(codes[b])
+
+
 def test_fp8_cache_write_saturates_and_skips(cuda_device):
     dev = cuda_device
     T, hkv, d, nb, bs = 6, 2, 64, 4, 8
