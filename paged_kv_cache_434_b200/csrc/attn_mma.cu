@@ -247,6 +247,7 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
   // score and output scales (the pools' k_scale / v_scale are already in g)
   const float sl2 = g.scale_log2;
   const float vsc = g.v_scale;
+  constexpr bool kPair = F8;
 
   for (;;) {
     if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs)) {
@@ -290,64 +291,171 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       l0 = l1 = 0.f;
       bad = false;
     }
-    bool released = false;
+    // F8: the next stage, when it belongs to the same item, is taken with this
+    // one: one softmax pass over 32 keys and twice the independent products
+    // per pass (the e4m3 path is bound by the latency of each warp's chain)
+    int stage2 = -1;
+    mmak::StageInfo si2 = si;
+    if (kPair && !(si.flags & (mmak::kLast | mmak::kBad))) {
+      const int s2 = stage + 1 == NS ? 0 : stage + 1;
+      const uint32_t ph2 = stage + 1 == NS ? phase ^ 1u : phase;
+      if (!mbar_wait_bounded(&full[s2], ph2, kWaitLimitNs)) {
+        if (g.err_word && lane == 0) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
+        break;
+      }
+      si2 = info[s2];
+      if (!(si2.flags & mmak::kBad)) stage2 = s2;  // a bad stage is taken alone
+      else si2 = si;
+    }
     if (si.flags & mmak::kBad) {
       bad = true;
     } else {
-      uint32_t kt = smem_u32(stages + stage * C::kStageBytes) + hh * C::kTile;
-      uint32_t vt = kt + C::kTensorBytes;
       constexpr uint32_t kHalf = HG * C::kTile;  // between the two halves (bf16)
-      // ---- S = Q K^T over 16 keys
-      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (F8) {
-        // one ldmatrix of the code tile gives two 16-dim steps x 16 keys: a
-        // lane holds 4 codes (dims 4j..4j+3) of one key per matrix
-        const int mi = lane >> 3;
-        const int key = (lane & 7) + ((mi & 1) << 3);
-        // two accumulator chains per half (even and odd 16-dim steps): the
-        // dependent mma chain of a stage is half as long
-        float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+      // ---- S = Q K^T over the 16 keys of stage stg
+      auto qk = [&](int stg, float* a0, float* a1) {
+        const uint32_t kt = smem_u32(stages + stg * C::kStageBytes) + hh * C::kTile;
+        if constexpr (F8) {
+          // one ldmatrix of the code tile gives two 16-dim steps x 16 keys: a
+          // lane holds 4 codes (dims 4j..4j+3) of one key per matrix
+          const int mi = lane >> 3;
+          const int key = (lane & 7) + ((mi & 1) << 3);
+          // two accumulator chains per half (even and odd 16-dim steps): the
+          // dependent mma chain of a stage is half as long
+          float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int kk = 0; kk < D / 16; kk += 2) {
-          uint32_t r[4];
-          ldmatrix_x4(kt + mmak::swz(key, kk + (mi >> 1)), r[0], r[1], r[2], r[3]);
+          for (int kk = 0; kk < D / 16; kk += 2) {
+            uint32_t r[4];
+            ldmatrix_x4(kt + mmak::swz(key, kk + (mi >> 1)), r[0], r[1], r[2], r[3]);
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint32_t lo = e4m3x2_to_f16x2(static_cast<uint16_t>(r[m] & 0xffffu));
-            const uint32_t hi = e4m3x2_to_f16x2(static_cast<uint16_t>(r[m] >> 16));
-            float* acc = (m >> 1) ? ((m & 1) ? t1 : t0) : ((m & 1) ? s1 : s0);
-            mma_f16_16816(acc, qa[kk + (m >> 1)], lo, hi);
+            for (int m = 0; m < 4; ++m) {
+              const uint32_t lo = e4m3x2_to_f16x2(static_cast<uint16_t>(r[m] & 0xffffu));
+              const uint32_t hi = e4m3x2_to_f16x2(static_cast<uint16_t>(r[m] >> 16));
+              float* acc = (m >> 1) ? ((m & 1) ? t1 : t0) : ((m & 1) ? a1 : a0);
+              mma_f16_16816(acc, qa[kk + (m >> 1)], lo, hi);
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            a0[e] += t0[e];
+            a1[e] += t1[e];
+          }
+        } else {
+          const int mi = lane >> 3;
+          const int key = (lane & 7) + ((mi >> 1) << 3);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int dh = kk >> 2, c16 = kk & 3;
+            const int chunk = 2 * c16 + (mi & 1);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(kt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
+            mma_bf16_16816(a0, qa[kk], b0, b1);
+            mma_bf16_16816(a1, qa[kk], b2, b3);
           }
         }
+      };
+      // ---- O += P V over the 16 keys of stage stg (nv of them valid)
+      auto pv = [&](int stg, const uint32_t* pa, int nv) {
+        const uint32_t vt = smem_u32(stages + stg * C::kStageBytes) + hh * C::kTile + C::kTensorBytes;
+        // keys past the end of the request: zero their V rows (P is 0 there,
+        // but the pool may hold non-finite garbage and 0 * inf is NaN)
+        if (!F8 && nv < kStageTokens) {
+          uint8_t* vrow = stages + stg * C::kStageBytes + C::kTensorBytes + hh * C::kTile;
+          for (int idx = lane; idx < (kStageTokens - nv) * 8 * NH; idx += 32) {
+            const int dh = idx / ((kStageTokens - nv) * 8);
+            const int rem = idx % ((kStageTokens - nv) * 8);
+            const int key = nv + rem / 8, chunk = rem % 8;
+            *reinterpret_cast<uint4*>(vrow + dh * HG * C::kTile + mmak::swz(key, chunk)) =
+                make_uint4(0, 0, 0, 0);
+          }
+          __syncwarp();
+        }
+        if constexpr (F8) {
+          // matrices: keys 0-7 / 8-15 of code chunk 2q, then of chunk 2q + 1
+          const int mi = lane >> 3;
+          const int key = (lane & 7) + ((mi & 1) << 3);
+          // keys past the end of the request: their (possibly NaN) codes are
+          // zeroed after widening, as halves of the key pairs (2t, 2t+1) and
+          // (2t+8, 2t+9) this lane holds
+          const int t2 = 2 * (lane & 3);
+          const bool tail = nv < kStageTokens;  // only a request's last stage
+          const uint32_t mk0 = (t2 < nv ? 0x0000ffffu : 0u) | (t2 + 1 < nv ? 0xffff0000u : 0u);
+          const uint32_t mk1 = (t2 + 8 < nv ? 0x0000ffffu : 0u) | (t2 + 9 < nv ? 0xffff0000u : 0u);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          s0[e] += t0[e];
-          s1[e] += t1[e];
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t r[4];
+            ldmatrix_x4_trans(vt + mmak::swz(key, 2 * q + (mi >> 1)), r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // code chunk 2q + h: even dims, then odd dims
+              const uint32_t lo = prmt_b32(r[2 * h], 0x3120u), hi = prmt_b32(r[2 * h + 1], 0x3120u);
+              uint32_t e0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo & 0xffffu));
+              uint32_t e1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi & 0xffffu));
+              uint32_t d0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo >> 16));
+              uint32_t d1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi >> 16));
+              if (tail) {
+                e0 &= mk0, d0 &= mk0;
+                e1 &= mk1, d1 &= mk1;
+              }
+              mma_f16_16816(o[2 * (2 * q + h)], pa, e0, e1);
+              mma_f16_16816(o[2 * (2 * q + h) + 1], pa, d0, d1);
+            }
+          }
+        } else {
+          const int mi = lane >> 3;
+          const int key = (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+          for (int n2 = 0; n2 < D / 16; ++n2) {
+            const int dh = n2 >> 2, c16 = n2 & 3;
+            const int chunk = 2 * c16 + (mi >> 1);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4_trans(vt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
+            mma_bf16_16816(o[2 * n2], pa, b0, b1);
+            mma_bf16_16816(o[2 * n2 + 1], pa, b2, b3);
+          }
+        }
+        if (!F8 && nv < kStageTokens) fence_proxy_async_smem();
+      };
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+      float u0[4] = {0.f, 0.f, 0.f, 0.f}, u1[4] = {0.f, 0.f, 0.f, 0.f};
+      if (kPair && stage2 >= 0) {
+        // both stages' products in one unrolled loop: independent chains interleave
+        const uint32_t ka = smem_u32(stages + stage * C::kStageBytes) + hh * C::kTile;
+        const uint32_t kb = smem_u32(stages + stage2 * C::kStageBytes) + hh * C::kTile;
+        const int mi = lane >> 3;
+        const int key = (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; kk += 2) {
+          uint32_t ra[4], rb[4];
+          ldmatrix_x4(ka + mmak::swz(key, kk + (mi >> 1)), ra[0], ra[1], ra[2], ra[3]);
+          ldmatrix_x4(kb + mmak::swz(key, kk + (mi >> 1)), rb[0], rb[1], rb[2], rb[3]);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int step = kk + (m >> 1);
+            mma_f16_16816((m & 1) ? s1 : s0, qa[step],
+                          e4m3x2_to_f16x2(static_cast<uint16_t>(ra[m] & 0xffffu)),
+                          e4m3x2_to_f16x2(static_cast<uint16_t>(ra[m] >> 16)));
+            mma_f16_16816((m & 1) ? u1 : u0, qa[step],
+                          e4m3x2_to_f16x2(static_cast<uint16_t>(rb[m] & 0xffffu)),
+                          e4m3x2_to_f16x2(static_cast<uint16_t>(rb[m] >> 16)));
+          }
         }
       } else {
-        const int mi = lane >> 3;
-        const int key = (lane & 7) + ((mi >> 1) << 3);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int dh = kk >> 2, c16 = kk & 3;
-          const int chunk = 2 * c16 + (mi & 1);
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4(kt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
-          mma_bf16_16816(s0, qa[kk], b0, b1);
-          mma_bf16_16816(s1, qa[kk], b2, b3);
-        }
+        qk(stage, s0, s1);
       }
-      // ---- mask, scale, online softmax
-      const int nv = si.nvalid;
-      float p[8];
+      // ---- mask, scale, online softmax (over both stages when paired)
+      const int nv = si.nvalid, nv2 = stage2 >= 0 ? si2.nvalid : 0;
+      float p[8], p2[8];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int key = qc + (e & 1);
         p[e] = key < nv ? s0[e] * sl2 : -INFINITY;
         p[4 + e] = key + 8 < nv ? s1[e] * sl2 : -INFINITY;
+        p2[e] = key < nv2 ? u0[e] * sl2 : -INFINITY;
+        p2[4 + e] = key + 8 < nv2 ? u1[e] * sl2 : -INFINITY;
       }
-      float mx0 = fmaxf(fmaxf(p[0], p[1]), fmaxf(p[4], p[5]));
-      float mx1 = fmaxf(fmaxf(p[2], p[3]), fmaxf(p[6], p[7]));
+      float mx0 = fmaxf(fmaxf(fmaxf(p[0], p[1]), fmaxf(p[4], p[5])),
+                        fmaxf(fmaxf(p2[0], p2[1]), fmaxf(p2[4], p2[5])));
+      float mx1 = fmaxf(fmaxf(fmaxf(p[2], p[3]), fmaxf(p[6], p[7])),
+                        fmaxf(fmaxf(p2[2], p2[3]), fmaxf(p2[6], p2[7])));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
@@ -362,13 +470,13 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
       const bool rescale = __any_sync(0xffffffffu, up0 || up1);
       m0 = mn0;
       m1 = mn1;
-      uint32_t pa[4];
-      float ps0 = 0.f, ps1 = 0.f;
-      {
-        const float e0 = fast_exp2(p[0] - mn0), e1 = fast_exp2(p[1] - mn0);
-        const float e2 = fast_exp2(p[2] - mn1), e3 = fast_exp2(p[3] - mn1);
-        const float e4 = fast_exp2(p[4] - mn0), e5 = fast_exp2(p[5] - mn0);
-        const float e6 = fast_exp2(p[6] - mn1), e7 = fast_exp2(p[7] - mn1);
+      // P as the A fragment of the PV product; the row sums use the same
+      // rounded weights the product sees
+      auto weights = [&](const float* q, uint32_t* pa, float& ps0, float& ps1) {
+        const float e0 = fast_exp2(q[0] - mn0), e1 = fast_exp2(q[1] - mn0);
+        const float e2 = fast_exp2(q[2] - mn1), e3 = fast_exp2(q[3] - mn1);
+        const float e4 = fast_exp2(q[4] - mn0), e5 = fast_exp2(q[5] - mn0);
+        const float e6 = fast_exp2(q[6] - mn1), e7 = fast_exp2(q[7] - mn1);
         float2 f0, f1, f2, f3;
         if constexpr (F8) {
           pa[0] = pack_f16x2(e0, e1);
@@ -386,10 +494,13 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
           f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
         }
-        // the row sums use the same rounded weights the PV product sees
-        ps0 = f0.x + f0.y + f2.x + f2.y;
-        ps1 = f1.x + f1.y + f3.x + f3.y;
-      }
+        ps0 += f0.x + f0.y + f2.x + f2.y;
+        ps1 += f1.x + f1.y + f3.x + f3.y;
+      };
+      uint32_t pa[4], pa2[4];
+      float ps0 = 0.f, ps1 = 0.f;
+      weights(p, pa, ps0, ps1);
+      if (stage2 >= 0) weights(p2, pa2, ps0, ps1);
       l0 = l0 * a0 + ps0;
       l1 = l1 * a1 + ps1;
       if (rescale) {
@@ -401,69 +512,59 @@ __global__ void __launch_bounds__((HG + 1) * 32, 1)
           o[j][3] *= a1;
         }
       }
-      // ---- keys past the end of the request: zero their V rows (P is 0 there,
-      // but the pool may hold non-finite garbage and 0 * inf is NaN)
-      if (!F8 && nv < kStageTokens) {
-        uint8_t* vrow = stages + stage * C::kStageBytes + C::kTensorBytes + hh * C::kTile;
-        for (int idx = lane; idx < (kStageTokens - nv) * 8 * NH; idx += 32) {
-          const int dh = idx / ((kStageTokens - nv) * 8);
-          const int rem = idx % ((kStageTokens - nv) * 8);
-          const int key = nv + rem / 8, chunk = rem % 8;
-          *reinterpret_cast<uint4*>(vrow + dh * HG * C::kTile + mmak::swz(key, chunk)) =
-              make_uint4(0, 0, 0, 0);
-        }
-        __syncwarp();
-      }
-      // ---- O += P V
-      if constexpr (F8) {
-        // matrices: keys 0-7 / 8-15 of code chunk 2q, then of chunk 2q + 1
+      if (kPair && stage2 >= 0) {
+        // both stages in one unrolled loop (the first is whole: it is not an
+        // item's last stage; the second may end the request)
+        const uint32_t va = smem_u32(stages + stage * C::kStageBytes) + hh * C::kTile + C::kTensorBytes;
+        const uint32_t vb = smem_u32(stages + stage2 * C::kStageBytes) + hh * C::kTile + C::kTensorBytes;
         const int mi = lane >> 3;
         const int key = (lane & 7) + ((mi & 1) << 3);
-        // keys past the end of the request: their (possibly NaN) codes are
-        // zeroed after widening, as halves of the key pairs (2t, 2t+1) and
-        // (2t+8, 2t+9) this lane holds
         const int t2 = 2 * (lane & 3);
-        const bool tail = nv < kStageTokens;  // only a request's last stage
-        const uint32_t mk0 = (t2 < nv ? 0x0000ffffu : 0u) | (t2 + 1 < nv ? 0xffff0000u : 0u);
-        const uint32_t mk1 = (t2 + 8 < nv ? 0x0000ffffu : 0u) | (t2 + 9 < nv ? 0xffff0000u : 0u);
+        const bool tail = nv2 < kStageTokens;
+        const uint32_t mk0 = (t2 < nv2 ? 0x0000ffffu : 0u) | (t2 + 1 < nv2 ? 0xffff0000u : 0u);
+        const uint32_t mk1 = (t2 + 8 < nv2 ? 0x0000ffffu : 0u) | (t2 + 9 < nv2 ? 0xffff0000u : 0u);
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
-          uint32_t r[4];
-          ldmatrix_x4_trans(vt + mmak::swz(key, 2 * q + (mi >> 1)), r[0], r[1], r[2], r[3]);
+          uint32_t ra[4], rb[4];
+          ldmatrix_x4_trans(va + mmak::swz(key, 2 * q + (mi >> 1)), ra[0], ra[1], ra[2], ra[3]);
+          ldmatrix_x4_trans(vb + mmak::swz(key, 2 * q + (mi >> 1)), rb[0], rb[1], rb[2], rb[3]);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {  // code chunk 2q + h: even dims, then odd dims
-            const uint32_t lo = prmt_b32(r[2 * h], 0x3120u), hi = prmt_b32(r[2 * h + 1], 0x3120u);
-            uint32_t e0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo & 0xffffu));
-            uint32_t e1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi & 0xffffu));
-            uint32_t d0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lo >> 16));
-            uint32_t d1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hi >> 16));
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t la = prmt_b32(ra[2 * h], 0x3120u), ha = prmt_b32(ra[2 * h + 1], 0x3120u);
+            const uint32_t lb = prmt_b32(rb[2 * h], 0x3120u), hb = prmt_b32(rb[2 * h + 1], 0x3120u);
+            uint32_t e0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lb & 0xffffu));
+            uint32_t e1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hb & 0xffffu));
+            uint32_t d0 = e4m3x2_to_f16x2(static_cast<uint16_t>(lb >> 16));
+            uint32_t d1 = e4m3x2_to_f16x2(static_cast<uint16_t>(hb >> 16));
             if (tail) {
               e0 &= mk0, d0 &= mk0;
               e1 &= mk1, d1 &= mk1;
             }
-            mma_f16_16816(o[2 * (2 * q + h)], pa, e0, e1);
-            mma_f16_16816(o[2 * (2 * q + h) + 1], pa, d0, d1);
+            mma_f16_16816(o[2 * (2 * q + h)], pa, e4m3x2_to_f16x2(static_cast<uint16_t>(la & 0xffffu)),
+                          e4m3x2_to_f16x2(static_cast<uint16_t>(ha & 0xffffu)));
+            mma_f16_16816(o[2 * (2 * q + h) + 1], pa, e4m3x2_to_f16x2(static_cast<uint16_t>(la >> 16)),
+                          e4m3x2_to_f16x2(static_cast<uint16_t>(ha >> 16)));
+            mma_f16_16816(o[2 * (2 * q + h)], pa2, e0, e1);
+            mma_f16_16816(o[2 * (2 * q + h) + 1], pa2, d0, d1);
           }
         }
       } else {
-        const int mi = lane >> 3;
-        const int key = (lane & 7) + ((mi & 1) << 3);
-#pragma unroll
-        for (int n2 = 0; n2 < D / 16; ++n2) {
-          const int dh = n2 >> 2, c16 = n2 & 3;
-          const int chunk = 2 * c16 + (mi >> 1);
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4_trans(vt + dh * kHalf + mmak::swz(key, chunk), b0, b1, b2, b3);
-          mma_bf16_16816(o[2 * n2], pa, b0, b1);
-          mma_bf16_16816(o[2 * n2 + 1], pa, b2, b3);
-        }
+        pv(stage, pa, nv);
       }
-      if (!F8 && nv < kStageTokens) fence_proxy_async_smem();
     }
     __syncwarp();
-    if (lane == 0 && !released) mbar_arrive(&empty[stage]);
+    if (lane == 0) {
+      mbar_arrive(&empty[stage]);
+      if (stage2 >= 0) mbar_arrive(&empty[stage2]);
+    }
+    if (stage2 >= 0) {  // the paired stage is consumed too
+      if (++stage == NS) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
 
-    if (si.flags & mmak::kLast) {
+    if (si2.flags & mmak::kLast) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
