@@ -67,7 +67,10 @@ typedef enum pa_status {
   PA_ERR_UNSUPPORTED = 2,  /* valid but unsupported (dtype, head_dim, ...)       */
   PA_ERR_WORKSPACE = 3,    /* workspace pointer NULL or smaller than required    */
   PA_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute ...) */
-  PA_ERR_DEVICE = 5        /* pa_read_error found device error bits set          */
+  PA_ERR_DEVICE_OOB = 5,   /* pa_read_error: the device found out-of-range input
+                              (any error bit but PA_ERRBIT_TIMEOUT)              */
+  PA_ERR_TIMEOUT = 6       /* pa_read_error: a bounded device wait gave up
+                              (PA_ERRBIT_TIMEOUT set, whatever else is)          */
 } pa_status;
 
 /* PA_FP8_E4M3: the pools hold e4m3 codes (1 sign, 4 exponent bits with bias
@@ -340,8 +343,9 @@ pa_status pa_kernel_timing_read(float* ms);
 
 /*
  * pa_read_error -- synchronise `stream`, copy *err_word to *host_bits and
- * reset it to 0.  Returns PA_OK when no bit was set, PA_ERR_DEVICE when some
- * were, PA_ERR_CUDA if a CUDA call failed (e.g. an earlier kernel faulted).
+ * reset it to 0.  Returns PA_OK when no bit was set, PA_ERR_TIMEOUT when
+ * PA_ERRBIT_TIMEOUT was set, PA_ERR_DEVICE_OOB when only other bits were,
+ * PA_ERR_CUDA if a CUDA call failed (e.g. an earlier kernel faulted).
  */
 pa_status pa_read_error(int32_t* err_word, int32_t* host_bits, void* stream);
 

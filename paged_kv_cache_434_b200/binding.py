@@ -16,7 +16,8 @@ import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libpa_b200.so")
 
-PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_DEVICE = range(6)
+(PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA, PA_ERR_DEVICE_OOB,
+ PA_ERR_TIMEOUT) = range(7)
 PA_F32, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
 
 ERRBIT_SLOT_OOB = 0x1
@@ -195,7 +196,7 @@ def read_error(err: torch.Tensor) -> int:
     """Synchronise the current stream, return the error bits and clear them."""
     bits = ctypes.c_int32(0)
     st = _lib().pa_read_error(_cuda(err, "err", torch.int32), ctypes.byref(bits), _stream())
-    if st not in (PA_OK, PA_ERR_DEVICE):
+    if st not in (PA_OK, PA_ERR_DEVICE_OOB, PA_ERR_TIMEOUT):
         raise PagedAttentionError(st, "pa_read_error")
     return bits.value
 

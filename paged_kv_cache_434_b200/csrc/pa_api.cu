@@ -267,7 +267,8 @@ const char* pa_status_str(int status) {
     case PA_ERR_UNSUPPORTED: return "unsupported configuration";
     case PA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case PA_ERR_CUDA: return "CUDA runtime error";
-    case PA_ERR_DEVICE: return "device reported error bits";
+    case PA_ERR_DEVICE_OOB: return "device found out-of-range input (error bits set)";
+    case PA_ERR_TIMEOUT: return "a bounded device wait gave up";
     default: return "unknown status";
   }
 }
@@ -542,7 +543,8 @@ pa_status pa_read_error(int32_t* err_word, int32_t* host_bits, void* stream) {
   if (cudaMemsetAsync(err_word, 0, sizeof(int32_t), s) != cudaSuccess) return PA_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return PA_ERR_CUDA;
   *host_bits = h;
-  return h ? PA_ERR_DEVICE : PA_OK;
+  if (h & PA_ERRBIT_TIMEOUT) return PA_ERR_TIMEOUT;
+  return h ? PA_ERR_DEVICE_OOB : PA_OK;
 }
 
 }  // extern "C"

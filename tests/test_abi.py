@@ -46,8 +46,8 @@ def test_binding_covers_every_export():
 
 
 def test_status_strings(lib):
-    for s in range(6):
-        assert lib.pa_status_str(s)
+    for s in range(7):
+        assert lib.pa_status_str(s) and lib.pa_status_str(s) != b"unknown status", s
     assert lib.pa_status_str(99) == b"unknown status"
     assert lib.pa_version() >= 100
 
@@ -267,7 +267,8 @@ def test_binding_constants_match_the_header():
     text = _header_text()
     enums = dict((k, int(v)) for k, v in re.findall(r"\b(PA_[A-Z0-9_]+)\s*=\s*(\d+)", text))
     for name in ("PA_OK", "PA_ERR_INVALID_ARG", "PA_ERR_UNSUPPORTED", "PA_ERR_WORKSPACE",
-                 "PA_ERR_CUDA", "PA_ERR_DEVICE", "PA_F32", "PA_BF16", "PA_FP8_E4M3"):
+                 "PA_ERR_CUDA", "PA_ERR_DEVICE_OOB", "PA_ERR_TIMEOUT", "PA_F32", "PA_BF16",
+                 "PA_FP8_E4M3"):
         assert getattr(B, name) == enums[name], name
     defines = dict(re.findall(r"#define\s+(PA_[A-Z0-9_]+)\s+\(?([0-9a-fx]+)", text))
     bits = {k: int(v, 0) for k, v in defines.items() if k.startswith("PA_ERRBIT_")}

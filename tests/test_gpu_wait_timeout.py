@@ -52,3 +52,24 @@ def test_limit_outside_its_range_is_refused(cuda_device):
         with pytest.raises(B.PagedAttentionError) as e:
             B.selftest_wait_timeout(bad, err)
         assert e.value.status == B.PA_ERR_INVALID_ARG
+
+
+def test_read_error_status_names_the_condition(cuda_device):
+    """pa_read_error's status: PA_ERR_TIMEOUT once a wait gave up (whatever
+    other bits are set), PA_ERR_DEVICE_OOB for out-of-range input alone, PA_OK
+    for a clean word; the bits come back either way."""
+    import ctypes
+
+    def status(word):
+        bits = ctypes.c_int32(0)
+        st = B._lib().pa_read_error(ctypes.c_void_p(word.data_ptr()), ctypes.byref(bits),
+                                    ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        return st, bits.value
+
+    err = P.new_error_word(cuda_device)
+    B.selftest_wait_timeout(1000, err)
+    err.add_(B.ERRBIT_BLOCK_OOB)          # queued after the wait on the same stream
+    assert status(err) == (B.PA_ERR_TIMEOUT, B.ERRBIT_TIMEOUT | B.ERRBIT_BLOCK_OOB)
+    err.fill_(B.ERRBIT_SEQ_TOO_LONG)
+    assert status(err) == (B.PA_ERR_DEVICE_OOB, B.ERRBIT_SEQ_TOO_LONG)
+    assert status(err) == (B.PA_OK, 0)
