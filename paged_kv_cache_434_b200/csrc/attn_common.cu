@@ -504,7 +504,7 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
     ws.qrow_bad[r] = 0;
     ws.nparts[r] = n;
     ws.qrow_info[r] = n >= 0 ? make_int4(r, L[k], 1, prefix) : make_int4(-1, 0, 0, 0);
-    if (n > 32) ws.merge_rows[g.num_qrows - 1 - atomicAdd(s_merge_big, 1)] = r;
+    if (n > kMergeWarpParts) ws.merge_rows[g.num_qrows - 1 - atomicAdd(s_merge_big, 1)] = r;
     else if (n >= 0 && n != 1) ws.merge_rows[atomicAdd(s_merge, 1)] = r;
   }
   __syncthreads();
@@ -810,7 +810,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     ws.nparts[r] = np + (info.w > 0 ? prefix_chunks : 0);  // the last ones: shared-prefix chunks
     // rows to merge: those a warp merges from the front of the list, those
     // with more than 32 partitions (a CTA each) from the back
-    if (ws.nparts[r] > 32)
+    if (ws.nparts[r] > kMergeWarpParts)
       ws.merge_rows[g.num_qrows - 1 - atomicAdd(&s_merge_big, 1)] = r;
     else if (ws.nparts[r] != 1)
       ws.merge_rows[atomicAdd(&s_merge, 1)] = r;
@@ -1109,10 +1109,10 @@ cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms
 // ======================================================================= merge
 // Rows with a single partition were written by the attention kernel; rows with
 // none get zeros; invalid rows are skipped.  The rows to merge come from the
-// planner's list.  Pass 1: one warp per (row, query head) whose partitions fit
-// in a warp (<= 32): lane k holds partition k's (m, l), the weights
-// 2^(m_k - M) are shuffled to all lanes and each lane accumulates D/32 output
-// columns.  Pass 2: one 32-warp CTA per remaining (row, head): max and
+// planner's list.  Pass 1: one warp per (row, query head) with at most
+// kMergeWarpParts (64) partitions: lane k holds partitions k and k + 32 (m, l),
+// the weights 2^(m_k - M) are shuffled to all lanes and each lane accumulates
+// D/32 output columns.  Pass 2: one 32-warp CTA per remaining (row, head): max and
 // denominator reduced over the CTA, then each warp accumulates every 8th
 // partition (4 in flight) and the warp sums are combined.
 constexpr int kMergeWarps = 32;
@@ -1129,12 +1129,14 @@ __device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView&
     return;
   }
   const int64_t base = idx * ws.max_parts;
-  const float2 ml = lane < np ? ws.part_ml[base + lane] : make_float2(-INFINITY, 0.f);
-  float M = ml.x;
+  const float2 ml0 = lane < np ? ws.part_ml[base + lane] : make_float2(-INFINITY, 0.f);
+  const float2 ml1 = lane + 32 < np ? ws.part_ml[base + lane + 32] : make_float2(-INFINITY, 0.f);
+  float M = fmaxf(ml0.x, ml1.x);
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float c = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
-  float den = c * ml.y;
+  const float c0 = (ml0.x == -INFINITY) ? 0.f : fast_exp2(ml0.x - M);
+  const float c1 = (ml1.x == -INFINITY) ? 0.f : fast_exp2(ml1.x - M);
+  float den = c0 * ml0.y + c1 * ml1.y;
 #pragma unroll
   for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   float acc[V];
@@ -1142,7 +1144,7 @@ __device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView&
   for (int e = 0; e < V; ++e) acc[e] = 0.f;
   const float* po = ws.part_o + base * D + lane * V;
   // up to 8 partial rows in flight per lane (and 32 warps per SM): a row of
-  // at most 32 partitions takes at most four round trips to L2
+  // at most 64 partitions takes at most eight round trips to L2
   constexpr int kBatch = 8;
   for (int k0 = 0; k0 < np; k0 += kBatch) {
     float x[kBatch][V];
@@ -1160,7 +1162,8 @@ __device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView&
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const float cu = __shfl_sync(0xffffffffu, c, min(k0 + u, 31));
+      const int k = min(k0 + u, kMergeWarpParts - 1);  // warp-uniform
+      const float cu = __shfl_sync(0xffffffffu, k < 32 ? c0 : c1, k & 31);
 #pragma unroll
       for (int e = 0; e < V; ++e) acc[e] = fmaf(x[u][e], cu, acc[e]);
     }
@@ -1180,12 +1183,14 @@ __global__ void __launch_bounds__(kMergeWarps * 32, 1) merge_kernel(AttnGeom g, 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t pairs = static_cast<int64_t>(ws.ctrl[5]) * g.num_heads;
   const int64_t big_pairs = static_cast<int64_t>(ws.ctrl[9]) * g.num_heads;
-  // pass 1: (row, head) pairs with at most 32 partitions, one warp each
-  for (int64_t pi = static_cast<int64_t>(blockIdx.x) * kMergeWarps + warp; pi < pairs;
+  // pass 1: (row, head) pairs with at most kMergeWarpParts partitions, one warp
+  // each, spread over the CTAs first (pair i on CTA i % grid): a batch of few
+  // pairs then loads its partials through every SM, not through a few
+  for (int64_t pi = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; pi < pairs;
        pi += static_cast<int64_t>(gridDim.x) * kMergeWarps) {
     const int r = ws.merge_rows[pi / g.num_heads];
     const int np = ws.nparts[r];
-    if (np == 1 || np < 0 || np > 32 || ws.qrow_bad[r]) continue;
+    if (np == 1 || np < 0 || np > kMergeWarpParts || ws.qrow_bad[r]) continue;
     merge_pair_warp<D>(g, ws, static_cast<int64_t>(r) * g.num_heads + pi % g.num_heads, np, lane);
   }
   // pass 2: pairs with more partitions (listed from the back), one CTA each
@@ -1193,7 +1198,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32, 1) merge_kernel(AttnGeom g, 
     const int r = ws.merge_rows[g.num_qrows - 1 - pi / g.num_heads];
     const int64_t idx = static_cast<int64_t>(r) * g.num_heads + pi % g.num_heads;
     const int np = ws.nparts[r];
-    if (np <= 32 || ws.qrow_bad[r]) continue;
+    if (np <= kMergeWarpParts || ws.qrow_bad[r]) continue;
     const int64_t out_base = idx * D;
     const int64_t base = idx * ws.max_parts;
     // M

@@ -112,6 +112,9 @@ struct PlanArgs {
 constexpr int kCascadeMinPrefix = 256;
 constexpr int kCascadeMinSeqs = 16;
 constexpr int kMaxPrefixChunks = 8;  // partitions reserved per row for the shared prefix
+// rows with at most this many split-KV partitions are merged by one warp per
+// (row, head); the others by one CTA per (row, head)
+constexpr int kMergeWarpParts = 64;
 
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error.
