@@ -1129,6 +1129,27 @@ __device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView&
     return;
   }
   const int64_t base = idx * ws.max_parts;
+  const float* po = ws.part_o + base * D + lane * V;
+  // up to 8 partial rows in flight per lane (and 32 warps per SM); the first
+  // batch is requested before the weights, so that its round trip to L2
+  // overlaps the one of the (m, l) pairs
+  constexpr int kBatch = 8;
+  float x[kBatch][V];
+  auto load_batch = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const bool ok = k0 + u < np;
+      if constexpr (V == 4) {
+        const float4 t4 = ok ? *reinterpret_cast<const float4*>(po + static_cast<int64_t>(k0 + u) * D)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u][0] = t4.x, x[u][1] = t4.y, x[u][2] = t4.z, x[u][3] = t4.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < V; ++e) x[u][e] = ok ? po[static_cast<int64_t>(k0 + u) * D + e] : 0.f;
+      }
+    }
+  };
+  load_batch(0);
   const float2 ml0 = lane < np ? ws.part_ml[base + lane] : make_float2(-INFINITY, 0.f);
   const float2 ml1 = lane + 32 < np ? ws.part_ml[base + lane + 32] : make_float2(-INFINITY, 0.f);
   float M = fmaxf(ml0.x, ml1.x);
@@ -1142,24 +1163,8 @@ __device__ __forceinline__ void merge_pair_warp(const AttnGeom& g, const WsView&
   float acc[V];
 #pragma unroll
   for (int e = 0; e < V; ++e) acc[e] = 0.f;
-  const float* po = ws.part_o + base * D + lane * V;
-  // up to 8 partial rows in flight per lane (and 32 warps per SM): a row of
-  // at most 64 partitions takes at most eight round trips to L2
-  constexpr int kBatch = 8;
   for (int k0 = 0; k0 < np; k0 += kBatch) {
-    float x[kBatch][V];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const bool ok = k0 + u < np;
-      if constexpr (V == 4) {
-        const float4 t4 = ok ? *reinterpret_cast<const float4*>(po + static_cast<int64_t>(k0 + u) * D)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        x[u][0] = t4.x, x[u][1] = t4.y, x[u][2] = t4.z, x[u][3] = t4.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < V; ++e) x[u][e] = ok ? po[static_cast<int64_t>(k0 + u) * D + e] : 0.f;
-      }
-    }
+    if (k0 > 0) load_batch(k0);
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int k = min(k0 + u, kMergeWarpParts - 1);  // warp-uniform
