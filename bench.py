@@ -573,16 +573,30 @@ def measure(args, name, rank, world, local, with_e2e=True, with_cpu=True):
             if own is not None and "bf16_gemm_tflops" in own:
                 prefill_roofline["frac_of_own_gemm"] = round(tf / own["bf16_gemm_tflops"], 4)
 
-    # ---- end to end: host buffers in, result back to the host, each step
+    # ---- end to end: host buffers in, result back to the host, each step.
+    # The step's inputs (Q, new K/V, tables, lengths, query offsets) sit in one
+    # pinned host buffer and go over in one copy, into one device buffer that
+    # the call reads through views; the output comes back in one copy.
     e2e = None
     if with_e2e and not args.no_e2e:
-        names = ["q", "k_new", "v_new"]
-        host = {n: t[n].cpu().pin_memory() for n in names}
-        host_idx = {n: idx[n].cpu().pin_memory() for n in ("block_tables", "seq_lens",
-                                                            "query_start_loc")}
+        segs = [(t, n) for n in ("q", "k_new", "v_new")] + \
+               [(idx, n) for n in ("block_tables", "seq_lens", "query_start_loc")
+                if idx.get(n) is not None]
+        offs, tot = [], 0
+        for src, n in segs:
+            tot = (tot + 255) // 256 * 256  # every view 256-byte aligned
+            offs.append(tot)
+            tot += src[n].numel() * src[n].element_size()
+        host_buf = torch.empty(tot, dtype=torch.uint8).pin_memory()
+        dev_buf = torch.empty(tot, dtype=torch.uint8, device=dev)
+        saved = [(src, n, src[n]) for src, n in segs]
+        for (src, n), off in zip(segs, offs):
+            x = src[n]
+            nb = x.numel() * x.element_size()
+            host_buf[off:off + nb].view(x.dtype).view(x.shape).copy_(x.cpu())
+            src[n] = dev_buf[off:off + nb].view(x.dtype).view(x.shape)
         out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h2d = sum(x.numel() * x.element_size() for x in list(host.values()) +
-                  list(host_idx.values()))
+        h2d = tot
         d2h = out_h.numel() * out_h.element_size()
         ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
@@ -591,15 +605,13 @@ def measure(args, name, rank, world, local, with_e2e=True, with_cpu=True):
         for (a, b) in ev2:
             flush.fill_(1)
             a.record(stream)
-            for n in names:
-                t[n].copy_(host[n], non_blocking=True)
-            for n, x in host_idx.items():
-                idx[n].copy_(x, non_blocking=True)
-            mid = torch.cuda.Event(enable_timing=True)
+            dev_buf.copy_(host_buf, non_blocking=True)
             step()
             out_h.copy_(out, non_blocking=True)
             b.record(stream)
         torch.cuda.synchronize()
+        for src, n, x in saved:  # the device tensors of the timed steps again
+            src[n] = x
         barrier(world)
         e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2) / 1e3, world, dev)
         e2e_val = (T * args.steps * world / e2e_s if name in ("mixed", "mixed_prefill")
