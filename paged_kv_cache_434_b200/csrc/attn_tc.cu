@@ -374,8 +374,10 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         mbar_arrive(&meta->item_empty[slot]);
         if (info.end) break;
         const bool hasB = info.ntok > Tq;
-        if (!mbar_wait_bounded(&meta->q_full, n & 1, kWaitLimitNs) || !wait_k(tile_base) ||
-            (n >= 1 && !mbar_wait_bounded(&meta->o_empty, (n - 1) & 1, kWaitLimitNs))) {
+        // (the first QK^T only writes S: it runs while the softmax warps still
+        // store the previous item's O; the first PV, which overwrites O,
+        // waits for them below)
+        if (!mbar_wait_bounded(&meta->q_full, n & 1, kWaitLimitNs) || !wait_k(tile_base)) {
           ok = false;
           break;
         }
@@ -386,6 +388,13 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
         for (int j = 0; j < info.n_kv && ok; ++j) {
           const int t = tile_base + j;
           const bool more = j + 1 < info.n_kv;
+          if (j == 0 && n >= 1) {
+            if (!mbar_wait_bounded(&meta->o_empty, (n - 1) & 1, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
           if (!mbar_wait_bounded(&meta->v_full[t & 1], (t >> 1) & 1, kWaitLimitNs) ||
               !pv(0, t, j == 0)) {
             ok = false;
