@@ -177,6 +177,14 @@ __global__ void __launch_bounds__(tck::kThreads, 1)
     regs_dec<104>();
     if (lane == 0) {
       for (int n = 0;; ++n) {
+        // claim item n only once every role has taken item n - 1 (at most one
+        // item ahead of the work): items are handed out longest first, and a
+        // CTA that held two claimed items at the end would stretch the tail
+        if (n >= 1 && !mbar_wait_bounded(&meta->item_empty[(n - 1) & 1], ((n - 1) >> 1) & 1,
+                                         kWaitLimitNs)) {
+          if (g.err_word) atomicOr(g.err_word, PA_ERRBIT_TIMEOUT);
+          break;
+        }
         const int it = atomicAdd(&ws.ctrl[3], 1);
         Item info{};
         info.end = it >= n_tiles;
