@@ -212,6 +212,17 @@ def test_determinism(cuda_device):
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("lens", [[1200, 40], [4000, 9], [1200, 4000, 17]])
+def test_merge_paths_by_partition_count(cuda_device, lens):
+    """Rows split into 33 to 64 partitions reach the per-warp merge's second
+    chunk of partitions; rows with more reach the per-CTA merge.  (In these
+    small batches the planner cuts a 1200-key row into 38 pieces and a
+    4000-key row into 125: two-stage pieces over most of the row, then
+    smaller ones.)"""
+    w = W.custom("merge_paths", lens, [1] * len(lens), 32, 8, 128, 16, "bf16", seed=31)
+    _check_all(w, cuda_device)
+
+
 # ---------------------------------------------------------------- device errors
 
 def test_error_bits_bad_inputs(cuda_device):
