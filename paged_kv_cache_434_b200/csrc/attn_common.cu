@@ -809,7 +809,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
     const int np = (units + P - 1) / P;
     ws.nparts[r] = np + (info.w > 0 ? prefix_chunks : 0);  // the last ones: shared-prefix chunks
     // rows to merge: those a warp merges from the front of the list, those
-    // with more than 32 partitions (a CTA each) from the back
+    // with more than kMergeWarpParts partitions (a CTA each) from the back
     if (ws.nparts[r] > kMergeWarpParts)
       ws.merge_rows[g.num_qrows - 1 - atomicAdd(&s_merge_big, 1)] = r;
     else if (ws.nparts[r] != 1)

@@ -24,7 +24,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 //                         [6] shared-prefix tokens (decode cascade, 0: none),
 //                         [7] key chunks the shared prefix is split into,
 //                         [8] CTAs of the tensor-core tile kernel that work,
-//                         [9] rows to merge with more than 32 partitions
+//                         [9] rows to merge with more than kMergeWarpParts partitions
 //                         (listed from the back of merge_rows)
 //   qrow_info int4[R]     {request b, key_len, valid, key_start}: the row's
 //                         partitions cover keys [key_start, key_len); keys
@@ -33,7 +33,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded device waits: 2 s
 //                         -1: invalid -> row left unwritten)
 //   qrow_bad  int32[R]    set when a block id outside the pool was met
 //   merge_rows int32[R]   rows the merge pass must write (0 or >1 partitions):
-//                         up to 32 partitions from the front, more from the back
+//                         up to kMergeWarpParts partitions from the front, more from the back
 //   items     int4[I]     {qrow, head group | partition << 16, stages, first
 //                         stage}: keys [key_start + 16 first, + 16 stages) of
 //                         the row, clipped to its length
