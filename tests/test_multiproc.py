@@ -22,6 +22,9 @@ def _free_port():
 
 
 def _rank_main(rank, world, port, out):
+    # host-side plumbing only: no rank may pick a GPU (on a one-GPU machine the
+    # second rank's device would not exist), so gloo is what runs
+    os.environ["CUDA_VISIBLE_DEVICES"] = ""
     sys.path.insert(0, ROOT)
     os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
                        "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
