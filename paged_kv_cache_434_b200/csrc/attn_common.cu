@@ -294,33 +294,34 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
       const int max_cols = min((s_minlen - 1) / g.block_size, g.max_blocks);
       if (tid == 0) s_first = max_cols;
       __syncthreads();
-      constexpr int kPairs = 16;  // pairs per thread and chunk
+      constexpr int kPairs = 8;  // pairs per thread and pass
       // a chunk's pairs are laid out as B rows x 2^lw columns (the chunk's width
       // rounded up to a power of two), so that a pair's request and column are
       // a shift and a mask of its index
-      int W = max(1, kPairs * kPlanThreads / B);  // columns per chunk
+      int W = max(1, 2 * kPairs * kPlanThreads / B);  // columns per chunk (two passes)
       for (int cb = 1; cb < max_cols; cb += W, W = min(W * 4, 1 << 24)) {
         const int ce = min(cb + W, max_cols);
         const int lw = 32 - __clz(max(ce - cb - 1, 0));  // 2^lw >= ce - cb
         const int64_t slots = static_cast<int64_t>(B) << lw;
         int mine = 0x7fffffff;
         for (int64_t i0 = 0; i0 < slots; i0 += kPairs * kPlanThreads) {
+          // every load is issued unconditionally (addresses clamped into the
+          // table, pairs outside the chunk masked afterwards), so that all of
+          // a thread's loads are in flight at once
           int v[kPairs], ref[kPairs];
 #pragma unroll
           for (int k = 0; k < kPairs; ++k) {
             const int64_t idx = i0 + tid + static_cast<int64_t>(k) * kPlanThreads;
-            const int j = cb + static_cast<int>(idx & ((1 << lw) - 1));
-            const int64_t b = idx >> lw;
-            v[k] = ref[k] = 0;
-            if (b < B && j < ce) {
-              v[k] = g.block_tables[b * g.max_blocks + j];
-              ref[k] = g.block_tables[j];
-            }
+            const int j = min(cb + static_cast<int>(idx & ((1 << lw) - 1)), ce - 1);
+            const int64_t b = min(idx >> lw, static_cast<int64_t>(B - 1));
+            v[k] = __ldg(g.block_tables + b * g.max_blocks + j);
+            ref[k] = __ldg(g.block_tables + j);
           }
 #pragma unroll
           for (int k = 0; k < kPairs; ++k) {
             const int64_t idx = i0 + tid + static_cast<int64_t>(k) * kPlanThreads;
-            if (v[k] != ref[k]) mine = min(mine, cb + static_cast<int>(idx & ((1 << lw) - 1)));
+            const int j = cb + static_cast<int>(idx & ((1 << lw) - 1));
+            if ((idx >> lw) < B && j < ce && v[k] != ref[k]) mine = min(mine, j);
           }
         }
         mine = __reduce_min_sync(0xffffffffu, mine);
