@@ -377,21 +377,22 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
       mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
     if (lane == 0) {
-      // the sizes are heuristics: float arithmetic (no 64-bit division)
-      const double work = static_cast<double>(total) * a.head_groups;
-      const double by_target = ceil(work / max(a.target_items, 1));
+      // the sizes are heuristics: single precision with fast divisions (no
+      // double or 64-bit division routines in this once-per-call, cold code)
+      const float work = static_cast<float>(total) * static_cast<float>(a.head_groups);
+      const float by_target = ceilf(__fdividef(work, static_cast<float>(max(a.target_items, 1))));
       const int by_cap = (mx + cap - 1) / cap;
-      const double P = fmax(static_cast<double>(a.min_part_stages), fmax(by_target, by_cap));
-      *s_P = static_cast<int>(fmin(fmax(P, 1.0), 1e9));
+      const float P = fmaxf(static_cast<float>(a.min_part_stages),
+                            fmaxf(by_target, static_cast<float>(by_cap)));
+      *s_P = static_cast<int>(fminf(fmaxf(P, 1.f), 1e9f));
       // big pieces: 80 % of the work, about two per SM; small pieces: the
       // rest, about four per SM
-      const double C = max(a.num_sms, 1);
-      s_Pb = static_cast<int>(fmin(fmax(0.4 * work / C, static_cast<double>(a.min_part_stages)),
-                                   1e9));
+      const float per_sm = __fdividef(work, static_cast<float>(max(a.num_sms, 1)));
+      s_Pb = static_cast<int>(fminf(fmaxf(0.4f * per_sm, static_cast<float>(a.min_part_stages)), 1e9f));
       // (at least kMinSmallStages: smaller pieces cost more in the merge than
       // they gain at the end)
-      s_Ps = static_cast<int>(fmin(fmax(0.05 * work / C, static_cast<double>(kMinSmallStages)),
-                                   static_cast<double>(s_Pb)));
+      s_Ps = static_cast<int>(fminf(fmaxf(0.05f * per_sm, static_cast<float>(kMinSmallStages)),
+                                    static_cast<float>(s_Pb)));
       *s_merge = 0;
       *s_merge_big = 0;
     }
@@ -416,9 +417,14 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
     my_big += nb[k] * a.head_groups;
     my_small += ns[k] * a.head_groups;
   }
-  int n_big = 0, n_small = 0;
-  const int big0 = block_exclusive_scan<int>(my_big, s_scan, &n_big);
-  const int small0 = block_exclusive_scan<int>(my_small, s_scan, &n_small);
+  // both offsets from one scan: big counts in the high 32 bits, small in the low
+  __shared__ unsigned long long s_scan64[33];
+  unsigned long long both = 0;
+  const unsigned long long pre = block_exclusive_scan<unsigned long long>(
+      (static_cast<unsigned long long>(my_big) << 32) | static_cast<unsigned long long>(my_small),
+      s_scan64, &both);
+  const int n_big = static_cast<int>(both >> 32), n_small = static_cast<int>(both & 0xffffffffull);
+  const int big0 = static_cast<int>(pre >> 32), small0 = static_cast<int>(pre & 0xffffffffull);
   // big items, spread over the CTA by binary search over the rows' first items
   {
     int pos = big0;
