@@ -222,7 +222,9 @@ constexpr int kMinSmallStages = 4;
 struct RowPieces {
   int pb, nb, ps, ns;
 };
-__device__ __forceinline__ RowPieces row_pieces(int n, int Pb, int Ps, int cap) {
+// (one out-of-line copy: the planner runs it cold once per call, and six inlined
+// copies cost more instruction fetches than the calls)
+__device__ __noinline__ RowPieces row_pieces(int n, int Pb, int Ps, int cap) {
   RowPieces p;
   if (cap < 2) {  // one piece per row
     p.pb = max(n, 1), p.nb = n > 0 ? 1 : 0, p.ps = 1, p.ns = 0;
