@@ -247,7 +247,7 @@ __device__ __noinline__ RowPieces row_pieces(int n, int Pb, int Ps, int cap) {
 
 __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsView& ws,
                                  int* s_rowpos, int* s_scan,
-                                 long long* s_sum, int* s_max, int* s_P, int* s_merge,
+                                 int* s_max, int* s_P, int* s_merge,
                                  int* s_merge_big) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int B = g.num_seqs;
@@ -337,8 +337,9 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
   }
   const int prefix = prefix_blocks * g.block_size;
 
-  // invalid requests: error bits, rows left unwritten (L = -1 from here on)
-  long long units_sum = 0;
+  // invalid requests: error bits, rows left unwritten (L = -1 from here on);
+  // the stage total only sizes the pieces, so it is summed in float
+  float units_sum = 0.f;
   int units_max = 0;
 #pragma unroll
   for (int k = 0; k < kFastPerThread; ++k) {
@@ -352,16 +353,15 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
       continue;
     }
     const int units = (L[k] - prefix + kStageTokens - 1) / kStageTokens;
-    units_sum += units;
+    units_sum += static_cast<float>(units);
     units_max = max(units_max, units);
   }
 #pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    units_sum += __shfl_xor_sync(0xffffffffu, units_sum, o);
-    units_max = max(units_max, __shfl_xor_sync(0xffffffffu, units_max, o));
-  }
+  for (int o = 16; o; o >>= 1) units_sum += __shfl_xor_sync(0xffffffffu, units_sum, o);
+  units_max = __reduce_max_sync(0xffffffffu, units_max);
+  __shared__ float s_fsum[32];
   if (lane == 0) {
-    s_sum[warp] = units_sum;
+    s_fsum[warp] = units_sum;
     s_max[warp] = units_max;
   }
   __shared__ int s_Pb, s_Ps;
@@ -371,17 +371,14 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
   const int cap = static_cast<int>(
       max(1LL, static_cast<long long>(ws.max_parts) - (prefix > 0 ? kMaxPrefixChunks : 0)));
   if (warp == 0) {
-    long long total = s_sum[lane];
-    int mx = s_max[lane];
+    float total = s_fsum[lane];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      total += __shfl_xor_sync(0xffffffffu, total, o);
-      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
+    for (int o = 16; o; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+    const int mx = __reduce_max_sync(0xffffffffu, s_max[lane]);
     if (lane == 0) {
       // the sizes are heuristics: single precision with fast divisions (no
       // double or 64-bit division routines in this once-per-call, cold code)
-      const float work = static_cast<float>(total) * static_cast<float>(a.head_groups);
+      const float work = total * static_cast<float>(a.head_groups);
       const float by_target = ceilf(__fdividef(work, static_cast<float>(max(a.target_items, 1))));
       const int by_cap = (mx + cap - 1) / cap;
       const float P = fmaxf(static_cast<float>(a.min_part_stages),
@@ -551,7 +548,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
 
   if (decode_mode && g.num_seqs <= kFastRows && g.num_qrows == g.num_seqs) {
     __shared__ int s_scan33[33];
-    plan_decode_fast(g, a, ws, s_rowpos, s_scan33, s_sum, s_max, &s_P,
+    plan_decode_fast(g, a, ws, s_rowpos, s_scan33, s_max, &s_P,
                      &s_merge, &s_merge_big);
     return;
   }
