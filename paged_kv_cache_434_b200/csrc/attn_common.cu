@@ -285,14 +285,15 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
   // The run is limited so that each request keeps at least one key of its own.
   __shared__ int s_first, s_minlen;
   int prefix_blocks = 0;
-  if (look_shared) {
-    const int w_min = __reduce_min_sync(0xffffffffu, all_ok ? min_len : 0);
+  // (the shortest row is looked up only when every table starts with row 0's
+  // first block: most batches leave after one barrier)
+  if (look_shared && __syncthreads_and(same && all_ok)) {
+    const int w_min = __reduce_min_sync(0xffffffffu, min_len);
     if (tid == 0) s_minlen = 0x7fffffff;
     __syncthreads();
     if (lane == 0) atomicMin(&s_minlen, w_min);
-    const bool cand = __syncthreads_and(same && all_ok) && s_minlen > kCascadeMinPrefix &&
-                      s_minlen != 0x7fffffff;
-    if (cand) {
+    __syncthreads();
+    if (s_minlen > kCascadeMinPrefix && s_minlen != 0x7fffffff) {
       const int max_cols = min((s_minlen - 1) / g.block_size, g.max_blocks);
       if (tid == 0) s_first = max_cols;
       __syncthreads();
