@@ -212,7 +212,7 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T* s_scan, T* total) {
 //     search over the rows' first items in shared memory.
 constexpr int kFastPerThread = 4;
 constexpr int kFastRows = kPlanThreads * kFastPerThread;
-constexpr int kMinSmallStages = 4;
+constexpr int kMinSmallStages = 8;
 
 // The pieces of a row of n stages: nb big ones of pb stages (whole pieces
 // within 80 % of the row), then ns small ones of ps.  A row that would need
@@ -389,8 +389,8 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
       // rest, about four per SM
       const float per_sm = __fdividef(work, static_cast<float>(max(a.num_sms, 1)));
       s_Pb = static_cast<int>(fminf(fmaxf(0.4f * per_sm, static_cast<float>(a.min_part_stages)), 1e9f));
-      // (at least kMinSmallStages: smaller pieces cost more in the merge than
-      // they gain at the end)
+      // (at least kMinSmallStages: smaller pieces cost more, in the merge and
+      // in each item's start, than they gain at the end)
       s_Ps = static_cast<int>(fminf(fmaxf(0.05f * per_sm, static_cast<float>(kMinSmallStages)),
                                     static_cast<float>(s_Pb)));
       *s_merge = 0;
