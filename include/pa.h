@@ -8,6 +8,8 @@
  *                     worked example: block_size 16, table [5,8,12], pos 25 -> 137)
  *   pa_cache_write    reshape_and_cache: scatter each new token's K/V row to
  *                     its slot ("Reshape & Cache"; "Paged Attention")
+ *   pa_slot_mapping_cache_write
+ *                     the two above in one launch
  *   pa_decode         GQA decode attention over the paged cache, FlashAttention
  *                     online softmax, split-KV partitions merged by log-sum-exp
  *                     ("Attention (FlashAttention, Scaled Dot-Product Attention)";
@@ -146,6 +148,30 @@ pa_status pa_slot_mapping(const int32_t* block_tables, int32_t max_blocks_per_se
 pa_status pa_cache_write(const void* k, const void* v, void* key_cache, void* value_cache,
                          const int64_t* slot_mapping, int64_t num_tokens,
                          const pa_cache_desc* cache, int32_t* err_word, void* stream);
+
+/*
+ * pa_slot_mapping_cache_write -- pa_slot_mapping and pa_cache_write in one
+ * launch (the walkthrough's two steps before attention: the slot of each new
+ * token, then reshape_and_cache into it).  The same results as the two calls:
+ * the slots (written to slot_mapping when it is not NULL), the pools, and the
+ * error bits of both (a token whose request fails the slot checks, or whose
+ * table entry is outside the pool, gets slot -1 and is not written).
+ *   k, v, key_cache, value_cache, cache: as for pa_cache_write
+ *   block_tables, max_blocks_per_seq, seq_lens, num_seqs: as for pa_slot_mapping
+ *   query_start_loc int32 [num_seqs + 1] as for pa_slot_mapping, or NULL for a
+ *                   decode step: one new token per request, token b of
+ *                   request b (num_tokens must then equal num_seqs)
+ *   slot_mapping    int64 [num_tokens] (output), may be NULL
+ * Returns PA_ERR_INVALID_ARG for NULL or misaligned buffers, negative sizes or
+ * a NULL query_start_loc with num_tokens != num_seqs; PA_ERR_UNSUPPORTED when
+ * max_blocks_per_seq * block_size exceeds 2^30.
+ */
+pa_status pa_slot_mapping_cache_write(const void* k, const void* v, void* key_cache,
+                                      void* value_cache, const int32_t* block_tables,
+                                      int32_t max_blocks_per_seq, const int32_t* query_start_loc,
+                                      const int32_t* seq_lens, int32_t num_seqs,
+                                      int64_t num_tokens, const pa_cache_desc* cache,
+                                      int64_t* slot_mapping, int32_t* err_word, void* stream);
 
 /*
  * pa_copy_blocks -- copy-on-write block copies ("第三部分 · 推理系统与基础设施",

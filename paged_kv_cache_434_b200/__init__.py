@@ -39,6 +39,7 @@ from .binding import (  # noqa: F401
     rope_cache_write,
     rope_cos_sin_cache,
     slot_mapping,
+    slot_mapping_cache_write,
     slot_mapping_positions,
     version,
 )

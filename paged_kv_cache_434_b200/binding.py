@@ -32,7 +32,8 @@ EXPORTS = ("pa_status_str", "pa_version", "pa_slot_mapping", "pa_cache_write",
            "pa_decode_workspace_size", "pa_decode", "pa_mixed_step_workspace_size",
            "pa_mixed_step", "pa_read_error", "pa_decode_no_alloc", "pa_kernel_timing_enable",
            "pa_kernel_timing_read", "pa_rope_cos_sin_cache", "pa_rope_cache_write",
-           "pa_copy_blocks", "pa_slot_mapping_positions", "pa_selftest_wait_timeout")
+           "pa_copy_blocks", "pa_slot_mapping_positions", "pa_selftest_wait_timeout",
+           "pa_slot_mapping_cache_write")
 
 
 class PagedAttentionError(RuntimeError):
@@ -59,6 +60,8 @@ _SIGNATURES = {
     "pa_version": ([], ctypes.c_int),
     "pa_slot_mapping": ([_vp, _i32, _vp, _vp, _i32, _i64, _i32, _i64, _vp, _vp, _vp], ctypes.c_int),
     "pa_cache_write": ([_vp, _vp, _vp, _vp, _vp, _i64, _desc_p, _vp, _vp], ctypes.c_int),
+    "pa_slot_mapping_cache_write": ([_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i64, _desc_p,
+                                     _vp, _vp, _vp], ctypes.c_int),
     "pa_decode_workspace_size": ([_i32, _i32, _i32, _desc_p], _sz),
     "pa_decode": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i32, _i32, _i32, _desc_p, _vp, _sz,
                    _vp, _vp], ctypes.c_int),
@@ -250,6 +253,39 @@ def cache_write(k, v, k_cache, v_cache, slot_mapping, err=None, kv_scales=None):
         _cuda(k, "k"), _cuda(v, "v"), _cuda(k_cache, "k_cache", ndim=4),
         _cuda(v_cache, "v_cache", ndim=4), _cuda(slot_mapping, "slot_mapping", torch.int64, 1),
         T, ctypes.byref(desc), _err_ptr(err), _stream()), "pa_cache_write")
+
+
+def slot_mapping_cache_write(k, v, k_cache, v_cache, block_tables, query_start_loc, seq_lens,
+                             slots=None, err=None, kv_scales=None):
+    """slot_mapping then cache_write in one launch (see pa_slot_mapping_cache_write).
+    query_start_loc None: a decode step, one new token per request.  Returns
+    the slots (allocated unless `slots` is given)."""
+    desc = cache_desc(k_cache, kv_scales)
+    T = k.shape[0]
+    B, W = block_tables.shape
+    for name, t in (("k", k), ("v", v)):
+        if t.dim() != 3 or tuple(t.shape[1:]) != (desc.num_kv_heads, desc.head_dim) or \
+                t.shape[0] != T or t.dtype != io_dtype(k_cache):
+            raise ValueError(f"{name} must be [num_tokens, num_kv_heads, head_dim] of the cache's "
+                             f"input dtype")
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype:
+        raise ValueError("v_cache must match k_cache")
+    _entries(seq_lens, "seq_lens", B)
+    if query_start_loc is not None:
+        _entries(query_start_loc, "query_start_loc", B + 1)
+    elif T != B:
+        raise ValueError("without query_start_loc every request has exactly one new token")
+    if slots is None:
+        slots = torch.empty(T, dtype=torch.int64, device=k.device)
+    _entries(slots, "slot_mapping", T)
+    _check(_lib().pa_slot_mapping_cache_write(
+        _cuda(k, "k"), _cuda(v, "v"), _cuda(k_cache, "k_cache", ndim=4),
+        _cuda(v_cache, "v_cache", ndim=4), _cuda(block_tables, "block_tables", torch.int32, 2), W,
+        None if query_start_loc is None else _cuda(query_start_loc, "query_start_loc", torch.int32, 1),
+        _cuda(seq_lens, "seq_lens", torch.int32, 1), B, T, ctypes.byref(desc),
+        _cuda(slots, "slot_mapping", torch.int64, 1), _err_ptr(err), _stream()),
+        "pa_slot_mapping_cache_write")
+    return slots
 
 
 def copy_blocks(k_cache, v_cache, block_mapping, err=None):

@@ -183,6 +183,13 @@ cudaError_t launch_slot_positions(const int32_t* block_tables, int32_t max_block
                                   const int64_t* positions, int64_t num_tokens,
                                   int32_t block_size, int64_t num_blocks, int64_t* slots,
                                   int32_t* err, int num_sms, cudaStream_t s);
+cudaError_t launch_slot_cache_write(const void* k, const void* v, void* kc, void* vc,
+                                    const int32_t* block_tables, int32_t max_blocks,
+                                    const int32_t* qsl, const int32_t* seq_lens, int32_t num_seqs,
+                                    int64_t num_tokens, int32_t block_size, int64_t num_blocks,
+                                    int64_t row_elems, int32_t elt_bytes, bool fp8,
+                                    float k_scale, float v_scale, int64_t* slots, int32_t* err,
+                                    cudaStream_t s);
 cudaError_t launch_cache_write_fp8(const void* k, const void* v, void* kc, void* vc,
                                    const int64_t* slots, int64_t num_tokens, int64_t row_elems,
                                    int64_t num_slots, float k_scale, float v_scale, int32_t* err,

@@ -317,6 +317,33 @@ pa_status pa_cache_write(const void* k, const void* v, void* key_cache, void* va
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+pa_status pa_slot_mapping_cache_write(const void* k, const void* v, void* key_cache,
+                                      void* value_cache, const int32_t* block_tables,
+                                      int32_t max_blocks_per_seq, const int32_t* query_start_loc,
+                                      const int32_t* seq_lens, int32_t num_seqs,
+                                      int64_t num_tokens, const pa_cache_desc* cache,
+                                      int64_t* slot_mapping, int32_t* err_word, void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_seqs < 0 || num_tokens < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARG;
+  if (!query_start_loc && num_tokens != num_seqs) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+  if (!k || !v || !key_cache || !value_cache || !block_tables || !seq_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_blocks_per_seq) * cache->block_size > (1LL << 30))
+    return PA_ERR_UNSUPPORTED;
+  const int64_t row_elems = static_cast<int64_t>(cache->num_kv_heads) * cache->head_dim;
+  const bool fp8 = cache->dtype == PA_FP8_E4M3;
+  cudaError_t e = launch_slot_cache_write(
+      k, v, key_cache, value_cache, block_tables, max_blocks_per_seq, query_start_loc, seq_lens,
+      num_seqs, num_tokens, cache->block_size, cache->num_blocks, row_elems,
+      fp8 ? 1 : elt_bytes(cache->dtype), fp8, cache->k_scale, cache->v_scale, slot_mapping,
+      err_word, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t max_blocks_per_seq,
                                 const pa_cache_desc* cache) {
   if (check_attn_args(num_seqs, num_seqs, num_heads, max_blocks_per_seq, PA_F32, cache) != PA_OK)
