@@ -703,9 +703,10 @@ def _in_step_tiles(line):
 def run_ours(args, rank, world, local):
     line = measure(args, args.workload, rank, world, local)
     if args.workload == "llama8b_decode" and not args.no_extras:
-        # The other half of the metric (a mixed continuous-batching step) and the
-        # shared-prefix decode batch, measured in the same process after the
-        # headline, each with its own timed region, clocks and launch count.
+        # The other half of the metric (a mixed continuous-batching step), the
+        # shared-prefix decode batch and the long-context split-KV batch,
+        # measured in the same process after the headline, each with its own
+        # timed region, clocks and launch count.
         torch.cuda.empty_cache()
         m = measure(args, "mixed", rank, world, local, with_cpu=False)
         line["mixed_step"] = {
@@ -729,6 +730,14 @@ def run_ours(args, rank, world, local):
             note="per attention call, on unique bytes: each physical block once (the shared "
                  "prefix once), Q read and fp32 O written, against the HBM copy peak")
         line["shared_prefix"]["suffix_partitions"] = sp["roofline"]
+        torch.cuda.empty_cache()
+        lc = measure(args, "long_context", rank, world, local, with_cpu=False)
+        line["long_context"] = {
+            k: lc[k] for k in ("metric", "value", "unit", "ms_per_step", "e2e", "kernel_ms",
+                               "gpu_launches", "clocks", "roofline")}
+        line["long_context"]["config"] = {k: lc["config"][k] for k in (
+            "workload", "num_seqs", "num_heads", "num_kv_heads", "block_size",
+            "kv_bytes_unique")}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
