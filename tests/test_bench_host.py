@@ -1,4 +1,4 @@
-"""The benchmark's algorithmic counts (host arithmetic, no GPU): prefill
+"""The benchmark's host side (no GPU): the algorithmic counts -- prefill
 FLOPs, unique K/V bytes with shared blocks counted once, the decode-launch
 bytes, the fused RoPE + cache write bytes, checked against direct sums over
 the workloads' definitions."""
@@ -68,3 +68,35 @@ def test_own_peaks_never_costs_the_benchmark_line(monkeypatch):
     monkeypatch.setattr(torch.cuda, "Event", no_events)
     r = bench.own_peaks(torch.device("cpu"), copy_bytes=1 << 20, gemm_n=64, iters=1)
     assert set(r) == {"error"} and r["error"]
+
+
+def test_default_line_carries_every_decode_config(monkeypatch, capsys):
+    """The default run's one JSON line: the Llama-3-8B decode headline plus the
+    mixed step (the metric's second half), the shared-prefix and the
+    long-context batches, each measured in the same process (measure() is
+    stubbed here: only the line's assembly is checked)."""
+    import json
+    import types
+
+    def fake_measure(args, name, rank, world, local, with_e2e=True, with_cpu=True):
+        roof = {"bound": "hbm", "frac": 1.0, "attention_call": {"ms": 1.0, "frac": 0.9}}
+        return {"metric": name, "value": 1.0, "unit": "u", "ms_per_step": 1.0, "e2e": {},
+                "kernel_ms": {"tiles": 0.5}, "gpu_launches": 4, "clocks": {},
+                "roofline": roof, "without_cache_write": {"value": 1.0},
+                "prefill_roofline": {"frac": 0.5},
+                "config": {"workload": name, "num_seqs": 1, "num_tokens": 1,
+                           "prefill_flops_per_step": 1e9, "num_heads": 1, "num_kv_heads": 1,
+                           "block_size": 16, "kv_bytes_unique": 1}}
+
+    monkeypatch.setattr(bench, "measure", fake_measure)
+    monkeypatch.setattr(bench.torch.cuda, "empty_cache", lambda: None)
+    args = types.SimpleNamespace(workload="llama8b_decode", no_extras=False)
+    bench.run_ours(args, 0, 1, 0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["metric"] == "llama8b_decode"
+    for key, name in (("mixed_step", "mixed"), ("shared_prefix", "shared_prefix"),
+                      ("long_context", "long_context")):
+        assert line[key]["metric"] == name and line[key]["config"]["workload"] == name
+    assert line["mixed_step"]["prefill_roofline"]["alone"] == {"frac": 0.5}
+    assert line["shared_prefix"]["attention_call"]["frac"] == 0.9
+    assert line["long_context"]["roofline"]["attention_call"]["frac"] == 0.9
