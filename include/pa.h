@@ -14,6 +14,9 @@
  *                     online softmax, split-KV partitions merged by log-sum-exp
  *                     ("Attention (FlashAttention, Scaled Dot-Product Attention)";
  *                     "总结": Flash-Decoding re-normalises with log-sum-exp)
+ *   pa_decode_step    a decode step's cache write and attention in one call:
+ *                     pa_slot_mapping_cache_write (one new token per request)
+ *                     then pa_decode, the write done in the planner's launch
  *   pa_mixed_step     causal varlen attention of a flattened continuous-batching
  *                     step mixing chunked-prefill tokens and decode tokens, every
  *                     K/V read through the block table (same section: the v1
@@ -286,6 +289,37 @@ pa_status pa_decode(const void* q, const void* key_cache, const void* value_cach
                     void* out, int32_t num_seqs, int32_t num_heads, int32_t max_blocks_per_seq,
                     int32_t out_dtype, const pa_cache_desc* cache, void* workspace,
                     size_t workspace_bytes, int32_t* err_word, void* stream);
+
+/*
+ * pa_decode_step -- one decode step of one layer: each request's new K/V row
+ * goes to its slot, then its query attends to all seq_lens[b] keys
+ * ("AI Infra入门干货总结：大模型是如何高效推理的", sections "Reshape & Cache",
+ * "Paged Attention" and "Attention (FlashAttention, Scaled Dot-Product
+ * Attention)": the step writes the token's K/V into the paged cache before
+ * the attention reads it).
+ * Results, error bits and the rows left unwritten are exactly those of
+ *     pa_slot_mapping_cache_write(k, v, key_cache, value_cache, block_tables,
+ *         max_blocks_per_seq, NULL, seq_lens, num_seqs, num_seqs, cache,
+ *         slot_mapping, err_word, stream)
+ *     pa_decode(q, key_cache, value_cache, block_tables, seq_lens, scale, out,
+ *         ..., workspace, workspace_bytes, err_word, stream)
+ * made back to back; the write runs in the CTAs beside the work planner, in
+ * the same launch, so it costs no launch of its own.
+ *   k, v          [num_seqs, num_kv_heads, head_dim] new rows, token b of
+ *                 request b at position seq_lens[b] - 1 (bf16 for PA_FP8_E4M3)
+ *   slot_mapping  int64 [num_seqs] (output), may be NULL
+ *   workspace     >= pa_decode_workspace_size(num_seqs, num_heads,
+ *                 max_blocks_per_seq, cache) bytes, as for pa_decode
+ *   other arguments as for pa_decode.
+ * Returns what pa_decode returns for the same arguments, and PA_ERR_INVALID_ARG
+ * for a NULL or misaligned k or v.  Nothing is written on a non-zero status.
+ */
+pa_status pa_decode_step(const void* q, const void* k, const void* v, void* key_cache,
+                         void* value_cache, const int32_t* block_tables, const int32_t* seq_lens,
+                         float scale, void* out, int32_t num_seqs, int32_t num_heads,
+                         int32_t max_blocks_per_seq, int32_t out_dtype, const pa_cache_desc* cache,
+                         int64_t* slot_mapping, void* workspace, size_t workspace_bytes,
+                         int32_t* err_word, void* stream);
 
 /* Bytes of workspace pa_mixed_step needs; 0 on bad arguments and beyond
  * 2^46 bytes, as for pa_decode_workspace_size. */

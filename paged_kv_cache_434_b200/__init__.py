@@ -11,6 +11,7 @@ its Python binding plus a seeded workload generator:
   slot_mapping_positions  slots from explicit (request, position) pairs
   decode         GQA decode attention, online softmax, split-KV + LSE merge
   decode_no_alloc  decode through the library's own static scratch
+  decode_step    a decode step's cache write and attention in one call
   mixed_step     causal varlen attention of a chunked-prefill + decode step
   step           slot_mapping -> cache_write -> attention, the per-layer path
 """
@@ -28,6 +29,7 @@ from .binding import (  # noqa: F401
     copy_blocks,
     decode,
     decode_no_alloc,
+    decode_step,
     decode_workspace_size,
     kernel_times,
     kernel_timing,

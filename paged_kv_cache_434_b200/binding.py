@@ -33,7 +33,7 @@ EXPORTS = ("pa_status_str", "pa_version", "pa_slot_mapping", "pa_cache_write",
            "pa_mixed_step", "pa_read_error", "pa_decode_no_alloc", "pa_kernel_timing_enable",
            "pa_kernel_timing_read", "pa_rope_cos_sin_cache", "pa_rope_cache_write",
            "pa_copy_blocks", "pa_slot_mapping_positions", "pa_selftest_wait_timeout",
-           "pa_slot_mapping_cache_write")
+           "pa_slot_mapping_cache_write", "pa_decode_step")
 
 
 class PagedAttentionError(RuntimeError):
@@ -65,6 +65,8 @@ _SIGNATURES = {
     "pa_decode_workspace_size": ([_i32, _i32, _i32, _desc_p], _sz),
     "pa_decode": ([_vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i32, _i32, _i32, _desc_p, _vp, _sz,
                    _vp, _vp], ctypes.c_int),
+    "pa_decode_step": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i32, _i32, _i32,
+                        _desc_p, _vp, _vp, _sz, _vp, _vp], ctypes.c_int),
     "pa_mixed_step_workspace_size": ([_i32, _i64, _i32, _i32, _desc_p], _sz),
     "pa_mixed_step": ([_vp, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _i32, _i64, _i32, _i32, _i32,
                        _desc_p, _vp, _sz, _vp, _vp], ctypes.c_int),
@@ -430,6 +432,39 @@ def decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=None,
         _dt(out), ctypes.byref(desc), _cuda(ws, "workspace"), ws.numel() * ws.element_size(),
         _err_ptr(err), _stream()), "pa_decode")
     return out
+
+
+def decode_step(q, k, v, k_cache, v_cache, block_tables, seq_lens, scale: float, out=None,
+                out_dtype=torch.float32, slots=None, workspace=None, err=None, kv_scales=None):
+    """One decode step: the new K/V rows (token b of request b) go to their
+    slots, then decode attention -- slot_mapping_cache_write(..., None, ...)
+    followed by decode(...), the write done in the planner's launch.  Returns
+    (out, slots)."""
+    desc = _check_attn(q, k_cache, v_cache, block_tables, seq_lens, out_dtype, kv_scales,
+                       num_seqs=q.shape[0] if q.dim() == 3 else None)
+    B, H, D = q.shape
+    W = block_tables.shape[1]
+    for name, t in (("k", k), ("v", v)):
+        if t.dim() != 3 or tuple(t.shape) != (B, desc.num_kv_heads, desc.head_dim) or \
+                t.dtype != io_dtype(k_cache):
+            raise ValueError(f"{name} must be [num_seqs, num_kv_heads, head_dim] of the cache's "
+                             f"input dtype")
+    if out is None:
+        out = torch.empty(B, H, D, dtype=out_dtype, device=q.device)
+    _out_shape(out, (B, H, D))
+    if slots is None:
+        slots = torch.empty(B, dtype=torch.int64, device=q.device)
+    _entries(slots, "slot_mapping", B)
+    nbytes = decode_workspace_size(B, H, W, k_cache)
+    ws = _workspace(nbytes, q.device, workspace)
+    _check(_lib().pa_decode_step(
+        _cuda(q, "q"), _cuda(k, "k"), _cuda(v, "v"), _cuda(k_cache, "k_cache"),
+        _cuda(v_cache, "v_cache"), _cuda(block_tables, "block_tables", torch.int32, 2),
+        _cuda(seq_lens, "seq_lens", torch.int32, 1), float(scale), _cuda(out, "out"), B, H, W,
+        _dt(out), ctypes.byref(desc), _cuda(slots, "slot_mapping", torch.int64, 1),
+        _cuda(ws, "workspace"), ws.numel() * ws.element_size(), _err_ptr(err), _stream()),
+        "pa_decode_step")
+    return out, slots
 
 
 def mixed_step(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, scale: float,

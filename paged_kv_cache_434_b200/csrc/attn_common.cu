@@ -23,6 +23,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "slot_write.cuh"
 
 namespace pa {
 
@@ -529,9 +530,8 @@ __device__ void plan_decode_fast(const AttnGeom& g, const PlanArgs& a, const WsV
   }
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs a, WsView ws) {
-  grid_launch_dependents();
-  grid_dependency_wait();  // seq_lens / tables / the workspace may come from the previous launch
+// The planner: one CTA of kPlanThreads threads.
+__device__ __forceinline__ void plan_body(const AttnGeom& g, const PlanArgs& a, const WsView& ws) {
   __shared__ long long s_sum[32];
   __shared__ int s_max[32];
   __shared__ int s_scan[32];
@@ -904,8 +904,44 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs
   }
 }
 
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(AttnGeom g, PlanArgs a, WsView ws) {
+  grid_launch_dependents();
+  grid_dependency_wait();  // seq_lens / tables / the workspace may come from the previous launch
+  plan_body(g, a, ws);
+}
+
+// A decode step's first launch: CTA 0 plans the attention while the other
+// CTAs write the step's new K/V rows into the pools (one warp per token and
+// K|V).  Neither half reads what the other writes -- the planner reads the
+// lengths and tables, the write reads those and the new rows and writes slots
+// and pool rows -- and the attention launches after this one read both
+// results only after griddepcontrol.wait, i.e. after the whole grid.
+template <bool F8>
+__global__ void __launch_bounds__(kPlanThreads) write_plan_kernel(AttnGeom g, PlanArgs a,
+                                                                  WsView ws, SlotWrite sw) {
+  grid_launch_dependents();
+  grid_dependency_wait();  // every input and the workspace may come from the previous launch
+  if (blockIdx.x == 0) {
+    plan_body(g, a, ws);
+    return;
+  }
+  const int64_t w =
+      static_cast<int64_t>(blockIdx.x - 1) * (kPlanThreads / 32) + (threadIdx.x >> 5);
+  slot_write_warp<F8>(sw, w, threadIdx.x & 31);
+}
+
 cudaError_t launch_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws, cudaStream_t s) {
   return launch_pdl<plan_kernel>(dim3(1), dim3(kPlanThreads), 0, s, g, a, ws);
+}
+
+cudaError_t launch_write_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws,
+                              const SlotWrite& sw, bool fp8, cudaStream_t s) {
+  constexpr int64_t kWarps = kPlanThreads / 32;
+  const int64_t write_ctas = (2 * sw.num_tokens + kWarps - 1) / kWarps;
+  if (write_ctas + 1 > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(1 + write_ctas));
+  if (fp8) return launch_pdl<write_plan_kernel<true>>(grid, dim3(kPlanThreads), 0, s, g, a, ws, sw);
+  return launch_pdl<write_plan_kernel<false>>(grid, dim3(kPlanThreads), 0, s, g, a, ws, sw);
 }
 
 // ======================================================================= generic

@@ -202,6 +202,10 @@ cudaError_t launch_cache_write(const void* k, const void* v, void* kc, void* vc,
                                const int64_t* slots, int64_t num_tokens, int64_t row_bytes,
                                int64_t num_slots, int32_t* err, cudaStream_t s);
 cudaError_t launch_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws, cudaStream_t s);
+struct SlotWrite;
+// The planner on CTA 0 and the slot mapping + cache write of sw on the others.
+cudaError_t launch_write_plan(const AttnGeom& g, const PlanArgs& a, const WsView& ws,
+                              const SlotWrite& sw, bool fp8, cudaStream_t s);
 cudaError_t launch_attn_generic(const AttnGeom& g, const WsView& ws, int num_sms,
                                 cudaStream_t s);
 cudaError_t launch_attn_mma(const AttnGeom& g, const WsView& ws, int num_sms, int heads_per_group,

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "slot_write.cuh"
 
 namespace pa {
 
@@ -216,8 +217,11 @@ class TimedCall {
   bool active_ = false;
 };
 
+// sw != nullptr: the call also writes the step's new K/V rows (decode form),
+// in the planner's launch.
 static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* workspace,
-                               size_t ws_bytes, cudaStream_t s) {
+                               size_t ws_bytes, cudaStream_t s, const SlotWrite* sw = nullptr,
+                               bool fp8 = false) {
   const WsLayout L = ws_layout(p.num_qrows, g.num_heads, g.head_dim, p.head_groups, p.max_parts,
                                p.max_tiles);
   if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -235,7 +239,8 @@ static pa_status run_attention(const AttnGeom& g, const AttnPlan& p, void* works
   a.num_sms = p.num_sms;
   TimedCall tm(s);
   tm.begin(PA_TK_PLAN);
-  if (launch_plan(g, a, ws, s) != cudaSuccess) return PA_ERR_CUDA;
+  if ((sw ? launch_write_plan(g, a, ws, *sw, fp8, s) : launch_plan(g, a, ws, s)) != cudaSuccess)
+    return PA_ERR_CUDA;
   tm.end(PA_TK_PLAN);
   if (p.use_tc) {
     tm.begin(PA_TK_TILES);
@@ -374,6 +379,37 @@ pa_status pa_decode(const void* q, const void* key_cache, const void* value_cach
                                out, num_seqs, num_seqs, num_heads, max_blocks_per_seq, out_dtype,
                                cache, err_word);
   return run_attention(g, p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_decode_step(const void* q, const void* k, const void* v, void* key_cache,
+                         void* value_cache, const int32_t* block_tables, const int32_t* seq_lens,
+                         float scale, void* out, int32_t num_seqs, int32_t num_heads,
+                         int32_t max_blocks_per_seq, int32_t out_dtype, const pa_cache_desc* cache,
+                         int64_t* slot_mapping, void* workspace, size_t workspace_bytes,
+                         int32_t* err_word, void* stream) {
+  pa_status st =
+      check_attn_args(num_seqs, num_seqs, num_heads, max_blocks_per_seq, out_dtype, cache);
+  if (st != PA_OK) return st;
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !k || !v || !key_cache || !value_cache || !block_tables || !seq_lens || !out)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(key_cache) ||
+      !aligned16(value_cache) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  const AttnPlan p = make_plan(num_seqs, num_heads, max_blocks_per_seq, cache, true);
+  if (!p.size_ok) return PA_ERR_UNSUPPORTED;
+  const AttnGeom g = make_geom(q, key_cache, value_cache, block_tables, seq_lens, nullptr, scale,
+                               out, num_seqs, num_seqs, num_heads, max_blocks_per_seq, out_dtype,
+                               cache, err_word);
+  const bool fp8 = cache->dtype == PA_FP8_E4M3;
+  const SlotWrite sw = make_slot_write(
+      k, v, key_cache, value_cache, block_tables, max_blocks_per_seq, nullptr, seq_lens,
+      num_seqs, num_seqs, cache->block_size, cache->num_blocks,
+      static_cast<int64_t>(cache->num_kv_heads) * cache->head_dim,
+      fp8 ? 1 : elt_bytes(cache->dtype), fp8, cache->k_scale, cache->v_scale, slot_mapping,
+      err_word);
+  return run_attention(g, p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), &sw,
+                       fp8);
 }
 
 size_t pa_mixed_step_workspace_size(int32_t num_seqs, int64_t num_tokens, int32_t num_heads,

@@ -14,8 +14,9 @@ from . import binding
 def step(q, k_new, v_new, k_cache, v_cache, block_tables, query_start_loc, seq_lens,
          scale: float, *, decode_only: bool = False, out=None, out_dtype=torch.float32,
          slots=None, workspace=None, err=None, kv_scales=None):
-    """Run slot_mapping -> cache_write (one launch) -> decode / mixed_step on the
-    current stream.
+    """Run slot_mapping -> cache_write -> decode / mixed_step on the current
+    stream: a decode step in one call (the write rides in the planner's
+    launch), a mixed step as the fused slot/cache write then the attention.
 
     q: [T, Hq, D]; k_new, v_new: [T, Hkv, D]; query_start_loc: [B+1] int32;
     seq_lens: [B] int32 (lengths after this step).  float8_e4m3fn pools take
@@ -23,15 +24,13 @@ def step(q, k_new, v_new, k_cache, v_cache, block_tables, query_start_loc, seq_l
     request has exactly one new token (T == B) and pa_decode is used.
     Returns out [T, Hq, D].
     """
-    # slot mapping and the cache write in one launch (a decode step needs no
-    # query offsets: token b belongs to request b)
+    if decode_only:  # token b belongs to request b: no query offsets needed
+        return binding.decode_step(q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens,
+                                   scale, out=out, out_dtype=out_dtype, slots=slots,
+                                   workspace=workspace, err=err, kv_scales=kv_scales)[0]
     binding.slot_mapping_cache_write(k_new, v_new, k_cache, v_cache, block_tables,
-                                     None if decode_only else query_start_loc, seq_lens,
-                                     slots=slots, err=err, kv_scales=kv_scales)
-    if decode_only:
-        return binding.decode(q, k_cache, v_cache, block_tables, seq_lens, scale, out=out,
-                              out_dtype=out_dtype, workspace=workspace, err=err,
-                              kv_scales=kv_scales)
+                                     query_start_loc, seq_lens, slots=slots, err=err,
+                                     kv_scales=kv_scales)
     return binding.mixed_step(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, scale,
                               out=out, out_dtype=out_dtype, workspace=workspace, err=err,
                               kv_scales=kv_scales)

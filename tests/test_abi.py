@@ -107,6 +107,29 @@ def test_attention_validation(lib):
                          None, 0, None, None) == B.PA_OK
 
 
+def test_decode_step_validation(lib):
+    """pa_decode_step refuses what pa_decode refuses, and a NULL or misaligned
+    new K/V row buffer, before launching anything."""
+    from paged_kv_cache_434_b200 import binding as B
+    d = _desc()
+
+    def call(q=16, k=16, v=16, heads=8, out_dtype=0, ws=256, ws_bytes=1 << 20, num_seqs=2):
+        return lib.pa_decode_step(q, k, v, 16, 16, 16, 16, 0.1, 16, num_seqs, heads, 4, out_dtype,
+                                  ctypes.byref(d), None, ws, ws_bytes, None, None)
+
+    assert call(k=None) == B.PA_ERR_INVALID_ARG
+    assert call(v=None) == B.PA_ERR_INVALID_ARG
+    assert call(v=24) == B.PA_ERR_INVALID_ARG            # not 16-byte aligned
+    assert call(q=None) == B.PA_ERR_INVALID_ARG
+    assert call(heads=3) == B.PA_ERR_INVALID_ARG         # not a multiple of num_kv_heads
+    assert call(heads=64) == B.PA_ERR_UNSUPPORTED        # group above 16
+    assert call(out_dtype=5) == B.PA_ERR_UNSUPPORTED
+    assert call(ws_bytes=16) == B.PA_ERR_WORKSPACE
+    assert call(ws=None) == B.PA_ERR_WORKSPACE
+    assert call(ws=272) == B.PA_ERR_WORKSPACE            # not 256-byte aligned
+    assert call(q=None, k=None, v=None, num_seqs=0) == B.PA_OK
+
+
 def test_workspace_sizes_are_positive_and_monotone(lib):
     d = _desc(num_kv_heads=8, head_dim=128, dtype=1)
     a = lib.pa_decode_workspace_size(64, 32, 512, ctypes.byref(d))
