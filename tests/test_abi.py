@@ -249,6 +249,7 @@ def test_binding_refuses_arrays_the_library_would_overrun():
     from paged_kv_cache_434_b200 import binding as B
     kc = torch.zeros(4, 16, 2, 64)
     q = torch.zeros(2, 8, 64)
+    kv = torch.zeros(2, 2, 64)
     i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)  # noqa: E731
     cases = [
         (lambda: P.decode(q, kc, kc, i32(1, 3), i32(2), 0.1), "block_tables"),
@@ -260,6 +261,12 @@ def test_binding_refuses_arrays_the_library_would_overrun():
                               out=torch.zeros(1, 8, 64)), "out"),
         (lambda: B.decode_no_alloc(q, kc, kc, i32(2, 3), i32(2), 0.1, torch.zeros(3, 8, 64)),
          "out"),
+        (lambda: P.decode_step(q, kv, kv, kc, kc, i32(1, 3), i32(2), 0.1), "block_tables"),
+        (lambda: P.decode_step(q, kv, kv, kc, kc, i32(2, 3), i32(1), 0.1), "seq_lens"),
+        (lambda: P.decode_step(q, kv, kv, kc, kc, i32(2, 3), i32(2), 0.1,
+                               out=torch.zeros(2, 8, 32)), "out"),
+        (lambda: P.decode_step(q, kv, kv, kc, kc, i32(2, 3), i32(2), 0.1,
+                               slots=torch.zeros(1, dtype=torch.int64)), "slot_mapping"),
         (lambda: P.slot_mapping(i32(2, 3), i32(2), i32(2), 16, 4, 5), "query_start_loc"),
         (lambda: P.slot_mapping(i32(2, 3), i32(3), i32(1), 16, 4, 5), "seq_lens"),
         (lambda: P.slot_mapping(i32(2, 3), i32(3), i32(2), 16, 4, 5,
@@ -279,6 +286,11 @@ def test_binding_refuses_arrays_the_library_would_overrun():
         with pytest.raises(ValueError, match=rf"^{name} must (be a \d-D tensor with at least|"
                                              rf"have shape)"):
             call()
+    # a decode step's new rows: one per request, of the cache's input dtype
+    for k in (torch.zeros(3, 2, 64), torch.zeros(2, 1, 64),
+              torch.zeros(2, 2, 64, dtype=torch.bfloat16)):
+        with pytest.raises(ValueError, match=r"^k must be \[num_seqs, num_kv_heads, head_dim\]"):
+            P.decode_step(q, k, kv, kc, kc, i32(2, 3), i32(2), 0.1)
 
 
 def _header_text():
