@@ -312,7 +312,9 @@ pa_status pa_decode(const void* q, const void* key_cache, const void* value_cach
  *                 max_blocks_per_seq, cache) bytes, as for pa_decode
  *   other arguments as for pa_decode.
  * Returns what pa_decode returns for the same arguments, and PA_ERR_INVALID_ARG
- * for a NULL or misaligned k or v.  Nothing is written on a non-zero status.
+ * for a NULL or misaligned k or v.  A status found on the host (every one but
+ * PA_ERR_CUDA) launches nothing, so the pools are left as they were; after
+ * PA_ERR_CUDA the launches before the failing one may have run.
  */
 pa_status pa_decode_step(const void* q, const void* k, const void* v, void* key_cache,
                          void* value_cache, const int32_t* block_tables, const int32_t* seq_lens,
